@@ -1,0 +1,200 @@
+/*
+ * bitnet.h -- C ABI of the sm_100a W1.58A8 BitLinear library.
+ *
+ * The library computes the BitNet b1.58 BitLinear forward pass: ternary
+ * {-1,0,+1} weights stored 2 bits each, int8 activations, an int32 matmul
+ * and an fp32 dequantisation stored as bf16, plus the fused FFN block built
+ * from it.  Sources of each operation are cited per entry point by page and
+ * section:
+ *   [Y]  youngju.dev, "BitNet論文分析：1-Bit LLMの時代 — 三値重みからCPU推論まで"
+ *   [D]  dashen-tech.com, "BitNet.cpp 深度解析：1-bit LLM 推論、CPU 上で 100B
+ *        モデルを 6 倍高速実行"
+ *   [A]  abeam.tech, review of "BitNet: 1-bit Pre-training for Large Language
+ *        Models" (JMLR 2025)
+ *   [R]  reinforz.co.jp, news article on "BitNet b1.58 2B4T"
+ *
+ * Conventions shared by every entry point
+ *   - All array pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or synchronises inside these calls.  Scratch
+ *     memory, where needed, is a caller-provided device workspace whose size
+ *     comes from the matching *_workspace_size() function.
+ *   - bf16 values are passed as their raw 16-bit patterns (uint16_t).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously on it.  Kernels that only read
+ *     weights before their first dependency are launched with programmatic
+ *     dependent launch, so back-to-back calls overlap their weight streaming.
+ *   - Row-major layouts: x [M,K], y [M,N], W [N,K] (out x in, like
+ *     nn.Linear), packed [N, K/4].
+ *   - Arguments are validated on the host before anything is launched; a
+ *     non-OK status means nothing was enqueued.  Launch failures return
+ *     BITNET_ERR_CUDA.  Device-side conditions (a bounded wait that expired,
+ *     a non-finite weight) are recorded in a per-device status word that
+ *     bitnet_last_device_status() reports.
+ *   - Pointers to x, y, packed and the workspace must be 16-byte aligned.
+ */
+#ifndef BITNET_B200_H_
+#define BITNET_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BITNET_API __attribute__((visibility("default")))
+#else
+#define BITNET_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BITNET_OK = 0,
+  BITNET_ERR_INVALID_ARG = 1,  /* null pointer where one is required, eps < 0 */
+  BITNET_ERR_SHAPE = 2,        /* M, N or K out of range, K % 4 != 0          */
+  BITNET_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned            */
+  BITNET_ERR_WORKSPACE = 4,    /* workspace null or smaller than required     */
+  BITNET_ERR_UNSUPPORTED = 5,  /* device is not sm_100 / feature unavailable  */
+  BITNET_ERR_CUDA = 6,         /* a CUDA runtime call failed                  */
+  BITNET_ERR_TIMEOUT = 7,      /* a device-side bounded wait gave up          */
+  BITNET_ERR_NONFINITE = 8     /* a weight was Inf or NaN (gamma set to NaN)  */
+} bitnet_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+BITNET_API const char* bitnet_status_string(int status);
+
+/* Library ABI version: 100 * major + minor. */
+BITNET_API int bitnet_version(void);
+
+/*
+ * Absmean ternary weight quantisation + I2_S 2-bit packing.
+ *   [Y] section "Absmean量子化関数" (weight_quant_ternary: gamma = mean|W|,
+ *       W_q = clamp(round(W / (gamma + 1e-5)), -1, 1));
+ *   [Y] section "アーキテクチャ概要" (I2_S: 00 = -1, 01 = 0, 10 = +1,
+ *       16 weights per 32-bit register); [D] section "2.3 I2_S 形式".
+ *
+ * W       [N,K] fp32, device, read only.  Must be finite.
+ * packed  [N,K/4] uint8, device, written.  Weight k of row n is code
+ *         (W_q + 1) at bits 2*(k%4) of byte n*K/4 + k/4 (LSB first).
+ *         Code 3 is never produced.
+ * gamma   one fp32 on the device, written: the fp32 value nearest (ties to
+ *         even) to the exact mean of |W| (independent of summation order).
+ *         The ternary threshold divides by gamma + 1e-5 (fp32 add, IEEE
+ *         division per element, round half to even); dequantisation later
+ *         multiplies by gamma itself.
+ * workspace  >= bitnet_pack_workspace_size(N, K) bytes of device memory; its
+ *         contents are overwritten.
+ * Requires K % 4 == 0, N >= 1, K >= 4, N*K < 2^39.  A non-finite weight sets
+ * gamma to NaN and records BITNET_ERR_NONFINITE in the device status word.
+ * Not performance-critical (run once per weight matrix).
+ */
+BITNET_API size_t bitnet_pack_workspace_size(int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_pack_weights(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                                  float* gamma, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/*
+ * Per-token absmax int8 activation quantisation.
+ *   [Y] section "Absmean量子化関数" (BitLinear_b158.activation_quant, per
+ *       token absmax with rounding and clamping); [R] section
+ *       "積極的量子化と三値化がもたらす学習効率の革新" (absmax, 8-bit, W1.58A8).
+ *
+ * s_t = 127 / max(max_k |x[t,k]|, 1e-5)          (fp32, IEEE division)
+ * xq[t,k] = clamp(rint(x[t,k] * s_t), -128, 127)  (one fp32 multiply)
+ * x       [M,K] bf16 bits, device.        xq   [M,K] int8, device, written.
+ * scale   [M] fp32, device, written (s_t).
+ * rowsum  [M] int32, device, written with sum_k xq[t,k]; may be NULL.
+ * Requires M >= 1, K >= 1, K % 4 == 0.
+ */
+BITNET_API bitnet_status bitnet_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq,
+                               float* scale, int32_t* rowsum, void* stream);
+
+/*
+ * BitLinear forward: y = dequant(quant(x) . W_q^T).
+ *   [D] section "3.1 計算コア：整数行列乗算" (Y = sum_pos - sum_neg, no
+ *       multiplications); [Y] section "Absmean量子化関数" (BitLinear_b158.forward:
+ *       F.linear on the quantised operands, then the scale restore).
+ *
+ * acc[t,n] = sum_k xq[t,k] * W_q[n,k]   (exact int32)
+ * d_t      = gamma / s_t                (fp32 division, once per token)
+ * y32      = fp32(acc) * d_t            (one fp32 multiply)
+ * y[t,n]   = bf16(y32), round to nearest even.
+ * No bias, no normalisation (the caller applies any norm).
+ *
+ * packed  [N,K/4] from bitnet_pack_weights.   gamma  device fp32 scalar.
+ * x       [M,K] bf16 bits.   y  [M,N] bf16 bits, written.
+ * y_f32   [M,N] fp32, written with y32 when non-NULL (debug / parity).
+ * acc     [M,N] int32, written with the exact accumulators when non-NULL.
+ * workspace  >= bitnet_linear_workspace_size(M, N, K) bytes (0 bytes, and a
+ *         NULL workspace, are accepted when that size is 0).
+ * Requires M >= 1, N >= 1, K >= 4, K % 4 == 0, K <= 524288.  M <= 8 with
+ * K % 64 == 0 runs the fused decode kernel (activation quantisation in its
+ * prologue, no workspace); larger M runs the tensor-core kernel.
+ */
+BITNET_API size_t bitnet_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N, int64_t K,
+                            const uint16_t* x, int64_t M, uint16_t* y, float* y_f32,
+                            int32_t* acc, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
+ * Optional intermediate outputs of bitnet_ffn, for parity checking.  Every
+ * member may be NULL.  Shapes: xq1 [M,H], acc_gate/acc_up [M,I], h [M,I]
+ * (the folded h' below), xq2 [M,I], acc_down [M,H], y_f32 [M,H].
+ */
+typedef struct {
+  int8_t* xq1;
+  int32_t* acc_gate;
+  int32_t* acc_up;
+  float* h;
+  int8_t* xq2;
+  int32_t* acc_down;
+  float* y_f32;
+} bitnet_ffn_debug;
+
+/*
+ * Fused BitNet FFN block:
+ *   RMSNorm(n1) -> act quant -> gate, up BitLinear -> ReLU(gate)^2 * up
+ *   -> RMSNorm(n2) -> act quant -> down BitLinear.   No residual.
+ *   [A] sections "モデル構造" (LLaMA-like FFN with RMSNorm) and
+ *       "正規化で分散を安定させる" (normalise before BitLinear, subln);
+ *   [R] section "BitNetが実現したCPU上での高効率AI処理" (ReLU^2);
+ *   [Y] section "Absmean量子化関数" (RMSNorm before the activation quantiser).
+ *
+ * Folded evaluation (absmax quantisation ignores a positive per-token scale):
+ *   r1 = 1/sqrt(mean(x^2) + eps);  u = x * n1;  xq1 = quant(u), s1
+ *   g' = fp32(acc_gate) * (gamma_gate / s1);  u' = fp32(acc_up) * (gamma_up / s1)
+ *   h' = (relu(g') * relu(g')) * u';  v = h' * n2;  xq2 = quant(v), s2
+ *   r2 = 1/sqrt(r1^6 * mean(h'^2) + eps)
+ *   y32 = (fp32(acc_down) * (gamma_down / s2)) * (r1^3 * r2);  y = bf16(y32)
+ * Every quantised code and integer accumulator is exact; the r factors are
+ * reductions whose rounding order is unspecified (y32 within 1e-5 relative).
+ *
+ * x [M,H] bf16 bits.  gate, up: packed [I, H/4]; down: packed [H, I/4];
+ * gamma_* device fp32 scalars.  norm1_w [H], norm2_w [I] fp32 gains, NULL
+ * means all ones.  eps >= 0.  y [M,H] bf16 bits written.
+ * workspace >= bitnet_ffn_workspace_size(M, H, I) bytes.
+ * debug  NULL or a host struct of optional device outputs (see above).
+ * Requires M >= 1, H % 64 == 0, I % 64 == 0, H, I >= 64.
+ */
+BITNET_API size_t bitnet_ffn_workspace_size(int64_t M, int64_t H, int64_t I);
+BITNET_API bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
+                         const float* norm1_w, const uint8_t* gate, const float* gamma_gate,
+                         const uint8_t* up, const float* gamma_up, const float* norm2_w,
+                         const uint8_t* down, const float* gamma_down, float eps,
+                         uint16_t* y, const bitnet_ffn_debug* debug, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, then return and clear the device status word of the
+ * current device: BITNET_OK, BITNET_ERR_TIMEOUT (a bounded wait expired; the
+ * affected outputs are unspecified) or BITNET_ERR_NONFINITE.  A failing
+ * synchronisation returns BITNET_ERR_CUDA.
+ */
+BITNET_API bitnet_status bitnet_last_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET_B200_H_ */

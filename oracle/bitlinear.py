@@ -159,13 +159,18 @@ def absmean_gamma(W: np.ndarray) -> np.float32:
     exp = (bits >> np.uint32(23)) & np.uint32(0xFF)
     if np.any(exp == 0xFF):
         raise ValueError("non-finite weight")
-    man = (bits & np.uint32(0x7FFFFF)).astype(np.uint64)
-    man = np.where(exp > 0, man | np.uint64(0x800000), man)
-    eb = np.maximum(exp, np.uint32(1)).astype(np.int64)
     total = 0                              # exact sum, in units of 2^-149
-    for e in np.unique(eb):
-        msum = int(man[eb == e].sum(dtype=np.uint64))
-        total += msum << int(e - 1)
+    chunk = 1 << 26
+    for c0 in range(0, count, chunk):
+        b = bits[c0:c0 + chunk]
+        e = exp[c0:c0 + chunk]
+        man = (b & np.uint32(0x7FFFFF)) | np.where(e > 0, np.uint32(0x800000), np.uint32(0))
+        eb = np.maximum(e, np.uint32(1))
+        # per-exponent mantissa sums: every partial sum is an integer below
+        # 2^26 * 2^24 = 2^50, so the float64 accumulation is exact
+        sums = np.bincount(eb, weights=man.astype(np.float64), minlength=256)
+        for k in np.flatnonzero(sums):
+            total += int(sums[k]) << int(k - 1)
     return round_rational_to_f32(total, count << 149)
 
 
@@ -212,16 +217,19 @@ def pack_weights(W: np.ndarray):
 def ternary_matmul(xq: np.ndarray, w: np.ndarray) -> np.ndarray:
     """acc[m, n] = sum_k x_q[m, k] * w[n, k], exact, int64 [M, N].
 
-    A float64 matrix product is used as a library step: every product and
-    every partial sum is an integer below 2^53, so any summation order gives
-    the exact integer result.
+    A floating-point matrix product is used as a library step: every product
+    and every partial sum is an integer of magnitude at most 128*K, below
+    2^24 (fp32) or 2^53 (fp64), so any summation order gives the exact
+    integer result.
     """
     xq = np.asarray(xq, dtype=np.int8)
     w = np.asarray(w, dtype=np.int8)
     K = xq.shape[1]
-    if 127 * K >= 2 ** 53:
-        raise ValueError("K too large for the exact fp64 product")
-    acc = xq.astype(np.float64) @ w.astype(np.float64).T
+    if 128 * K >= 2 ** 53:
+        raise ValueError("K too large for an exact floating-point product")
+    # fp32 when every partial sum is an integer below 2^24 (then also exact)
+    ft = np.float32 if 128 * K < 2 ** 24 else np.float64
+    acc = xq.astype(ft) @ w.astype(ft).T
     return acc.astype(np.int64)
 
 

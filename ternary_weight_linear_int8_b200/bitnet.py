@@ -1,0 +1,223 @@
+"""Thin Python binding of the C ABI in include/bitnet.h.
+
+Argument marshalling only: PyTorch provides device memory and the current
+stream; every step of the computation runs in the library's CUDA kernels.
+The binding refuses to run when the shared library is missing (there is no
+fallback of any kind).
+
+Function names match the C entry points.  Tensors must live on the CUDA
+device; bf16 arrays may be passed as torch.bfloat16 or as 16-bit integer
+tensors holding the bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitnet_b200.so")
+
+STATUS = {
+    0: "BITNET_OK", 1: "BITNET_ERR_INVALID_ARG", 2: "BITNET_ERR_SHAPE", 3: "BITNET_ERR_ALIGN",
+    4: "BITNET_ERR_WORKSPACE", 5: "BITNET_ERR_UNSUPPORTED", 6: "BITNET_ERR_CUDA",
+    7: "BITNET_ERR_TIMEOUT", 8: "BITNET_ERR_NONFINITE",
+}
+
+# name -> (restype, argtypes)
+_P, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+SIGNATURES = {
+    "bitnet_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "bitnet_version": (ctypes.c_int, []),
+    "bitnet_pack_workspace_size": (_SZ, [_I64, _I64]),
+    "bitnet_pack_weights": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
+    "bitnet_quant_act": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "bitnet_linear_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "bitnet_linear": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I64, _P, _P, _P, _P, _SZ, _P]),
+    "bitnet_ffn_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "bitnet_ffn": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _F,
+                                  _P, _P, _P, _SZ, _P]),
+    "bitnet_last_device_status": (ctypes.c_int, [_P]),
+}
+
+
+class FfnDebug(ctypes.Structure):
+    _fields_ = [("xq1", _P), ("acc_gate", _P), ("acc_up", _P), ("h", _P), ("xq2", _P),
+                ("acc_down", _P), ("y_f32", _P)]
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, func: str, status: int):
+        super().__init__(f"{func} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "ternary_weight_linear_int8_b200/build.py (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(name, st):
+    if st != 0:
+        raise BitnetError(name, st)
+
+
+def _dev(t, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _bits16(t, name):
+    _dev(t, name)
+    if t.element_size() != 2:
+        raise ValueError(f"{name} must hold 16-bit (bf16) elements")
+    return t
+
+
+def _workspace(nbytes, device, ws=None):
+    if nbytes == 0:
+        return None
+    if ws is not None and ws.numel() * ws.element_size() >= nbytes:
+        return ws
+    return torch.empty(int(nbytes), dtype=torch.uint8, device=device)
+
+
+def bitnet_status_string(status: int) -> str:
+    return lib().bitnet_status_string(status).decode()
+
+
+def bitnet_version() -> int:
+    return lib().bitnet_version()
+
+
+def bitnet_pack_weights(W: torch.Tensor, packed=None, gamma=None, workspace=None):
+    """W fp32 [N,K] -> (packed uint8 [N,K/4], gamma fp32 [1])."""
+    _dev(W, "W")
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float32 tensor")
+    N, K = W.shape
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device) if packed is None else packed
+    gamma = torch.empty(1, dtype=torch.float32, device=W.device) if gamma is None else gamma
+    nb = lib().bitnet_pack_workspace_size(N, K)
+    ws = _workspace(nb, W.device, workspace)
+    st = lib().bitnet_pack_weights(_ptr(W), N, K, _ptr(packed), _ptr(gamma), _ptr(ws), nb, _stream())
+    _check("bitnet_pack_weights", st)
+    return packed, gamma
+
+
+def bitnet_quant_act(x: torch.Tensor, with_rowsum: bool = True):
+    """x bf16 [M,K] -> (x_q int8 [M,K], scale fp32 [M], rowsum int32 [M] or None)."""
+    _bits16(x, "x")
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s = torch.empty(M, dtype=torch.float32, device=x.device)
+    rs = torch.empty(M, dtype=torch.int32, device=x.device) if with_rowsum else None
+    st = lib().bitnet_quant_act(_ptr(x), M, K, _ptr(xq), _ptr(s), _ptr(rs), _stream())
+    _check("bitnet_quant_act", st)
+    return xq, s, rs
+
+
+def bitnet_linear_workspace_size(M: int, N: int, K: int) -> int:
+    return lib().bitnet_linear_workspace_size(M, N, K)
+
+
+def bitnet_linear(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, y=None,
+                  want_f32: bool = False, want_acc: bool = False, workspace=None):
+    """y = BitLinear(x) on packed weights.  Returns (y bf16 [M,N], y_f32, acc)."""
+    _dev(packed, "packed")
+    _dev(gamma, "gamma")
+    _bits16(x, "x")
+    N, Kb = packed.shape
+    M, K = x.shape
+    if K != 4 * Kb:
+        raise ValueError("x and packed disagree on K")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    y32 = torch.empty((M, N), dtype=torch.float32, device=x.device) if want_f32 else None
+    acc = torch.empty((M, N), dtype=torch.int32, device=x.device) if want_acc else None
+    nb = lib().bitnet_linear_workspace_size(M, N, K)
+    ws = _workspace(nb, x.device, workspace)
+    st = lib().bitnet_linear(_ptr(packed), _ptr(gamma), N, K, _ptr(x), M, _ptr(y), _ptr(y32),
+                             _ptr(acc), _ptr(ws), nb, _stream())
+    _check("bitnet_linear", st)
+    return y, y32, acc
+
+
+def bitnet_ffn_workspace_size(M: int, H: int, I: int) -> int:
+    return lib().bitnet_ffn_workspace_size(M, H, I)
+
+
+@dataclass
+class FfnWeights:
+    gate: torch.Tensor
+    gamma_gate: torch.Tensor
+    up: torch.Tensor
+    gamma_up: torch.Tensor
+    down: torch.Tensor
+    gamma_down: torch.Tensor
+    norm1_w: torch.Tensor | None = None
+    norm2_w: torch.Tensor | None = None
+
+
+def bitnet_ffn(x: torch.Tensor, w: FfnWeights, eps: float = 1e-5, y=None, debug: bool = False,
+               workspace=None):
+    """Fused FFN block.  Returns (y bf16 [M,H], dict of debug outputs or None)."""
+    _bits16(x, "x")
+    M, H = x.shape
+    I = w.gate.shape[0]
+    dev = x.device
+    y = torch.empty((M, H), dtype=torch.bfloat16, device=dev) if y is None else y
+    dbg = None
+    dstruct = None
+    if debug:
+        dbg = {
+            "xq1": torch.empty((M, H), dtype=torch.int8, device=dev),
+            "acc_gate": torch.empty((M, I), dtype=torch.int32, device=dev),
+            "acc_up": torch.empty((M, I), dtype=torch.int32, device=dev),
+            "h": torch.empty((M, I), dtype=torch.float32, device=dev),
+            "xq2": torch.empty((M, I), dtype=torch.int8, device=dev),
+            "acc_down": torch.empty((M, H), dtype=torch.int32, device=dev),
+            "y_f32": torch.empty((M, H), dtype=torch.float32, device=dev),
+        }
+        dstruct = FfnDebug(*[_ptr(dbg[k]) for k in
+                             ("xq1", "acc_gate", "acc_up", "h", "xq2", "acc_down", "y_f32")])
+    nb = lib().bitnet_ffn_workspace_size(M, H, I)
+    ws = _workspace(nb, dev, workspace)
+    st = lib().bitnet_ffn(_ptr(x), M, H, I, _ptr(w.norm1_w), _ptr(w.gate), _ptr(w.gamma_gate),
+                          _ptr(w.up), _ptr(w.gamma_up), _ptr(w.norm2_w), _ptr(w.down),
+                          _ptr(w.gamma_down), float(eps), _ptr(y),
+                          ctypes.byref(dstruct) if dstruct is not None else None,
+                          _ptr(ws), nb, _stream())
+    _check("bitnet_ffn", st)
+    return y, dbg
+
+
+def bitnet_last_device_status() -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    return lib().bitnet_last_device_status(_stream())

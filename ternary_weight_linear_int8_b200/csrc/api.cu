@@ -1,0 +1,371 @@
+// C ABI of the library: argument validation, planning (which kernel, how
+// much workspace) and dispatch.  Declarations and the contract of every entry
+// point are in include/bitnet.h.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+using namespace bitnet;
+
+// Defined in the kernel sources of this translation unit.
+size_t bitnet_pack_workspace_size_impl();
+bitnet_status bitnet_pack_launch(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                                 float* gamma, void* workspace, cudaStream_t stream, int num_sms);
+bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* gain, int64_t M,
+                                  int64_t K, int8_t* xq, int64_t ld_q, bool perm, float* scale,
+                                  int32_t* rowsum, double* sumsq, int8_t* xq_natural,
+                                  cudaStream_t stream);
+bitnet_status bitnet_gemv_launch(int mode, GemvArgs a, int num_sms, cudaStream_t stream);
+bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
+                                 const uint8_t* w1, GemmArgs a, int bn, cudaStream_t stream);
+int bitnet_gemm_pick_bn(int M);
+
+namespace {
+
+// Ragged K (K % 64 != 0): one thread per output, natural-layout x_q.
+__global__ void __launch_bounds__(256) generic_linear_kernel(const uint8_t* __restrict__ packed,
+                                                             const float* __restrict__ gamma,
+                                                             int N, int K, int M,
+                                                             const int8_t* __restrict__ xq,
+                                                             const float* __restrict__ scale,
+                                                             uint16_t* y, float* y_f32,
+                                                             int32_t* acc_out) {
+  pdl_wait();
+  const int64_t total = (int64_t)M * N;
+  for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < total;
+       o += (int64_t)gridDim.x * blockDim.x) {
+    const int m = (int)(o / N), n = (int)(o % N);
+    const uint8_t* row = packed + (int64_t)n * (K / 4);
+    const int8_t* xr = xq + (int64_t)m * K;
+    int acc = 0;
+    for (int k = 0; k < K; ++k) {
+      const int code = (row[k >> 2] >> (2 * (k & 3))) & 3;
+      acc += (int)xr[k] * (code - 1);
+    }
+    const float y32 = __fmul_rn(__int2float_rn(acc), __fdiv_rn(*gamma, scale[m]));
+    y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+    if (y_f32) y_f32[o] = y32;
+    if (acc_out) acc_out[o] = acc;
+  }
+}
+
+struct DevInfo {
+  int num_sms = 0;
+  int major = 0;
+};
+
+bitnet_status device_info(DevInfo* out) {
+  static DevInfo cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BITNET_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return BITNET_ERR_UNSUPPORTED;
+  if (cache[dev].num_sms == 0) {
+    DevInfo d;
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return BITNET_ERR_CUDA;
+    cache[dev] = d;
+  }
+  *out = cache[dev];
+  if (out->major != 10) return BITNET_ERR_UNSUPPORTED;
+  return BITNET_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t al256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// Which kernel serves bitnet_linear for this shape.
+enum LinearPath { kPathGemv = 0, kPathGemm = 1, kPathGeneric = 2 };
+
+int gemv_mpad(int64_t M) {
+  const int64_t MT = M == 1 ? 1 : (M == 2 ? 2 : 4);
+  return (int)(((M + MT - 1) / MT) * MT);
+}
+
+bool gemv_fits(int64_t M, int64_t K) {
+  return M <= 8 && K % 64 == 0 && (int64_t)gemv_mpad(M) * K <= 65536;
+}
+
+LinearPath linear_path(int64_t M, int64_t K) {
+  if (K % 64 != 0) return kPathGeneric;
+  if (gemv_fits(M, K)) return kPathGemv;
+  return kPathGemm;
+}
+
+// Split K over CTAs when the tile grid would leave most SMs idle.
+int plan_ksplit(int64_t M, int64_t N, int64_t K, int bn, int num_sms) {
+  if (M > 256) return 1;
+  const int64_t tiles = ((N + 127) / 128) * ((M + bn - 1) / bn);
+  const int64_t kst = (K + 127) / 128;
+  if (tiles * 2 > num_sms) return 1;
+  int64_t ks = num_sms / tiles;
+  if (ks > 8) ks = 8;
+  if (ks > kst / 2) ks = kst / 2;
+  return ks < 1 ? 1 : (int)ks;
+}
+
+struct LinearWs {
+  size_t xq, scale, rowsum, acc, total;
+};
+
+LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
+  LinearWs w{};
+  const LinearPath p = linear_path(M, K);
+  if (p == kPathGemv) return w;
+  w.xq = 0;
+  w.scale = al256((size_t)M * K);
+  w.rowsum = w.scale + al256((size_t)M * 4);
+  w.acc = w.rowsum + al256((size_t)M * 4);
+  w.total = w.acc;
+  // split-K accumulators are reserved for every small-M tensor-core shape
+  if (p == kPathGemm && M <= 256) w.total = w.acc + al256((size_t)M * N * 4);
+  return w;
+}
+
+struct FfnWs {
+  bool gemv;
+  size_t h, xq1, s1, rs1, ss1, xq2, s2, rs2, ss2, acc0, acc1, total;
+};
+
+FfnWs ffn_ws_layout(int64_t M, int64_t H, int64_t I) {
+  FfnWs w{};
+  w.gemv = gemv_fits(M, H) && gemv_fits(M, I);
+  size_t off = 0;
+  w.h = off;
+  off += al256((size_t)M * I * 4);
+  if (!w.gemv) {
+    w.xq1 = off; off += al256((size_t)M * H);
+    w.s1 = off; off += al256((size_t)M * 4);
+    w.rs1 = off; off += al256((size_t)M * 4);
+    w.ss1 = off; off += al256((size_t)M * 8);
+    w.xq2 = off; off += al256((size_t)M * I);
+    w.s2 = off; off += al256((size_t)M * 4);
+    w.rs2 = off; off += al256((size_t)M * 4);
+    w.ss2 = off; off += al256((size_t)M * 8);
+    if (M <= 256) {   // split-K accumulators: gate (and later down), up
+      w.acc0 = off; off += al256((size_t)M * (H > I ? H : I) * 4);
+      w.acc1 = off; off += al256((size_t)M * I * 4);
+    }
+  }
+  w.total = off;
+  return w;
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+extern "C" {
+
+const char* bitnet_status_string(int status) {
+  switch (status) {
+    case BITNET_OK: return "BITNET_OK";
+    case BITNET_ERR_INVALID_ARG: return "BITNET_ERR_INVALID_ARG";
+    case BITNET_ERR_SHAPE: return "BITNET_ERR_SHAPE";
+    case BITNET_ERR_ALIGN: return "BITNET_ERR_ALIGN";
+    case BITNET_ERR_WORKSPACE: return "BITNET_ERR_WORKSPACE";
+    case BITNET_ERR_UNSUPPORTED: return "BITNET_ERR_UNSUPPORTED";
+    case BITNET_ERR_CUDA: return "BITNET_ERR_CUDA";
+    case BITNET_ERR_TIMEOUT: return "BITNET_ERR_TIMEOUT";
+    case BITNET_ERR_NONFINITE: return "BITNET_ERR_NONFINITE";
+    default: return "BITNET_ERR_UNKNOWN";
+  }
+}
+
+int bitnet_version(void) { return 100; }
+
+size_t bitnet_pack_workspace_size(int64_t N, int64_t K) {
+  (void)N;
+  (void)K;
+  return bitnet_pack_workspace_size_impl();
+}
+
+bitnet_status bitnet_pack_weights(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                                  float* gamma, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (!W || !packed || !gamma) return BITNET_ERR_INVALID_ARG;
+  if (N < 1 || K < 4 || K % 4 != 0 || N > (int64_t(1) << 39) / K) return BITNET_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(packed) || ((uintptr_t)gamma & 3u)) return BITNET_ERR_ALIGN;
+  if (!workspace || workspace_bytes < bitnet_pack_workspace_size(N, K))
+    return BITNET_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  return bitnet_pack_launch(W, N, K, packed, gamma, workspace, as_stream(stream), d.num_sms);
+}
+
+bitnet_status bitnet_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* scale,
+                               int32_t* rowsum, void* stream) {
+  if (!x || !xq || !scale) return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || K < 4 || K % 4 != 0 || M > 0x7fffffff || K > (int64_t(1) << 31))
+    return BITNET_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(xq) || ((uintptr_t)scale & 3u) || ((uintptr_t)rowsum & 3u))
+    return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  return bitnet_quant_launch(x, false, nullptr, M, K, xq, K, false, scale, rowsum, nullptr,
+                             nullptr, as_stream(stream));
+}
+
+size_t bitnet_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 4) return 0;
+  return linear_ws_layout(M, N, K).total;
+}
+
+bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N, int64_t K,
+                            const uint16_t* x, int64_t M, uint16_t* y, float* y_f32,
+                            int32_t* acc, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (!packed || !gamma || !x || !y) return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 4 || K % 4 != 0 || K > 524288 || M > 0x7fffffff || N > 0x7fffffff)
+    return BITNET_ERR_SHAPE;
+  if (!aligned16(packed) || !aligned16(x) || !aligned16(y) || ((uintptr_t)gamma & 3u) ||
+      ((uintptr_t)y_f32 & 3u) || ((uintptr_t)acc & 3u))
+    return BITNET_ERR_ALIGN;
+  const LinearWs L = linear_ws_layout(M, N, K);
+  if (L.total > 0) {
+    if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  }
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  const LinearPath p = linear_path(M, K);
+  if (p == kPathGemv) {
+    GemvArgs a{};
+    a.w0 = packed; a.gamma0 = gamma;
+    a.N = (int)N; a.K = (int)K; a.M = (int)M;
+    a.x = x;
+    a.y = y; a.y_f32 = y_f32; a.acc0 = acc;
+    return bitnet_gemv_launch(kLinear, a, d.num_sms, s);
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + L.xq);
+  float* sc = reinterpret_cast<float*>(ws + L.scale);
+  int32_t* rs = reinterpret_cast<int32_t*>(ws + L.rowsum);
+  if (p == kPathGeneric) {
+    st = bitnet_quant_launch(x, false, nullptr, M, K, xq, K, false, sc, rs, nullptr, nullptr, s);
+    if (st != BITNET_OK) return st;
+    int64_t blocks = (M * N + 255) / 256;
+    if (blocks > (int64_t)d.num_sms * 16) blocks = (int64_t)d.num_sms * 16;
+    generic_linear_kernel<<<(unsigned)blocks, 256, 0, s>>>(packed, gamma, (int)N, (int)K, (int)M,
+                                                          xq, sc, y, y_f32, acc);
+    return cudaGetLastError() == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+  }
+  st = bitnet_quant_launch(x, false, nullptr, M, K, xq, K, true, sc, rs, nullptr, nullptr, s);
+  if (st != BITNET_OK) return st;
+  const int bn = bitnet_gemm_pick_bn((int)M);
+  GemmArgs a{};
+  a.M = (int)M; a.N = (int)N; a.K = (int)K;
+  a.ksplit = plan_ksplit(M, N, K, bn, d.num_sms);
+  a.scale = sc; a.rowsum = rs; a.gamma0 = gamma;
+  a.y = y; a.y_f32 = y_f32; a.acc0 = acc;
+  if (a.ksplit > 1) {
+    a.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc);
+    if (cudaMemsetAsync(a.acc_ws0, 0, (size_t)M * N * 4, s) != cudaSuccess) return BITNET_ERR_CUDA;
+  }
+  return bitnet_gemm_launch(0 /*linear*/, xq, packed, nullptr, a, bn, s);
+}
+
+size_t bitnet_ffn_workspace_size(int64_t M, int64_t H, int64_t I) {
+  if (M < 1 || H < 1 || I < 1) return 0;
+  return ffn_ws_layout(M, H, I).total;
+}
+
+bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
+                         const float* norm1_w, const uint8_t* gate, const float* gamma_gate,
+                         const uint8_t* up, const float* gamma_up, const float* norm2_w,
+                         const uint8_t* down, const float* gamma_down, float eps, uint16_t* y,
+                         const bitnet_ffn_debug* debug, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  if (!x || !gate || !gamma_gate || !up || !gamma_up || !down || !gamma_down || !y)
+    return BITNET_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !(eps < 3.0e38f)) return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || H < 64 || I < 64 || H % 64 != 0 || I % 64 != 0 || H > 524288 || I > 524288 ||
+      M > 0x7fffffff)
+    return BITNET_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(gate) || !aligned16(up) || !aligned16(down))
+    return BITNET_ERR_ALIGN;
+  const FfnWs L = ffn_ws_layout(M, H, I);
+  if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  bitnet_ffn_debug dbg{};
+  if (debug) dbg = *debug;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* h = reinterpret_cast<float*>(ws + L.h);
+  if (L.gemv) {
+    GemvArgs g{};
+    g.w0 = gate; g.gamma0 = gamma_gate; g.w1 = up; g.gamma1 = gamma_up;
+    g.N = (int)I; g.K = (int)H; g.M = (int)M;
+    g.x = x; g.gain = norm1_w;
+    g.h = dbg.h ? dbg.h : h;
+    g.acc0 = dbg.acc_gate; g.acc1 = dbg.acc_up; g.xq_dbg = dbg.xq1;
+    st = bitnet_gemv_launch(kGlu, g, d.num_sms, s);
+    if (st != BITNET_OK) return st;
+    GemvArgs dn{};
+    dn.w0 = down; dn.gamma0 = gamma_down;
+    dn.N = (int)H; dn.K = (int)I; dn.M = (int)M;
+    dn.x = g.h; dn.gain = norm2_w; dn.xnorm = x; dn.H = (int)H; dn.eps = eps;
+    dn.y = y; dn.y_f32 = dbg.y_f32; dn.acc0 = dbg.acc_down; dn.xq_dbg = dbg.xq2;
+    return bitnet_gemv_launch(kDown, dn, d.num_sms, s);
+  }
+  int8_t* xq1 = reinterpret_cast<int8_t*>(ws + L.xq1);
+  float* s1 = reinterpret_cast<float*>(ws + L.s1);
+  int32_t* rs1 = reinterpret_cast<int32_t*>(ws + L.rs1);
+  double* ss1 = reinterpret_cast<double*>(ws + L.ss1);
+  int8_t* xq2 = reinterpret_cast<int8_t*>(ws + L.xq2);
+  float* s2 = reinterpret_cast<float*>(ws + L.s2);
+  int32_t* rs2 = reinterpret_cast<int32_t*>(ws + L.rs2);
+  double* ss2 = reinterpret_cast<double*>(ws + L.ss2);
+  float* hbuf = dbg.h ? dbg.h : h;
+  st = bitnet_quant_launch(x, false, norm1_w, M, H, xq1, H, true, s1, rs1, ss1, dbg.xq1, s);
+  if (st != BITNET_OK) return st;
+  const int bn = bitnet_gemm_pick_bn((int)M);
+  GemmArgs g{};
+  g.M = (int)M; g.N = (int)I; g.K = (int)H;
+  g.ksplit = plan_ksplit(M, I, H, bn, d.num_sms);
+  g.scale = s1; g.rowsum = rs1; g.gamma0 = gamma_gate; g.gamma1 = gamma_up;
+  g.h = hbuf; g.acc0 = dbg.acc_gate; g.acc1 = dbg.acc_up;
+  if (g.ksplit > 1) {
+    g.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
+    g.acc_ws1 = reinterpret_cast<int32_t*>(ws + L.acc1);
+    if (cudaMemsetAsync(g.acc_ws0, 0, (size_t)M * I * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(g.acc_ws1, 0, (size_t)M * I * 4, s) != cudaSuccess)
+      return BITNET_ERR_CUDA;
+  }
+  st = bitnet_gemm_launch(1 /*glu*/, xq1, gate, up, g, bn, s);
+  if (st != BITNET_OK) return st;
+  st = bitnet_quant_launch(hbuf, true, norm2_w, M, I, xq2, I, true, s2, rs2, ss2, dbg.xq2, s);
+  if (st != BITNET_OK) return st;
+  GemmArgs dn{};
+  dn.M = (int)M; dn.N = (int)H; dn.K = (int)I;
+  dn.ksplit = plan_ksplit(M, H, I, bn, d.num_sms);
+  dn.scale = s2; dn.rowsum = rs2; dn.gamma0 = gamma_down;
+  dn.sumsq_h = ss2; dn.sumsq_x = ss1; dn.H = (int)H; dn.eps = eps;
+  dn.y = y; dn.y_f32 = dbg.y_f32; dn.acc0 = dbg.acc_down;
+  if (dn.ksplit > 1) {
+    dn.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
+    if (cudaMemsetAsync(dn.acc_ws0, 0, (size_t)M * H * 4, s) != cudaSuccess) return BITNET_ERR_CUDA;
+  }
+  return bitnet_gemm_launch(2 /*down*/, xq2, down, nullptr, dn, bn, s);
+}
+
+bitnet_status bitnet_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return BITNET_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return BITNET_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return BITNET_ERR_CUDA;
+  }
+  return static_cast<bitnet_status>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,516 @@
+// Prefill / batched kernel: tcgen05 kind::i8 MMAs with TMEM accumulators.
+//
+// The matmul with ternary weights is an integer contraction (dashen-tech.com
+// "BitNet.cpp 深度解析", section "3.1 計算コア：整数行列乗算"); with many tokens it
+// is a dense one, so it runs on the 5th-generation tensor cores:
+//
+//   D[n, t] = sum_k code[n, k] * x_q[t, k]      (int8 x int8 -> int32, TMEM)
+//   acc     = D - sum_k x_q[t, k]               (code = w + 1, so this is sum w*x_q)
+//
+// Orientation: the MMA's M side (128 rows) is a tile of output features, its
+// N side (BN = 32..256 columns) a tile of tokens.  Per K-stage of 128:
+//   * warp 0 (one thread) issues TMA loads of the token tile of x_q (already in
+//     the kernels' permuted K order, 128B-swizzled) and of the packed 2-bit
+//     weight tile (128 rows x 32 bytes);
+//   * warps 2..5 unpack the packed tile to int8 codes {0,1,2} straight into
+//     the 128B-swizzled K-major layout the MMA descriptor expects: each packed
+//     32-bit word becomes the four code planes (w >> 2t) & 0x03030303, which
+//     is exactly the permuted order of x_q;
+//   * warp 1 (one thread) issues 4 MMAs of K = 32 per stage per weight matrix
+//     and commits completion to the stage's barrier;
+//   * after the last stage warps 2..5 read the accumulators out of TMEM
+//     (32 lanes x 32 columns per load) and apply the epilogue.
+// Every wait on a barrier is bounded (see mbar_wait).  TMA loads use no
+// cluster multicast.
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace bitnet {
+
+enum GemmMode : int { gLinear = 0, gGlu = 1, gDown = 2 };
+
+struct GemmArgs {
+  int M, N, K;
+  int ksplit;               // >1: accumulate D into acc_ws with integer atomics
+  const float* scale;       // [M] activation scales s
+  const int32_t* rowsum;    // [M] sum of x_q
+  const float* gamma0;
+  const float* gamma1;
+  const double* sumsq_h;    // Down: [M] sum of h'^2 over the inner dim (= K)
+  const double* sumsq_x;    // Down: [M] sum of x^2 over the block input
+  int H;                    // Down: width of the block input
+  float eps;
+  uint16_t* y;              // Linear/Down [M,N]
+  float* y_f32;             // optional [M,N]
+  int32_t* acc0;            // optional [M,N]
+  int32_t* acc1;            // optional [M,N] (Glu up)
+  float* h;                 // Glu [M,N]
+  int32_t* acc_ws0;         // split-K accumulators [M,N]
+  int32_t* acc_ws1;
+};
+
+constexpr int kBM = 128;                 // features per tile (MMA M)
+constexpr int kBK = 128;                 // K elements (bytes) per stage
+constexpr int kGemmThreads = 192;
+
+template <int BN, int NMAT>
+struct GemmCfg {
+  static constexpr int kB = BN * kBK;                 // x_q tile bytes
+  static constexpr int kA = kBM * kBK;                // one unpacked weight tile
+  static constexpr int kP = kBM * (kBK / 4);          // one packed weight tile
+  static constexpr int kStage = kB + NMAT * (kA + kP);
+  static constexpr int kStages0 = (220 * 1024) / kStage;
+  static constexpr int kStages = kStages0 > 6 ? 6 : (kStages0 < 2 ? 2 : kStages0);
+  static constexpr int kCols0 = NMAT * BN;
+  static constexpr int kTmemCols = kCols0 <= 32 ? 32 : kCols0 <= 64 ? 64 : kCols0 <= 128 ? 128
+                                 : kCols0 <= 256 ? 256 : 512;
+  static constexpr int kAux = 1024;                   // barriers + tmem slot
+  static constexpr int kTok = BN * 16;                // per-token scalars
+  static constexpr size_t kSmem = 1024 /*align slack*/ + (size_t)kStages * kStage + kAux + kTok;
+  // instruction descriptor: D s32, A s8, B s8, both K-major, N = BN, M = 128
+  static constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) |
+                                     ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+};
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3fffu);
+  d |= (uint64_t)1u << 16;                 // leading byte offset (unused for SW128 K-major)
+  d |= (uint64_t)(1024u >> 4) << 32;       // stride byte offset
+  d |= (uint64_t)1u << 46;                 // descriptor version (sm_100)
+  d |= (uint64_t)2u << 61;                 // 128-byte swizzle
+  return d;
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_mma_i8(uint32_t dtmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+        "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+        "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+        "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void epi_sync() {
+  asm volatile("bar.sync 2, 128;" ::: "memory");
+}
+
+template <int MODE, int BN, int NMAT>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw0,
+                const __grid_constant__ CUtensorMap tw1, const GemmArgs a) {
+  using C = GemmCfg<BN, NMAT>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled tiles
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
+  uint8_t* aux = smem + (size_t)S * C::kStage;
+  uint64_t* tma_full = reinterpret_cast<uint64_t*>(aux);
+  uint64_t* a_full = tma_full + S;
+  uint64_t* mma_done = a_full + S;
+  uint64_t* accum_full = mma_done + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_full + 1);
+  float* tok_d0 = reinterpret_cast<float*>(aux + C::kAux);
+  float* tok_d1 = tok_d0 + BN;
+  float* tok_f = tok_d1 + BN;
+  int* tok_rs = reinterpret_cast<int*>(tok_f + BN);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_tile = blockIdx.x, m_tile = blockIdx.y;
+  const int kst = (a.K + kBK - 1) / kBK;
+  const int k0 = (int)(((int64_t)blockIdx.z * kst) / a.ksplit);
+  const int k1 = (int)(((int64_t)(blockIdx.z + 1) * kst) / a.ksplit);
+  const int nk = k1 - k0;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&tma_full[s], 1);
+      mbar_init(&a_full[s], 4);
+      mbar_init(&mma_done[s], 1);
+    }
+    mbar_init(accum_full, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tx);
+    prefetch_tmap(&tw0);
+    if (NMAT == 2) prefetch_tmap(&tw1);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"((uint32_t)C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (tid == 0) pdl_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_normal();
+      const uint64_t pol_x = policy_evict_last();
+      const uint32_t bytes = (uint32_t)(C::kB + NMAT * C::kP);
+      // weights do not depend on the previous kernel: prefetch the first
+      // stages before waiting for it, then add the activation tiles.
+      const int pre = nk < S ? nk : S;
+      for (int u = 0; u < pre; ++u) {
+        uint8_t* st = smem + (size_t)u * C::kStage;
+        const int kx = (k0 + u) * kBK;
+        mbar_arrive_expect_tx(&tma_full[u], bytes);
+        tma_load_2d(st + C::kB + NMAT * C::kA, &tw0, &tma_full[u], kx / 4, n_tile * kBM, pol_w);
+        if (NMAT == 2)
+          tma_load_2d(st + C::kB + NMAT * C::kA + C::kP, &tw1, &tma_full[u], kx / 4,
+                      n_tile * kBM, pol_w);
+      }
+      pdl_wait();
+      for (int u = 0; u < pre; ++u) {
+        uint8_t* st = smem + (size_t)u * C::kStage;
+        tma_load_2d(st, &tx, &tma_full[u], (k0 + u) * kBK, m_tile * BN, pol_x);
+      }
+      for (int u = pre; u < nk; ++u) {
+        const int s = u % S;
+        if (!mbar_wait(&mma_done[s], ((u / S) - 1) & 1)) break;
+        uint8_t* st = smem + (size_t)s * C::kStage;
+        const int kx = (k0 + u) * kBK;
+        mbar_arrive_expect_tx(&tma_full[s], bytes);
+        tma_load_2d(st, &tx, &tma_full[s], kx, m_tile * BN, pol_x);
+        tma_load_2d(st + C::kB + NMAT * C::kA, &tw0, &tma_full[s], kx / 4, n_tile * kBM, pol_w);
+        if (NMAT == 2)
+          tma_load_2d(st + C::kB + NMAT * C::kA + C::kP, &tw1, &tma_full[s], kx / 4,
+                      n_tile * kBM, pol_w);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      for (int u = 0; u < nk && ok; ++u) {
+        const int s = u % S;
+        const uint32_t ph = (u / S) & 1;
+        ok = mbar_wait(&a_full[s], ph) && mbar_wait(&tma_full[s], ph);
+        if (!ok) break;
+        tc_fence_after();
+        uint8_t* st = smem + (size_t)s * C::kStage;
+        const uint64_t bdesc = sw128_desc(smem_u32(st));
+#pragma unroll
+        for (int mat = 0; mat < NMAT; ++mat) {
+          const uint64_t adesc = sw128_desc(smem_u32(st + C::kB + mat * C::kA));
+#pragma unroll
+          for (int kk = 0; kk < kBK / 32; ++kk) {
+            // advance 32 bytes of K inside the swizzle atom: +2 in 16-byte units
+            tc_mma_i8(tmem + mat * BN, adesc + 2 * kk, bdesc + 2 * kk, C::kIdesc,
+                      (u > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(&mma_done[s]);
+      }
+      tc_commit(accum_full);
+    }
+  } else {
+    // ------------------------------------- unpack (then epilogue) warps
+    const int ut = tid - 64;                 // 0..127: one weight row each
+    bool ok = true;
+    for (int u = 0; u < nk; ++u) {
+      const int s = u % S;
+      if (!mbar_wait(&tma_full[s], (u / S) & 1)) { ok = false; break; }
+      uint8_t* st = smem + (size_t)s * C::kStage;
+#pragma unroll
+      for (int mat = 0; mat < NMAT; ++mat) {
+        const uint4* pk = reinterpret_cast<const uint4*>(st + C::kB + NMAT * C::kA + mat * C::kP +
+                                                         ut * (kBK / 4));
+        const uint4 p0 = pk[0], p1 = pk[1];
+        const uint32_t wv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+        uint8_t* arow = st + C::kB + mat * C::kA + ut * kBK;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t w = wv[j];
+          const uint4 o = make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u,
+                                     (w >> 4) & 0x03030303u, (w >> 6) & 0x03030303u);
+          *reinterpret_cast<uint4*>(arow + ((j ^ (ut & 7)) << 4)) = o;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[s]);
+    }
+
+    // --------------------------------------------------------- epilogue
+    pdl_wait();
+    const int et = ut;                       // 0..127
+    for (int c = et; c < BN; c += 128) {
+      const int tok = m_tile * BN + c;
+      float d0 = 0.f, d1 = 0.f, f = 0.f;
+      int rs = 0;
+      if (tok < a.M) {
+        const float s = a.scale[tok];
+        d0 = __fdiv_rn(*a.gamma0, s);
+        if (MODE == gGlu) d1 = __fdiv_rn(*a.gamma1, s);
+        rs = a.rowsum[tok];
+        if (MODE == gDown) {
+          const double eps = (double)a.eps;
+          const double r1 = 1.0 / sqrt(a.sumsq_x[tok] / (double)a.H + eps);
+          const double r1_3 = r1 * r1 * r1;
+          const double r2 = 1.0 / sqrt(r1_3 * r1_3 * (a.sumsq_h[tok] / (double)a.K) + eps);
+          f = (float)(r1_3 * r2);
+        }
+      }
+      tok_d0[c] = d0;
+      tok_d1[c] = d1;
+      tok_f[c] = f;
+      tok_rs[c] = rs;
+    }
+    epi_sync();
+    if (ok && !mbar_wait(accum_full, 0)) ok = false;
+    tc_fence_after();
+    if (ok) {
+      const int lb = 32 * (warp & 3);        // TMEM lanes this warp may access
+      const int n = n_tile * kBM + lb + lane;
+      const uint32_t tbase = tmem + ((uint32_t)lb << 16);
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tbase + c0, v0);
+        if (NMAT == 2) tmem_ld32(tbase + BN + c0, v1);
+        if (n < a.N) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int c = c0 + i;
+            const int tok = m_tile * BN + c;
+            if (tok >= a.M) continue;
+            const int64_t o = (int64_t)tok * a.N + n;
+            if (a.ksplit > 1) {
+              atomicAdd(&a.acc_ws0[o], (int)v0[i]);
+              if (NMAT == 2) atomicAdd(&a.acc_ws1[o], (int)v1[i]);
+              continue;
+            }
+            const int ac = (int)v0[i] - tok_rs[c];
+            if (MODE == gGlu) {
+              const int au = (int)v1[i] - tok_rs[c];
+              const float g = __fmul_rn(__int2float_rn(ac), tok_d0[c]);
+              const float uu = __fmul_rn(__int2float_rn(au), tok_d1[c]);
+              const float rg = fmaxf(g, 0.0f);
+              a.h[o] = __fmul_rn(__fmul_rn(rg, rg), uu);
+              if (a.acc0) a.acc0[o] = ac;
+              if (a.acc1) a.acc1[o] = au;
+            } else {
+              float y32 = __fmul_rn(__int2float_rn(ac), tok_d0[c]);
+              if (MODE == gDown) y32 = __fmul_rn(y32, tok_f[c]);
+              a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+              if (a.y_f32) a.y_f32[o] = y32;
+              if (a.acc0) a.acc0[o] = ac;
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    // every MMA has completed once accum_full has (it is committed last)
+    mbar_wait(accum_full, 0);
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"((uint32_t)C::kTmemCols)
+                 : "memory");
+  }
+}
+
+// Split-K finalisation: integer accumulators -> the mode's epilogue.
+template <int MODE>
+__global__ void __launch_bounds__(256) splitk_finalize_kernel(const GemmArgs a) {
+  pdl_wait();
+  const int64_t total = (int64_t)a.M * a.N;
+  for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < total;
+       o += (int64_t)gridDim.x * blockDim.x) {
+    const int tok = (int)(o / a.N);
+    const float s = a.scale[tok];
+    const int rs = a.rowsum[tok];
+    const int ac = a.acc_ws0[o] - rs;
+    if (MODE == gGlu) {
+      const int au = a.acc_ws1[o] - rs;
+      const float g = __fmul_rn(__int2float_rn(ac), __fdiv_rn(*a.gamma0, s));
+      const float uu = __fmul_rn(__int2float_rn(au), __fdiv_rn(*a.gamma1, s));
+      const float rg = fmaxf(g, 0.0f);
+      a.h[o] = __fmul_rn(__fmul_rn(rg, rg), uu);
+      if (a.acc0) a.acc0[o] = ac;
+      if (a.acc1) a.acc1[o] = au;
+    } else {
+      float y32 = __fmul_rn(__int2float_rn(ac), __fdiv_rn(*a.gamma0, s));
+      if (MODE == gDown) {
+        const double eps = (double)a.eps;
+        const double r1 = 1.0 / sqrt(a.sumsq_x[tok] / (double)a.H + eps);
+        const double r1_3 = r1 * r1 * r1;
+        const double r2 = 1.0 / sqrt(r1_3 * r1_3 * (a.sumsq_h[tok] / (double)a.K) + eps);
+        y32 = __fmul_rn(y32, (float)(r1_3 * r2));
+      }
+      a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+      if (a.y_f32) a.y_f32[o] = y32;
+      if (a.acc0) a.acc0[o] = ac;
+    }
+  }
+  pdl_launch_dependents();
+}
+
+}  // namespace bitnet
+
+// ------------------------------------------------------------------ host
+using namespace bitnet;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D uint8 tensor map: inner extent `inner` bytes, `rows` rows, row stride
+// `stride` bytes, box `box_inner` x `box_rows`.
+static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                        uint64_t stride, uint32_t box_inner, uint32_t box_rows, bool sw128) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {stride};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int MODE, int BN, int NMAT>
+static cudaError_t launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw0,
+                                 const CUtensorMap& tw1, const GemmArgs& a, dim3 grid,
+                                 cudaStream_t stream) {
+  using C = GemmCfg<BN, NMAT>;
+  static int configured_dev_mask = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(configured_dev_mask & (1 << (dev & 31)))) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<MODE, BN, NMAT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmem);
+    if (e != cudaSuccess) return e;
+    configured_dev_mask |= 1 << (dev & 31);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<MODE, BN, NMAT>, tx, tw0, tw1, a);
+}
+
+int bitnet_gemm_pick_bn(int M) {
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  if (M <= 128) return 128;
+  return 256;
+}
+
+// Launch the tensor-core kernel (and, with ksplit > 1, its finaliser).
+// xq: [M, K] int8 in the permuted K order; w0/w1: packed [N, K/4].
+bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
+                                 const uint8_t* w1, GemmArgs a, int bn, cudaStream_t stream) {
+  CUtensorMap tx, tw0, tw1;
+  const int nmat = mode == gGlu ? 2 : 1;
+  if (!make_map_u8(&tx, xq, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, kBK, (uint32_t)bn, true))
+    return BITNET_ERR_CUDA;
+  if (!make_map_u8(&tw0, w0, (uint64_t)a.K / 4, (uint64_t)a.N, (uint64_t)a.K / 4, kBK / 4, kBM,
+                   false))
+    return BITNET_ERR_CUDA;
+  if (nmat == 2) {
+    if (!make_map_u8(&tw1, w1, (uint64_t)a.K / 4, (uint64_t)a.N, (uint64_t)a.K / 4, kBK / 4, kBM,
+                     false))
+      return BITNET_ERR_CUDA;
+  } else {
+    tw1 = tw0;
+  }
+  dim3 grid((a.N + kBM - 1) / kBM, (a.M + bn - 1) / bn, a.ksplit);
+  cudaError_t e = cudaErrorInvalidValue;
+#define BITNET_GEMM_BN(MODE_, NMAT_)                                              \
+  switch (bn) {                                                                   \
+    case 32: e = launch_gemm_t<MODE_, 32, NMAT_>(tx, tw0, tw1, a, grid, stream); break;   \
+    case 64: e = launch_gemm_t<MODE_, 64, NMAT_>(tx, tw0, tw1, a, grid, stream); break;   \
+    case 128: e = launch_gemm_t<MODE_, 128, NMAT_>(tx, tw0, tw1, a, grid, stream); break; \
+    default: e = launch_gemm_t<MODE_, 256, NMAT_>(tx, tw0, tw1, a, grid, stream); break;  \
+  }
+  if (mode == gLinear) { BITNET_GEMM_BN(gLinear, 1) }
+  else if (mode == gGlu) { BITNET_GEMM_BN(gGlu, 2) }
+  else { BITNET_GEMM_BN(gDown, 1) }
+#undef BITNET_GEMM_BN
+  if (e != cudaSuccess) return BITNET_ERR_CUDA;
+  if (a.ksplit > 1) {
+    cudaLaunchConfig_t cfg = {};
+    const int64_t total = (int64_t)a.M * a.N;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (mode == gLinear) e = cudaLaunchKernelEx(&cfg, splitk_finalize_kernel<gLinear>, a);
+    else if (mode == gGlu) e = cudaLaunchKernelEx(&cfg, splitk_finalize_kernel<gGlu>, a);
+    else e = cudaLaunchKernelEx(&cfg, splitk_finalize_kernel<gDown>, a);
+    if (e != cudaSuccess) return BITNET_ERR_CUDA;
+  }
+  return BITNET_OK;
+}

@@ -1,0 +1,455 @@
+// Decode kernel (M <= 8 tokens): streams packed ternary weights from HBM
+// through a shared-memory ring filled by bulk async copies, with the per-token
+// activation quantisation fused into its prologue.
+//
+// dashen-tech.com "BitNet.cpp 深度解析", section "3.1 計算コア：整数行列乗算":
+// the product with ternary weights is sum_pos - sum_neg.  Here it is taken in
+// the offset form sum_k x_q * code - sum_k x_q (code = w + 1 in {0,1,2}), so a
+// packed 32-bit word of 16 codes needs only four AND masks and four dp4a:
+// plane t = word & (0x03030303 << 2t) holds, byte b, the code of k = 4b + t
+// times 4^t, and the activations sit in shared memory in the matching order.
+//
+// Layout of work: one CTA per SM-slot owns a contiguous range of output rows;
+// warp 8 is the producer (bulk copies of whole rows, a few stages ahead);
+// warps 0..7 each take blocks of 4 rows, lane l reading words l, l+32, ... of
+// each row, then a butterfly reduction across the warp leaves row r's total
+// in lane 8r.
+//
+// Programmatic dependent launch: the producer starts streaming weights
+// before griddepcontrol.wait, the consumers wait before reading activations.
+#include "common.cuh"
+
+namespace bitnet {
+
+enum GemvMode : int { kLinear = 0, kGlu = 1, kDown = 2 };
+
+struct GemvArgs {
+  const uint8_t* w0;      // packed [N, K/4]   (Glu: gate)
+  const float* gamma0;
+  const uint8_t* w1;      // Glu: up
+  const float* gamma1;
+  int N, K, M;
+  const void* x;          // Linear/Glu: bf16 [M,K]; Down: fp32 h' [M,K]
+  const float* gain;      // optional [K] (RMSNorm weight)
+  const uint16_t* xnorm;  // Down: block input x [M,H] (for r1)
+  int H;
+  float eps;
+  uint16_t* y;            // Linear/Down [M,N]
+  float* y_f32;           // optional [M,N]
+  int32_t* acc0;          // optional [M,N]
+  int32_t* acc1;          // optional [M,N] (Glu up)
+  float* h;               // Glu output h' [M,N]
+  int8_t* xq_dbg;         // optional natural-layout x_q [M,K], written by CTA 0
+  int rows_per_stage;     // multiple of 4
+  int stages;             // 2..8
+};
+
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMaxTok = 8;
+
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+
+// Halving step of the butterfly: n values -> n/2, exchanging with lane ^ off.
+template <int N>
+__device__ __forceinline__ void halve(const int (&v)[N], int (&o)[N / 2], int off, int lane) {
+  const bool hi = (lane & off) != 0;
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    const int keep = hi ? v[i + N / 2] : v[i];
+    const int send = hi ? v[i] : v[i + N / 2];
+    o[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+  }
+}
+
+__device__ __forceinline__ float load_src(const void* x, bool f32, int64_t idx) {
+  if (f32) return static_cast<const float*>(x)[idx];
+  return bf16_bits_to_float(static_cast<const uint16_t*>(x)[idx]);
+}
+
+template <int MODE, int MT>
+__global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
+  constexpr int NMAT = (MODE == kGlu) ? 2 : 1;
+  constexpr int NR = 4 * NMAT;             // values per lane per row block
+  constexpr bool kF32Src = (MODE == kDown);
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + 8;
+  float* tok_s = reinterpret_cast<float*>(smem + 128);
+  float* tok_d0 = tok_s + kMaxTok;
+  float* tok_d1 = tok_d0 + kMaxTok;
+  float* tok_f = tok_d1 + kMaxTok;
+  int* tok_rs = reinterpret_cast<int*>(tok_f + kMaxTok);
+  float* red_f = reinterpret_cast<float*>(smem + 384);          // [8 warps][8 tok]
+  int* red_i = reinterpret_cast<int*>(smem + 640);              // [8][8]
+  double* red_d = reinterpret_cast<double*>(smem + 1024);       // [8][8][2]
+  const int M = a.M, K = a.K, N = a.N;
+  const int Mpad = ((M + MT - 1) / MT) * MT;
+  uint8_t* xperm = smem + 2048;
+  const int xbytes = ((Mpad * K + 127) / 128) * 128;
+  uint8_t* ring = xperm + xbytes;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Kb = K >> 2;                   // bytes per packed row
+  const int Kw = K >> 4;                   // 32-bit words per packed row
+  const int n0 = (int)(((int64_t)blockIdx.x * N) / gridDim.x);
+  const int n1 = (int)(((int64_t)(blockIdx.x + 1) * N) / gridDim.x);
+  const int RS = a.rows_per_stage, S = a.stages;
+  const int nchunks = (n1 - n0 + RS - 1) / RS;
+  const int stage_bytes = RS * Kb * NMAT;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) pdl_launch_dependents();
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % S;
+        if (c >= S && !mbar_wait(&empty[s], ((c / S) - 1) & 1)) break;
+        const int r0 = n0 + c * RS;
+        const int nr = min(RS, n1 - r0);
+        const uint32_t bytes = (uint32_t)nr * Kb;
+        mbar_arrive_expect_tx(&full[s], bytes * NMAT);
+        uint8_t* dst = ring + (size_t)s * stage_bytes;
+        bulk_g2s(dst, a.w0 + (int64_t)r0 * Kb, bytes, &full[s], pol);
+        if (NMAT == 2) bulk_g2s(dst + (size_t)RS * Kb, a.w1 + (int64_t)r0 * Kb, bytes, &full[s], pol);
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- prologue
+  pdl_wait();
+  // zero the padding tokens of the activation buffer
+  for (int i = M * K + tid * 16; i < Mpad * K; i += kConsumerWarps * 32 * 16)
+    *reinterpret_cast<uint4*>(xperm + i) = make_uint4(0, 0, 0, 0);
+
+  float am[kMaxTok];
+  double ss[kMaxTok], sx[kMaxTok];
+#pragma unroll
+  for (int m = 0; m < kMaxTok; ++m) { am[m] = 0.f; ss[m] = 0.0; sx[m] = 0.0; }
+  for (int k = tid; k < K; k += kConsumerWarps * 32) {
+    const float g = a.gain ? a.gain[k] : 1.0f;
+#pragma unroll
+    for (int m = 0; m < kMaxTok; ++m) {
+      if (m < M) {
+        const float v = load_src(a.x, kF32Src, (int64_t)m * K + k);
+        const float vg = a.gain ? __fmul_rn(v, g) : v;
+        am[m] = fmaxf(am[m], fabsf(vg));
+        if (MODE == kDown) ss[m] += (double)v * (double)v;
+      }
+    }
+  }
+  if (MODE == kDown) {
+    for (int k = tid; k < a.H; k += kConsumerWarps * 32) {
+#pragma unroll
+      for (int m = 0; m < kMaxTok; ++m)
+        if (m < M) {
+          const double v = (double)bf16_bits_to_float(a.xnorm[(int64_t)m * a.H + k]);
+          sx[m] += v * v;
+        }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < kMaxTok; ++m) {
+    if (m < M) {
+      const float w = warp_max(am[m]);
+      if (lane == 0) red_f[warp * kMaxTok + m] = w;
+      if (MODE == kDown) {
+        const double d1 = warp_sum_d(ss[m]);
+        const double d2 = warp_sum_d(sx[m]);
+        if (lane == 0) {
+          red_d[(warp * kMaxTok + m) * 2 + 0] = d1;
+          red_d[(warp * kMaxTok + m) * 2 + 1] = d2;
+        }
+      }
+    }
+  }
+  consumer_sync();
+  if (tid < M) {
+    const int m = tid;
+    float amax = 0.f;
+    double s1 = 0.0, s2 = 0.0;
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      amax = fmaxf(amax, red_f[w * kMaxTok + m]);
+      if (MODE == kDown) {
+        s1 += red_d[(w * kMaxTok + m) * 2 + 0];
+        s2 += red_d[(w * kMaxTok + m) * 2 + 1];
+      }
+    }
+    const float s = qscale(amax);
+    tok_s[m] = s;
+    tok_d0[m] = __fdiv_rn(*a.gamma0, s);
+    if (MODE == kGlu) tok_d1[m] = __fdiv_rn(*a.gamma1, s);
+    if (MODE == kDown) {
+      const double eps = (double)a.eps;
+      const double r1 = 1.0 / sqrt(s2 / (double)a.H + eps);
+      const double r1_3 = r1 * r1 * r1;
+      const double r2 = 1.0 / sqrt(r1_3 * r1_3 * (s1 / (double)K) + eps);
+      tok_f[m] = (float)(r1_3 * r2);
+    }
+  }
+  consumer_sync();
+  // pass 2: quantise into the permuted layout, group of 16 per thread
+  int rs[kMaxTok];
+#pragma unroll
+  for (int m = 0; m < kMaxTok; ++m) rs[m] = 0;
+  for (int g = tid; g < Kw; g += kConsumerWarps * 32) {
+#pragma unroll
+    for (int m = 0; m < kMaxTok; ++m) {
+      if (m < M) {
+        const float s = tok_s[m];
+        int q[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int k = g * 16 + i;
+          const float v = load_src(a.x, kF32Src, (int64_t)m * K + k);
+          const float vg = a.gain ? __fmul_rn(v, a.gain[k]) : v;
+          q[i] = quant_code(vg, s);
+          rs[m] += q[i];
+        }
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          w[t] = (uint32_t)(q[t] & 0xff) | ((uint32_t)(q[4 + t] & 0xff) << 8) |
+                 ((uint32_t)(q[8 + t] & 0xff) << 16) | ((uint32_t)(q[12 + t] & 0xff) << 24);
+        *reinterpret_cast<uint4*>(xperm + (int64_t)m * K + g * 16) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+        if (a.xq_dbg && blockIdx.x == 0) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) a.xq_dbg[(int64_t)m * K + g * 16 + i] = (int8_t)q[i];
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < kMaxTok; ++m) {
+    if (m < M) {
+      const int t = warp_sum_i(rs[m]);
+      if (lane == 0) red_i[warp * kMaxTok + m] = t;
+    }
+  }
+  consumer_sync();
+  if (tid < M) {
+    int t = 0;
+    for (int w = 0; w < kConsumerWarps; ++w) t += red_i[w * kMaxTok + tid];
+    tok_rs[tid] = t;
+  }
+  consumer_sync();
+
+  // ------------------------------------------------------------- main loop
+  const uint4* x4 = reinterpret_cast<const uint4*>(xperm);
+  bool ok = true;
+  for (int c = 0; c < nchunks && ok; ++c) {
+    const int s = c % S;
+    if (!mbar_wait(&full[s], (c / S) & 1)) { ok = false; break; }
+    const int r0 = n0 + c * RS;
+    const int nr = min(RS, n1 - r0);
+    const uint32_t* st = reinterpret_cast<const uint32_t*>(ring + (size_t)s * stage_bytes);
+    const int nblk = (nr + 3) >> 2;
+    for (int b = warp; b < nblk; b += kConsumerWarps) {
+      for (int tg = 0; tg < M; tg += MT) {
+        int acc[NR][MT];
+        int acc4[NR][4];   // MT == 1: one accumulator per code plane
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+#pragma unroll
+          for (int t = 0; t < MT; ++t) acc[r][t] = 0;
+#pragma unroll
+          for (int p = 0; p < 4; ++p) acc4[r][p] = 0;
+        }
+        for (int j = lane; j < Kw; j += 32) {
+          uint32_t w[NR];
+#pragma unroll
+          for (int r = 0; r < NR; ++r) {
+            // value index r = 2*row + mat for Glu, = row otherwise
+            const int row = (NMAT == 2) ? (r >> 1) : r;
+            const int mat = (NMAT == 2) ? (r & 1) : 0;
+            w[r] = st[(size_t)(mat * RS + 4 * b + row) * Kw + j];
+          }
+          uint4 xv[MT];
+#pragma unroll
+          for (int t = 0; t < MT; ++t) xv[t] = x4[(size_t)(tg + t) * Kw + j];
+#pragma unroll
+          for (int r = 0; r < NR; ++r) {
+            if (MT == 1) {
+              acc4[r][0] = dp4a_su((int)xv[0].x, w[r] & 0x03030303u, acc4[r][0]);
+              acc4[r][1] = dp4a_su((int)xv[0].y, w[r] & 0x0c0c0c0cu, acc4[r][1]);
+              acc4[r][2] = dp4a_su((int)xv[0].z, w[r] & 0x30303030u, acc4[r][2]);
+              acc4[r][3] = dp4a_su((int)xv[0].w, w[r] & 0xc0c0c0c0u, acc4[r][3]);
+            } else {
+              const uint32_t c0 = w[r] & 0x03030303u;
+              const uint32_t c1 = (w[r] >> 2) & 0x03030303u;
+              const uint32_t c2 = (w[r] >> 4) & 0x03030303u;
+              const uint32_t c3 = (w[r] >> 6) & 0x03030303u;
+#pragma unroll
+              for (int t = 0; t < MT; ++t) {
+                int v = acc[r][t];
+                v = dp4a_su((int)xv[t].x, c0, v);
+                v = dp4a_su((int)xv[t].y, c1, v);
+                v = dp4a_su((int)xv[t].z, c2, v);
+                v = dp4a_su((int)xv[t].w, c3, v);
+                acc[r][t] = v;
+              }
+            }
+          }
+        }
+        if (MT == 1) {
+#pragma unroll
+          for (int r = 0; r < NR; ++r)
+            acc[r][0] = acc4[r][0] + (acc4[r][1] >> 2) + (acc4[r][2] >> 4) + (acc4[r][3] >> 6);
+        }
+        // butterfly: lane l ends with value index (l >> 32/NR-bits) summed
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          int v[NR];
+#pragma unroll
+          for (int r = 0; r < NR; ++r) v[r] = acc[r][t];
+          int tot;
+          if constexpr (NR == 4) {
+            int h2[2], h1[1];
+            halve<4>(*reinterpret_cast<int(*)[4]>(v), h2, 16, lane);
+            halve<2>(h2, h1, 8, lane);
+            tot = h1[0];
+            tot += __shfl_xor_sync(0xffffffffu, tot, 4);
+            tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+            tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+          } else {
+            int h4[4], h2[2], h1[1];
+            halve<8>(*reinterpret_cast<int(*)[8]>(v), h4, 16, lane);
+            halve<4>(h4, h2, 8, lane);
+            halve<2>(h2, h1, 4, lane);
+            tot = h1[0];
+            tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+            tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+          }
+          int other = 0;
+          if (NMAT == 2) other = __shfl_xor_sync(0xffffffffu, tot, 4);   // up total
+          const int m = tg + t;
+          const int row = lane >> 3;                    // 0..3
+          const bool writer = (lane & 7) == 0;
+          const int n = r0 + 4 * b + row;
+          if (writer && m < M && 4 * b + row < nr) {
+            const int64_t o = (int64_t)m * N + n;
+            const int rsum = tok_rs[m];
+            if (MODE == kGlu) {
+              const int ag = tot - rsum, au = other - rsum;
+              const float g = __fmul_rn(__int2float_rn(ag), tok_d0[m]);
+              const float u = __fmul_rn(__int2float_rn(au), tok_d1[m]);
+              const float rg = fmaxf(g, 0.0f);
+              a.h[o] = __fmul_rn(__fmul_rn(rg, rg), u);
+              if (a.acc0) a.acc0[o] = ag;
+              if (a.acc1) a.acc1[o] = au;
+            } else {
+              const int ac = tot - rsum;
+              float y32 = __fmul_rn(__int2float_rn(ac), tok_d0[m]);
+              if (MODE == kDown) y32 = __fmul_rn(y32, tok_f[m]);
+              a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+              if (a.y_f32) a.y_f32[o] = y32;
+              if (a.acc0) a.acc0[o] = ac;
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+}
+
+template <int MODE, int MT>
+static cudaError_t launch_one(const GemvArgs& a, int grid, size_t smem, cudaStream_t stream) {
+  static unsigned long long configured = 0;   // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(configured & (1ull << (dev & 63)))) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MODE, MT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    configured |= 1ull << (dev & 63);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<MODE, MT>, a);
+}
+
+// Host-side planning: stage rows and ring depth under a shared-memory budget
+// that leaves room for a second CTA per SM (the next kernel in the stream).
+struct GemvPlan {
+  int grid, rows_per_stage, stages;
+  size_t smem;
+};
+
+static GemvPlan plan_gemv(int M, int N, int K, int nmat, int num_sms, int MT) {
+  GemvPlan p{};
+  const int Mpad = ((M + MT - 1) / MT) * MT;
+  const size_t xbytes = (((size_t)Mpad * K + 127) / 128) * 128;
+  const size_t budget = 112 * 1024;
+  const size_t head = 2048 + xbytes;
+  const size_t row_bytes = (size_t)(K / 4) * nmat;
+  int blocks = (N + 3) / 4;
+  p.grid = blocks < num_sms ? blocks : num_sms;
+  const int rows_per_cta = (N + p.grid - 1) / p.grid;
+  const size_t ring = budget > head + 2 * 4 * row_bytes ? budget - head : 2 * 4 * row_bytes;
+  int rs = (int)((32 * 1024) / row_bytes);
+  rs = rs / 4 * 4;
+  if (rs < 4) rs = 4;
+  const int rows_cap = (rows_per_cta + 3) / 4 * 4;
+  if (rs > rows_cap) rs = rows_cap;
+  int st = (int)(ring / ((size_t)rs * row_bytes));
+  if (st > 8) st = 8;
+  if (st < 2) st = 2;
+  p.rows_per_stage = rs;
+  p.stages = st;
+  p.smem = head + (size_t)st * rs * row_bytes;
+  return p;
+}
+
+}  // namespace bitnet
+
+using namespace bitnet;
+
+size_t bitnet_gemv_smem_bytes(int M, int N, int K, int nmat, int num_sms) {
+  const int MT = M == 1 ? 1 : (M == 2 ? 2 : 4);
+  return plan_gemv(M, N, K, nmat, num_sms, MT).smem;
+}
+
+bitnet_status bitnet_gemv_launch(int mode, GemvArgs a, int num_sms, cudaStream_t stream) {
+  const int nmat = mode == kGlu ? 2 : 1;
+  const int MT = a.M == 1 ? 1 : (a.M == 2 ? 2 : 4);
+  const GemvPlan p = plan_gemv(a.M, a.N, a.K, nmat, num_sms, MT);
+  if (p.smem > 227 * 1024) return BITNET_ERR_UNSUPPORTED;
+  a.rows_per_stage = p.rows_per_stage;
+  a.stages = p.stages;
+  cudaError_t e = cudaErrorInvalidValue;
+#define BITNET_GEMV_CASE(MODE_)                                                       \
+  if (mode == MODE_) {                                                                \
+    if (MT == 1) e = launch_one<MODE_, 1>(a, p.grid, p.smem, stream);                 \
+    else if (MT == 2) e = launch_one<MODE_, 2>(a, p.grid, p.smem, stream);            \
+    else e = launch_one<MODE_, 4>(a, p.grid, p.smem, stream);                         \
+  }
+  BITNET_GEMV_CASE(kLinear)
+  BITNET_GEMV_CASE(kGlu)
+  BITNET_GEMV_CASE(kDown)
+#undef BITNET_GEMV_CASE
+  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}

@@ -1,0 +1,105 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+symbol include/bitnet.h declares, and rejects bad arguments on the host
+before touching CUDA (the pointers below are never dereferenced)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from ternary_weight_linear_int8_b200 import bitnet as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitnet.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(bitnet_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    return B.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    # and the binding knows every one of them
+    assert set(names) <= set(B.SIGNATURES)
+
+
+def test_status_strings_and_version(L):
+    assert B.bitnet_version() == 100
+    for code, name in B.STATUS.items():
+        assert B.bitnet_status_string(code) == name
+    assert B.bitnet_status_string(99) == "BITNET_ERR_UNKNOWN"
+
+
+def test_workspace_sizes_are_host_only(L):
+    assert L.bitnet_pack_workspace_size(400, 512) >= 2052
+    assert L.bitnet_linear_workspace_size(1, 6912, 2560) == 0          # fused decode kernel
+    assert L.bitnet_linear_workspace_size(4096, 6912, 2560) >= 4096 * 2560
+    assert L.bitnet_linear_workspace_size(64, 2560, 6912) >= 64 * 6912 + 64 * 2560 * 4
+    assert L.bitnet_linear_workspace_size(8, 400, 68) >= 8 * 68        # ragged K
+    assert L.bitnet_ffn_workspace_size(1, 8192, 28672) == 28672 * 4
+    assert L.bitnet_ffn_workspace_size(2048, 8192, 28672) > 2048 * 28672 * 4
+
+
+FAKE = 0x10000          # 16-byte aligned, never dereferenced
+MIS = 0x10001           # misaligned
+
+
+def test_linear_validation(L):
+    lin = L.bitnet_linear
+    ok_args = dict(packed=FAKE, gamma=FAKE, N=400, K=512, x=FAKE, M=8, y=FAKE, y32=None,
+                   acc=None, ws=None, nb=0, stream=None)
+
+    def call(**kw):
+        a = dict(ok_args, **kw)
+        return lin(a["packed"], a["gamma"], a["N"], a["K"], a["x"], a["M"], a["y"], a["y32"],
+                   a["acc"], a["ws"], a["nb"], a["stream"])
+
+    assert call(packed=None) == 1
+    assert call(y=None) == 1
+    assert call(K=510) == 2
+    assert call(K=0) == 2
+    assert call(M=0) == 2
+    assert call(N=-1) == 2
+    assert call(x=MIS) == 3
+    assert call(packed=MIS) == 3
+    assert call(y32=FAKE + 2) == 3
+    # tensor-core shapes need a workspace
+    assert call(M=4096, K=2560, N=6912) == 4
+    assert call(M=4096, K=2560, N=6912, ws=FAKE, nb=16) == 4
+
+
+def test_pack_quant_ffn_validation(L):
+    assert L.bitnet_pack_weights(None, 4, 4, FAKE, FAKE, FAKE, 4096, None) == 1
+    assert L.bitnet_pack_weights(FAKE, 4, 6, FAKE, FAKE, FAKE, 4096, None) == 2
+    assert L.bitnet_pack_weights(MIS, 4, 8, FAKE, FAKE, FAKE, 4096, None) == 3
+    assert L.bitnet_pack_weights(FAKE, 4, 8, FAKE, FAKE, FAKE, 16, None) == 4
+    assert L.bitnet_pack_weights(FAKE, 4, 8, FAKE, FAKE, None, 4096, None) == 4
+    assert L.bitnet_quant_act(None, 1, 8, FAKE, FAKE, None, None) == 1
+    assert L.bitnet_quant_act(FAKE, 1, 6, FAKE, FAKE, None, None) == 2
+    assert L.bitnet_quant_act(FAKE, 1, 8, MIS, FAKE, None, None) == 3
+    f = L.bitnet_ffn
+    args = [FAKE, 1, 256, 512, None, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1e-5, FAKE, None,
+            FAKE, 1 << 20, None]
+    a = list(args); a[5] = None
+    assert f(*a) == 1
+    a = list(args); a[12] = -1.0
+    assert f(*a) == 1
+    a = list(args); a[2] = 200
+    assert f(*a) == 2
+    a = list(args); a[0] = MIS
+    assert f(*a) == 3
+    a = list(args); a[16] = 16
+    assert f(*a) == 4
