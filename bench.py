@@ -1,0 +1,525 @@
+#!/usr/bin/env python3
+"""Benchmark of the W1.58A8 BitLinear hot path on B200.
+
+Headline workload (one "step"): 2B-class decode, M = 1 token, a chain of 30
+layers x {up [6912,2560], down [2560,6912]} = 60 distinct packed matrices
+(265 MB of packed weights, larger than the 126 MB L2), each BitLinear fed the
+previous one's bf16 output, captured in one CUDA graph (kernels use
+programmatic dependent launch).  Per step the path runs activation quant
+(fused), the ternary int8 matmul and the dequant/bf16 store for all 60
+matrices.  value = packed-weight bytes streamed / device time (GB/s).
+
+Secondary figures (same JSON line, "secondary"): prefill GEMM TOPS at M=4096,
+batched decode M in {4,16,64}, and the 100B-class FFN block at M=1 and 2048.
+
+--impl reference times the CPU oracle (the only other implementation there
+is) on the same metric, a bounded sample per step.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: launched with torch.distributed.run, one rank per GPU; each rank
+runs an independent replica of the workload (weak scaling, no collective on
+the data path); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W1.58A8 BitLinear GEMV GB/s (% of HBM peak); GEMM TOPS (% of int8 peak)"
+HIDDEN, INTER, LAYERS = 2560, 6912, 30
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_OVER_BF16 = 2.0            # nominal dense int8 : bf16 tensor-core ratio (4.5 : 2.25 PFLOP/s)
+KERNEL_SOURCES = ["common.cuh", "gemv.cu", "gemm.cu", "quant.cu", "pack.cu", "api.cu"]
+
+
+# ---------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "ternary_weight_linear_int8_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(name):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (the summary records their hash)."""
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_h = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
+    m_t = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_h or not m_t or m_h.group(1) != kernel_hash():
+        return None
+    return float(m_t.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons with NVML in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, period=0.02):
+        self.samples = []
+        self.period = period
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_sm = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((time.time(), sm, r, pw))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        self._stop.set()
+        self.t.join()
+        win = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples[-5:]
+        reasons = set()
+        for s in win:
+            for bit, name in self.REASONS.items():
+                if s[2] & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median([s[1] for s in win]) if win else None,
+                "sm_max_mhz": self.max_sm, "reasons": sorted(reasons),
+                "samples": len(win),
+                "power_w_median": statistics.median([s[3] for s in win]) if win else None}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# -------------------------------------------------------- CPU reference arm
+def oracle_decode_sample(n_layers, seed_base=0):
+    """Pack a few decode layers with the oracle (untimed) and return them."""
+    from oracle import bitlinear as O
+    from ternary_weight_linear_int8_b200 import inputs
+    layers = []
+    for l in range(n_layers):
+        N, K = (INTER, HIDDEN) if l % 2 == 0 else (HIDDEN, INTER)
+        W = inputs.weights(N, K, seed=inputs.layer_seed(l + seed_base))
+        layers.append(O.pack_weights(W))
+    return layers
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle_chain(layers, x_bits, repeats):
+    from oracle import bitlinear as O
+    t0 = time.perf_counter()
+    nbytes = 0
+    for _ in range(repeats):
+        cur = x_bits
+        for packed, g in layers:
+            out = O.linear(packed, g, cur)
+            cur = out["y"]
+            nbytes += packed.nbytes
+    dt = time.perf_counter() - t0
+    return nbytes, dt
+
+
+def cpu_baseline(target_s=10.0):
+    from ternary_weight_linear_int8_b200 import inputs
+    layers = oracle_decode_sample(2)
+    x = inputs.activations((1, HIDDEN), seed=0)
+    nbytes, dt = time_oracle_chain(layers, x, 1)          # warm
+    reps = max(1, int(target_s / max(dt, 1e-3)))
+    nbytes, dt = time_oracle_chain(layers, x, reps)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{reps} passes over 2 of the 60 decode layers (up [6912,2560] then "
+                      f"down [2560,6912]), M=1, oracle.linear from oracle-packed weights; "
+                      f"{dt:.1f} s of CPU time; matmul in BLAS, elementwise steps "
+                      f"single-threaded numpy"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    from ternary_weight_linear_int8_b200 import inputs
+    layers = oracle_decode_sample(2)
+    x = inputs.activations((1, HIDDEN), seed=0)
+    for _ in range(args.warmup):
+        time_oracle_chain(layers, x, 1)
+    t0 = time.perf_counter()
+    nbytes, _ = 0, 0
+    for _ in range(args.steps):
+        nb, _dt = time_oracle_chain(layers, x, 1)
+        nbytes += nb
+    dt = time.perf_counter() - t0
+    val = nbytes / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": "decode GEMV M=1, 2B-class chain; reference = CPU oracle on a "
+                               "bounded sample: each step = 2 of the 60 layers "
+                               "(up [6912,2560], down [2560,6912])",
+                   "M": 1},
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": "each step: oracle.linear over 2 decode layers (one up, one "
+                                   "down), M=1, oracle-packed weights"},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------- GPU arm
+def build_decode_chain(B, inputs, torch, dev, n_layers=2 * LAYERS):
+    packs = []
+    for l in range(n_layers):
+        N, K = (INTER, HIDDEN) if l % 2 == 0 else (HIDDEN, INTER)
+        W = torch.from_numpy(inputs.weights(N, K, seed=inputs.layer_seed(l))).to(dev)
+        packs.append(B.bitnet_pack_weights(W))
+        del W
+    return packs
+
+
+def chain_calls(B, packs, x, bufs):
+    cur = x
+    for l, (p, g) in enumerate(packs):
+        out = bufs[l % 2]
+        B.bitnet_linear(p, g, cur, y=out)
+        cur = out
+    return cur
+
+
+def capture(torch, fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def time_graph(torch, graph, stream, steps, warmup, barrier=None):
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            graph.replay()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(stream)
+    e1.synchronize()
+    t1 = time.time()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    return e0.elapsed_time(e1), t0, t1
+
+
+def secondary_measurements(B, inputs, torch, dev, stream, pk):
+    """Prefill GEMM TOPS, batched decode, FFN block; kernel-timed via graphs."""
+    out = {}
+    int8_peak = pk["bf16_tflops"] * INT8_OVER_BF16
+    # prefill M=4096 on up and down
+    M = 4096
+    xs = {K: torch.from_numpy(inputs.activations((M, K), seed=0).view(np.int16)).to(dev)
+          for K in (HIDDEN, INTER)}
+    Wu = torch.from_numpy(inputs.weights(INTER, HIDDEN, seed=1000)).to(dev)
+    Wd = torch.from_numpy(inputs.weights(HIDDEN, INTER, seed=1001)).to(dev)
+    pu, pd = B.bitnet_pack_weights(Wu), B.bitnet_pack_weights(Wd)
+    del Wu, Wd
+    yu = torch.empty((M, INTER), dtype=torch.bfloat16, device=dev)
+    yd = torch.empty((M, HIDDEN), dtype=torch.bfloat16, device=dev)
+    wsu = torch.empty(B.bitnet_linear_workspace_size(M, INTER, HIDDEN), dtype=torch.uint8, device=dev)
+    wsd = torch.empty(B.bitnet_linear_workspace_size(M, HIDDEN, INTER), dtype=torch.uint8, device=dev)
+    for name, (p, x, y, ws, N, K) in {"up": (pu, xs[HIDDEN], yu, wsu, INTER, HIDDEN),
+                                      "down": (pd, xs[INTER], yd, wsd, HIDDEN, INTER)}.items():
+        g = capture(torch, lambda: B.bitnet_linear(*p, x, y=y, workspace=ws), stream)
+        ms, _, _ = time_graph(torch, g, stream, 50, 5)
+        ops = 2.0 * M * N * K
+        tops = ops / (ms / 50 * 1e-3) / 1e12
+        out[f"prefill_M4096_{name}"] = {"TOPS": round(tops, 1), "us_per_call": round(ms / 50 * 1e3, 2),
+                                        "frac_int8_peak": round(tops / int8_peak, 4),
+                                        "includes": "activation quant kernel + tcgen05 GEMM"}
+        del g
+    del xs, yu, yd, wsu, wsd
+    # batched decode: the same 60-layer chain with M tokens
+    packs = pk["_packs"]
+    for M in (4, 16, 64):
+        x = torch.from_numpy(inputs.activations((M, HIDDEN), seed=0, outliers=True).view(np.int16)).to(dev)
+        bufs = [torch.empty((M, INTER), dtype=torch.bfloat16, device=dev),
+                torch.empty((M, HIDDEN), dtype=torch.bfloat16, device=dev)]
+        wsb = torch.empty(max(B.bitnet_linear_workspace_size(M, INTER, HIDDEN),
+                              B.bitnet_linear_workspace_size(M, HIDDEN, INTER), 16),
+                          dtype=torch.uint8, device=dev)
+
+        def run():
+            cur = x
+            for l, (p, g_) in enumerate(packs):
+                B.bitnet_linear(p, g_, cur, y=bufs[l % 2], workspace=wsb)
+                cur = bufs[l % 2]
+        g = capture(torch, run, stream)
+        ms, _, _ = time_graph(torch, g, stream, 20, 3)
+        t = ms / 20 * 1e-3
+        nbytes = sum(p.numel() for p, _ in packs)
+        ops = 2.0 * M * sum(p.numel() * 4 for p, _ in packs)
+        out[f"decode_chain_M{M}"] = {"GB/s": round(nbytes / t / 1e9, 1),
+                                     "TOPS": round(ops / t / 1e12, 2),
+                                     "frac_hbm": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4),
+                                     "us_per_step": round(t * 1e6, 1)}
+        del g
+    # FFN 100B-class: two distinct blocks rotated
+    H, I = 8192, 28672
+    blocks = []
+    for b in range(2):
+        ws_ = []
+        for (n, k, sd) in ((I, H, 2000 + 3 * b), (I, H, 2001 + 3 * b), (H, I, 2002 + 3 * b)):
+            W = torch.from_numpy(inputs.weights(n, k, seed=sd)).to(dev)
+            ws_.append(B.bitnet_pack_weights(W))
+            del W
+        blocks.append(B.FfnWeights(ws_[0][0], ws_[0][1], ws_[1][0], ws_[1][1], ws_[2][0], ws_[2][1]))
+    for M in (1, 2048):
+        x = torch.from_numpy(inputs.activations((M, H), seed=0).view(np.int16)).to(dev)
+        y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        wsf = torch.empty(B.bitnet_ffn_workspace_size(M, H, I), dtype=torch.uint8, device=dev)
+
+        def run_ffn():
+            for w in blocks:
+                B.bitnet_ffn(x, w, eps=1e-5, y=y, workspace=wsf)
+        g = capture(torch, run_ffn, stream)
+        iters = 20 if M == 1 else 5
+        ms, _, _ = time_graph(torch, g, stream, iters, 2)
+        t = ms / iters * 1e-3 / 2                    # per block
+        nbytes = 3 * H * I / 4
+        ops = 2.0 * M * 3 * H * I
+        out[f"ffn_100b_M{M}"] = {"GB/s": round(nbytes / t / 1e9, 1), "TOPS": round(ops / t / 1e12, 1),
+                                 "us_per_block": round(t * 1e6, 1),
+                                 "frac_hbm" if M == 1 else "frac_int8_peak":
+                                     round(nbytes / t / 1e9 / pk["hbm_gbs"], 4) if M == 1
+                                     else round(ops / t / 1e12 / int8_peak, 4)}
+        del g, wsf
+    return out
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    from ternary_weight_linear_int8_b200 import bitnet as B
+    from ternary_weight_linear_int8_b200 import inputs
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    barrier = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        barrier = dist.barrier
+    B.lib()
+    pk = peaks()
+    stream = torch.cuda.Stream(device=dev)
+
+    # ------------------------------------------------ headline: decode chain
+    packs = build_decode_chain(B, inputs, torch, dev)
+    pk["_packs"] = packs
+    x_host = inputs.activations((1, HIDDEN), seed=0)
+    x = torch.from_numpy(x_host.view(np.int16)).to(dev)
+    bufs = [torch.empty((1, INTER), dtype=torch.bfloat16, device=dev),
+            torch.empty((1, HIDDEN), dtype=torch.bfloat16, device=dev)]
+    torch.cuda.synchronize()
+    graph = capture(torch, lambda: chain_calls(B, packs, x, bufs), stream)
+    sampler = ClockSampler(local)
+    sampler.start()
+    ms, t0, t1 = time_graph(torch, graph, stream, args.steps, args.warmup, barrier)
+    clocks = sampler.stop(t0, t1)
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    # the graph's output equals an eager chain, bit for bit
+    y_graph = bufs[1].clone()
+    chain_calls(B, packs, x, bufs)
+    torch.cuda.synchronize()
+    check_ok = bool(torch.equal(y_graph.view(torch.int16), bufs[1].view(torch.int16)))
+    status = B.bitnet_last_device_status()
+
+    n_launch = len(packs)
+    step_s = ms / args.steps * 1e-3
+    packed_bytes = sum(p.numel() for p, _ in packs)
+    value = world * packed_bytes / step_s / 1e9
+    # roofline for the decode kernel: algorithmic bytes per launch / avg launch time
+    alg_bytes = packed_bytes / n_launch + 2 * HIDDEN + 2 * INTER + 4
+    launch_s = step_s / n_launch
+    achieved = alg_bytes / launch_s / 1e9
+    traffic = profile_traffic("gemv_decode_2b_m1.md")
+
+    # --------------------------------------------------- e2e through the API
+    # per step: pinned host x -> device, 60 bitnet_linear calls through the
+    # binding (eager, no graph), device -> pinned host y
+    xh = torch.from_numpy(x_host.view(np.int16)).pin_memory()
+    yh = torch.empty((1, HIDDEN), dtype=torch.int16).pin_memory()
+    xd = torch.empty((1, HIDDEN), dtype=torch.int16, device=dev)
+    e2e_steps = max(5, min(args.steps, 200))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            xd.copy_(xh, non_blocking=True)
+            out = chain_calls(B, packs, xd, bufs)
+            yh.copy_(out.view(torch.int16), non_blocking=True)
+        torch.cuda.synchronize()
+        if barrier:
+            barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            xd.copy_(xh, non_blocking=True)
+            out = chain_calls(B, packs, xd, bufs)
+            yh.copy_(out.view(torch.int16), non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e = {"value": world * packed_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
+           "ms_per_step": e2e_ms,
+           "how": "pinned host x -> device, 60 eager bitnet_linear calls through the Python "
+                  "binding, device -> pinned host y; CUDA events"}
+
+    secondary = None
+    if not args.no_secondary and rank == 0:
+        try:
+            secondary = secondary_measurements(B, inputs, torch, dev, stream, pk)
+        except Exception as exc:  # report, never hide
+            secondary = {"error": repr(exc)}
+
+    if rank == 0:
+        cpu = None if args.no_cpu else cpu_baseline(args.cpu_seconds)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic",
+            "config": {"workload": "2B-class decode GEMV chain, M=1: 30 layers x (up [6912,2560], "
+                                   "down [2560,6912]) = 60 distinct 2-bit packed matrices, "
+                                   "each fed the previous bf16 output; one CUDA graph per step",
+                       "M": 1, "matrices": n_launch, "packed_bytes_per_step": packed_bytes,
+                       "l2": "inputs larger than L2 (265 MB packed weights > 126 MB L2), no flush",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+                         "traffic": traffic, "kernel": "gemv_kernel<Linear,1>",
+                         "peak_source": pk["source"],
+                         "algorithmic_bytes_per_launch": alg_bytes,
+                         "launch_us": round(launch_s * 1e6, 3)},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": n_launch * args.steps,
+            "clocks": clocks,
+            "device_status": B.bitnet_status_string(status),
+            "graph_equals_eager": check_ok,
+            "secondary": secondary,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del graph
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
