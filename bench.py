@@ -368,6 +368,31 @@ def secondary_measurements(B, inputs, torch, dev, stream, pk):
     return out
 
 
+def profile_case(case):
+    """A handful of calls of one workload, for ncu (no timing, no output)."""
+    import torch
+    from ternary_weight_linear_int8_b200 import bitnet as B
+    from ternary_weight_linear_int8_b200 import inputs
+    dev = torch.device("cuda", 0)
+    if case == "prefill":
+        M, N, K = 4096, INTER, HIDDEN
+        x = torch.from_numpy(inputs.activations((M, K), seed=0).view(np.int16)).to(dev)
+        W = torch.from_numpy(inputs.weights(N, K, seed=1000)).to(dev)
+        p, g = B.bitnet_pack_weights(W)
+        for _ in range(4):
+            B.bitnet_linear(p, g, x)
+    else:
+        H, I, M = 8192, INTER * 4 + 1024, 2048
+        x = torch.from_numpy(inputs.activations((M, H), seed=0).view(np.int16)).to(dev)
+        ws = [B.bitnet_pack_weights(torch.from_numpy(inputs.weights(n, k, seed=2000 + i)).to(dev))
+              for i, (n, k) in enumerate(((I, H), (I, H), (H, I)))]
+        w = B.FfnWeights(ws[0][0], ws[0][1], ws[1][0], ws[1][1], ws[2][0], ws[2][1])
+        for _ in range(2):
+            B.bitnet_ffn(x, w)
+    torch.cuda.synchronize()
+    return 0 if B.bitnet_last_device_status() == 0 else 1
+
+
 def run_ours(args, world, rank, local):
     import torch
     from ternary_weight_linear_int8_b200 import bitnet as B
@@ -512,10 +537,14 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile-case", choices=["prefill", "ffn2048"], default=None,
+                    help="run a few calls of one workload for an ncu capture, print nothing")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup()
+    if args.profile_case:
+        return profile_case(args.profile_case)
     if args.impl == "reference":
         return run_reference(args, world, rank)
     return run_ours(args, world, rank, local)

@@ -42,6 +42,7 @@ struct GemvArgs {
   int8_t* xq_dbg;         // optional natural-layout x_q [M,K], written by CTA 0
   int rows_per_stage;     // multiple of 4
   int stages;             // 2..8
+  int wk;                 // K-slices per 4-row block
 };
 
 constexpr int kConsumerWarps = 8;
@@ -69,11 +70,47 @@ __device__ __forceinline__ float load_src(const void* x, bool f32, int64_t idx) 
   return bf16_bits_to_float(static_cast<const uint16_t*>(x)[idx]);
 }
 
+// 16 consecutive activations (one group) as floats: two 16-byte loads of
+// bf16 bits, or four of fp32.
+template <bool kF32>
+__device__ __forceinline__ void load_group16(const void* x, int64_t idx, float (&v)[16]) {
+  if (kF32) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + idx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 t = p[i];
+      v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    }
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + idx);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint4 t = p[i];
+      const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+        v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void load_gain16(const float* g, int64_t idx, float (&v)[16]) {
+  const float4* p = reinterpret_cast<const float4*>(g + idx);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 t = p[i];
+    v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+  }
+}
+
 template <int MODE, int MT>
 __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
   constexpr int NMAT = (MODE == kGlu) ? 2 : 1;
   constexpr int NR = 4 * NMAT;             // values per lane per row block
   constexpr bool kF32Src = (MODE == kDown);
+  constexpr int NT = kConsumerWarps * 32;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + 8;
@@ -87,16 +124,20 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
   double* red_d = reinterpret_cast<double*>(smem + 1024);       // [8][8][2]
   const int M = a.M, K = a.K, N = a.N;
   const int Mpad = ((M + MT - 1) / MT) * MT;
+  const int RS = a.rows_per_stage, S = a.stages, WK = a.wk;
   uint8_t* xperm = smem + 2048;
   const int xbytes = ((Mpad * K + 127) / 128) * 128;
-  uint8_t* ring = xperm + xbytes;
+  // per-stage integer accumulators [2 parity][NMAT][RS][kMaxTok]
+  int* acc_s = reinterpret_cast<int*>(xperm + xbytes);
+  const int acc_words = NMAT * RS * kMaxTok;
+  const int acc_bytes = ((2 * acc_words * 4 + 127) / 128) * 128;
+  uint8_t* ring = xperm + xbytes + acc_bytes;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Kb = K >> 2;                   // bytes per packed row
   const int Kw = K >> 4;                   // 32-bit words per packed row
   const int n0 = (int)(((int64_t)blockIdx.x * N) / gridDim.x);
   const int n1 = (int)(((int64_t)(blockIdx.x + 1) * N) / gridDim.x);
-  const int RS = a.rows_per_stage, S = a.stages;
   const int nchunks = (n1 - n0 + RS - 1) / RS;
   const int stage_bytes = RS * Kb * NMAT;
 
@@ -130,34 +171,44 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
   }
 
   // -------------------------------------------------------------- prologue
+  for (int i = tid; i < 2 * acc_words; i += NT) acc_s[i] = 0;
   pdl_wait();
-  // zero the padding tokens of the activation buffer
-  for (int i = M * K + tid * 16; i < Mpad * K; i += kConsumerWarps * 32 * 16)
+  for (int i = M * K + tid * 16; i < Mpad * K; i += NT * 16)
     *reinterpret_cast<uint4*>(xperm + i) = make_uint4(0, 0, 0, 0);
 
+  // pass 1: per-token absmax of src*gain (and, for Down, sums of squares)
   float am[kMaxTok];
   double ss[kMaxTok], sx[kMaxTok];
 #pragma unroll
   for (int m = 0; m < kMaxTok; ++m) { am[m] = 0.f; ss[m] = 0.0; sx[m] = 0.0; }
-  for (int k = tid; k < K; k += kConsumerWarps * 32) {
-    const float g = a.gain ? a.gain[k] : 1.0f;
+#pragma unroll 2
+  for (int g = tid; g < Kw; g += NT) {
+    float gn[16];
+    if (a.gain) load_gain16(a.gain, (int64_t)g * 16, gn);
 #pragma unroll
     for (int m = 0; m < kMaxTok; ++m) {
       if (m < M) {
-        const float v = load_src(a.x, kF32Src, (int64_t)m * K + k);
-        const float vg = a.gain ? __fmul_rn(v, g) : v;
-        am[m] = fmaxf(am[m], fabsf(vg));
-        if (MODE == kDown) ss[m] += (double)v * (double)v;
+        float v[16];
+        load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float vg = a.gain ? __fmul_rn(v[i], gn[i]) : v[i];
+          am[m] = fmaxf(am[m], fabsf(vg));
+          if (MODE == kDown) ss[m] += (double)v[i] * (double)v[i];
+        }
       }
     }
   }
   if (MODE == kDown) {
-    for (int k = tid; k < a.H; k += kConsumerWarps * 32) {
+#pragma unroll 2
+    for (int g = tid; g < (a.H >> 4); g += NT) {
 #pragma unroll
       for (int m = 0; m < kMaxTok; ++m)
         if (m < M) {
-          const double v = (double)bf16_bits_to_float(a.xnorm[(int64_t)m * a.H + k]);
-          sx[m] += v * v;
+          float v[16];
+          load_group16<false>(a.xnorm, (int64_t)m * a.H + g * 16, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) sx[m] += (double)v[i] * (double)v[i];
         }
     }
   }
@@ -201,21 +252,24 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
     }
   }
   consumer_sync();
-  // pass 2: quantise into the permuted layout, group of 16 per thread
+  // pass 2: quantise into the permuted layout, one group of 16 per step
   int rs[kMaxTok];
 #pragma unroll
   for (int m = 0; m < kMaxTok; ++m) rs[m] = 0;
-  for (int g = tid; g < Kw; g += kConsumerWarps * 32) {
+#pragma unroll 2
+  for (int g = tid; g < Kw; g += NT) {
+    float gn[16];
+    if (a.gain) load_gain16(a.gain, (int64_t)g * 16, gn);
 #pragma unroll
     for (int m = 0; m < kMaxTok; ++m) {
       if (m < M) {
         const float s = tok_s[m];
+        float v[16];
+        load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, v);
         int q[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int k = g * 16 + i;
-          const float v = load_src(a.x, kF32Src, (int64_t)m * K + k);
-          const float vg = a.gain ? __fmul_rn(v, a.gain[k]) : v;
+          const float vg = a.gain ? __fmul_rn(v[i], gn[i]) : v[i];
           q[i] = quant_code(vg, s);
           rs[m] += q[i];
         }
@@ -249,122 +303,147 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
   consumer_sync();
 
   // ------------------------------------------------------------- main loop
+  // A stage holds RS whole rows (of each matrix).  Work items are (block of
+  // 4 rows, K-slice) pairs, WK slices per block, dealt to the 8 warps round
+  // robin; each item's per-row totals are added into shared-memory integer
+  // accumulators (exact, order-free), and after a barrier the stage's
+  // outputs are finished from them.
   const uint4* x4 = reinterpret_cast<const uint4*>(xperm);
   bool ok = true;
-  for (int c = 0; c < nchunks && ok; ++c) {
+  for (int c = 0; c < nchunks; ++c) {
     const int s = c % S;
-    if (!mbar_wait(&full[s], (c / S) & 1)) { ok = false; break; }
+    if (ok && !mbar_wait(&full[s], (c / S) & 1)) ok = false;
     const int r0 = n0 + c * RS;
     const int nr = min(RS, n1 - r0);
-    const uint32_t* st = reinterpret_cast<const uint32_t*>(ring + (size_t)s * stage_bytes);
-    const int nblk = (nr + 3) >> 2;
-    for (int b = warp; b < nblk; b += kConsumerWarps) {
-      for (int tg = 0; tg < M; tg += MT) {
-        int acc[NR][MT];
-        int acc4[NR][4];   // MT == 1: one accumulator per code plane
+    int* acc = acc_s + (c & 1) * acc_words;
+    if (ok) {
+      const uint32_t* st = reinterpret_cast<const uint32_t*>(ring + (size_t)s * stage_bytes);
+      const int nitems = ((nr + 3) >> 2) * WK;
+      for (int it = warp; it < nitems; it += kConsumerWarps) {
+        const int b = it / WK, q = it - b * WK;
+        const int j0 = (q * Kw) / WK, j1 = ((q + 1) * Kw) / WK;
+        const uint32_t* rowp[NR];
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
-#pragma unroll
-          for (int t = 0; t < MT; ++t) acc[r][t] = 0;
-#pragma unroll
-          for (int p = 0; p < 4; ++p) acc4[r][p] = 0;
+          const int row = (NMAT == 2) ? (r >> 1) : r;
+          const int mat = (NMAT == 2) ? (r & 1) : 0;
+          rowp[r] = st + (mat * RS + 4 * b + row) * Kw;
         }
-        for (int j = lane; j < Kw; j += 32) {
-          uint32_t w[NR];
+        for (int tg = 0; tg < M; tg += MT) {
+          int acc_r[NR][MT];
+          int acc4[NR][4];   // MT == 1: one accumulator per code plane
 #pragma unroll
           for (int r = 0; r < NR; ++r) {
-            // value index r = 2*row + mat for Glu, = row otherwise
-            const int row = (NMAT == 2) ? (r >> 1) : r;
-            const int mat = (NMAT == 2) ? (r & 1) : 0;
-            w[r] = st[(size_t)(mat * RS + 4 * b + row) * Kw + j];
+#pragma unroll
+            for (int t = 0; t < MT; ++t) acc_r[r][t] = 0;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) acc4[r][p] = 0;
           }
-          uint4 xv[MT];
+          const uint4* xt = x4 + tg * Kw;
+#pragma unroll 2
+          for (int j = j0 + lane; j < j1; j += 32) {
+            uint32_t w[NR];
 #pragma unroll
-          for (int t = 0; t < MT; ++t) xv[t] = x4[(size_t)(tg + t) * Kw + j];
+            for (int r = 0; r < NR; ++r) w[r] = rowp[r][j];
+            uint4 xv[MT];
 #pragma unroll
-          for (int r = 0; r < NR; ++r) {
-            if (MT == 1) {
-              acc4[r][0] = dp4a_su((int)xv[0].x, w[r] & 0x03030303u, acc4[r][0]);
-              acc4[r][1] = dp4a_su((int)xv[0].y, w[r] & 0x0c0c0c0cu, acc4[r][1]);
-              acc4[r][2] = dp4a_su((int)xv[0].z, w[r] & 0x30303030u, acc4[r][2]);
-              acc4[r][3] = dp4a_su((int)xv[0].w, w[r] & 0xc0c0c0c0u, acc4[r][3]);
-            } else {
-              const uint32_t c0 = w[r] & 0x03030303u;
-              const uint32_t c1 = (w[r] >> 2) & 0x03030303u;
-              const uint32_t c2 = (w[r] >> 4) & 0x03030303u;
-              const uint32_t c3 = (w[r] >> 6) & 0x03030303u;
+            for (int t = 0; t < MT; ++t) xv[t] = xt[t * Kw + j];
 #pragma unroll
-              for (int t = 0; t < MT; ++t) {
-                int v = acc[r][t];
-                v = dp4a_su((int)xv[t].x, c0, v);
-                v = dp4a_su((int)xv[t].y, c1, v);
-                v = dp4a_su((int)xv[t].z, c2, v);
-                v = dp4a_su((int)xv[t].w, c3, v);
-                acc[r][t] = v;
+            for (int r = 0; r < NR; ++r) {
+              if constexpr (MT == 1) {
+                acc4[r][0] = dp4a_su((int)xv[0].x, w[r] & 0x03030303u, acc4[r][0]);
+                acc4[r][1] = dp4a_su((int)xv[0].y, w[r] & 0x0c0c0c0cu, acc4[r][1]);
+                acc4[r][2] = dp4a_su((int)xv[0].z, w[r] & 0x30303030u, acc4[r][2]);
+                acc4[r][3] = dp4a_su((int)xv[0].w, w[r] & 0xc0c0c0c0u, acc4[r][3]);
+              } else {
+                const uint32_t c0 = w[r] & 0x03030303u;
+                const uint32_t c1 = (w[r] >> 2) & 0x03030303u;
+                const uint32_t c2 = (w[r] >> 4) & 0x03030303u;
+                const uint32_t c3 = (w[r] >> 6) & 0x03030303u;
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                  int v = acc_r[r][t];
+                  v = dp4a_su((int)xv[t].x, c0, v);
+                  v = dp4a_su((int)xv[t].y, c1, v);
+                  v = dp4a_su((int)xv[t].z, c2, v);
+                  v = dp4a_su((int)xv[t].w, c3, v);
+                  acc_r[r][t] = v;
+                }
               }
             }
           }
-        }
-        if (MT == 1) {
+          if constexpr (MT == 1) {
 #pragma unroll
-          for (int r = 0; r < NR; ++r)
-            acc[r][0] = acc4[r][0] + (acc4[r][1] >> 2) + (acc4[r][2] >> 4) + (acc4[r][3] >> 6);
-        }
-        // butterfly: lane l ends with value index (l >> 32/NR-bits) summed
-#pragma unroll
-        for (int t = 0; t < MT; ++t) {
-          int v[NR];
-#pragma unroll
-          for (int r = 0; r < NR; ++r) v[r] = acc[r][t];
-          int tot;
-          if constexpr (NR == 4) {
-            int h2[2], h1[1];
-            halve<4>(*reinterpret_cast<int(*)[4]>(v), h2, 16, lane);
-            halve<2>(h2, h1, 8, lane);
-            tot = h1[0];
-            tot += __shfl_xor_sync(0xffffffffu, tot, 4);
-            tot += __shfl_xor_sync(0xffffffffu, tot, 2);
-            tot += __shfl_xor_sync(0xffffffffu, tot, 1);
-          } else {
-            int h4[4], h2[2], h1[1];
-            halve<8>(*reinterpret_cast<int(*)[8]>(v), h4, 16, lane);
-            halve<4>(h4, h2, 8, lane);
-            halve<2>(h2, h1, 4, lane);
-            tot = h1[0];
-            tot += __shfl_xor_sync(0xffffffffu, tot, 2);
-            tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+            for (int r = 0; r < NR; ++r)
+              acc_r[r][0] = acc4[r][0] + (acc4[r][1] >> 2) + (acc4[r][2] >> 4) + (acc4[r][3] >> 6);
           }
-          int other = 0;
-          if (NMAT == 2) other = __shfl_xor_sync(0xffffffffu, tot, 4);   // up total
-          const int m = tg + t;
-          const int row = lane >> 3;                    // 0..3
-          const bool writer = (lane & 7) == 0;
-          const int n = r0 + 4 * b + row;
-          if (writer && m < M && 4 * b + row < nr) {
-            const int64_t o = (int64_t)m * N + n;
-            const int rsum = tok_rs[m];
-            if (MODE == kGlu) {
-              const int ag = tot - rsum, au = other - rsum;
-              const float g = __fmul_rn(__int2float_rn(ag), tok_d0[m]);
-              const float u = __fmul_rn(__int2float_rn(au), tok_d1[m]);
-              const float rg = fmaxf(g, 0.0f);
-              a.h[o] = __fmul_rn(__fmul_rn(rg, rg), u);
-              if (a.acc0) a.acc0[o] = ag;
-              if (a.acc1) a.acc1[o] = au;
+#pragma unroll
+          for (int t = 0; t < MT; ++t) {
+            int v[NR];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) v[r] = acc_r[r][t];
+            int tot;
+            int row, mat;
+            bool writer;
+            if constexpr (NR == 4) {
+              int h2[2], h1[1];
+              halve<4>(v, h2, 16, lane);
+              halve<2>(h2, h1, 8, lane);
+              tot = h1[0];
+              tot += __shfl_xor_sync(0xffffffffu, tot, 4);
+              tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+              tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+              row = lane >> 3; mat = 0; writer = (lane & 7) == 0;
             } else {
-              const int ac = tot - rsum;
-              float y32 = __fmul_rn(__int2float_rn(ac), tok_d0[m]);
-              if (MODE == kDown) y32 = __fmul_rn(y32, tok_f[m]);
-              a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
-              if (a.y_f32) a.y_f32[o] = y32;
-              if (a.acc0) a.acc0[o] = ac;
+              int h4[4], h2[2], h1[1];
+              halve<8>(v, h4, 16, lane);
+              halve<4>(h4, h2, 8, lane);
+              halve<2>(h2, h1, 4, lane);
+              tot = h1[0];
+              tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+              tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+              row = lane >> 3; mat = (lane >> 2) & 1; writer = (lane & 3) == 0;
             }
+            const int m = tg + t;
+            if (writer && m < M && 4 * b + row < nr)
+              atomicAdd(&acc[(mat * RS + 4 * b + row) * kMaxTok + m], tot);
           }
         }
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
+    consumer_sync();
+    // finish this stage's outputs; clear the accumulators for stage c + 2
+    for (int o = tid; o < nr * M; o += NT) {
+      const int row = o / M, m = o - row * M;
+      const int n = r0 + row;
+      const int64_t oo = (int64_t)m * N + n;
+      const int rsum = tok_rs[m];
+      int* p0 = &acc[row * kMaxTok + m];
+      if (MODE == kGlu) {
+        int* p1 = &acc[(RS + row) * kMaxTok + m];
+        const int ag = *p0 - rsum, au = *p1 - rsum;
+        *p0 = 0;
+        *p1 = 0;
+        const float g = __fmul_rn(__int2float_rn(ag), tok_d0[m]);
+        const float u = __fmul_rn(__int2float_rn(au), tok_d1[m]);
+        const float rg = fmaxf(g, 0.0f);
+        if (ok) a.h[oo] = __fmul_rn(__fmul_rn(rg, rg), u);
+        if (ok && a.acc0) a.acc0[oo] = ag;
+        if (ok && a.acc1) a.acc1[oo] = au;
+      } else {
+        const int ac = *p0 - rsum;
+        *p0 = 0;
+        float y32 = __fmul_rn(__int2float_rn(ac), tok_d0[m]);
+        if (MODE == kDown) y32 = __fmul_rn(y32, tok_f[m]);
+        if (ok) {
+          a.y[oo] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+          if (a.y_f32) a.y_f32[oo] = y32;
+          if (a.acc0) a.acc0[oo] = ac;
+        }
+      }
+    }
   }
 }
 
@@ -395,31 +474,49 @@ static cudaError_t launch_one(const GemvArgs& a, int grid, size_t smem, cudaStre
 // Host-side planning: stage rows and ring depth under a shared-memory budget
 // that leaves room for a second CTA per SM (the next kernel in the stream).
 struct GemvPlan {
-  int grid, rows_per_stage, stages;
+  int grid, rows_per_stage, stages, wk;
   size_t smem;
 };
+
+// K-slices per row block: balance (blocks x slices) items over the 8 warps
+// against the per-item reduction cost (about half a 32-word step).
+static int pick_wk(int nb, int Kw) {
+  int best = 1;
+  double best_cost = 1e30;
+  for (int wk = 1; wk <= 32; wk *= 2) {
+    if (wk > 1 && Kw / wk < 8) break;
+    const double rounds = (double)((nb * wk + kConsumerWarps - 1) / kConsumerWarps);
+    const double iters = (double)((Kw / wk + 31) / 32);
+    const double cost = rounds * (iters + 0.5);
+    if (cost < best_cost - 1e-9) { best_cost = cost; best = wk; }
+  }
+  return best;
+}
 
 static GemvPlan plan_gemv(int M, int N, int K, int nmat, int num_sms, int MT) {
   GemvPlan p{};
   const int Mpad = ((M + MT - 1) / MT) * MT;
   const size_t xbytes = (((size_t)Mpad * K + 127) / 128) * 128;
   const size_t budget = 112 * 1024;
-  const size_t head = 2048 + xbytes;
   const size_t row_bytes = (size_t)(K / 4) * nmat;
   int blocks = (N + 3) / 4;
   p.grid = blocks < num_sms ? blocks : num_sms;
   const int rows_per_cta = (N + p.grid - 1) / p.grid;
-  const size_t ring = budget > head + 2 * 4 * row_bytes ? budget - head : 2 * 4 * row_bytes;
   int rs = (int)((32 * 1024) / row_bytes);
   rs = rs / 4 * 4;
   if (rs < 4) rs = 4;
   const int rows_cap = (rows_per_cta + 3) / 4 * 4;
   if (rs > rows_cap) rs = rows_cap;
+  const size_t acc_bytes = ((2 * (size_t)nmat * rs * kMaxTok * 4 + 127) / 128) * 128;
+  const size_t head = 2048 + xbytes + acc_bytes;
+  const size_t ring = budget > head + 2 * (size_t)rs * row_bytes ? budget - head
+                                                                  : 2 * (size_t)rs * row_bytes;
   int st = (int)(ring / ((size_t)rs * row_bytes));
   if (st > 8) st = 8;
   if (st < 2) st = 2;
   p.rows_per_stage = rs;
   p.stages = st;
+  p.wk = pick_wk(rs / 4, K / 16);
   p.smem = head + (size_t)st * rs * row_bytes;
   return p;
 }
@@ -440,6 +537,7 @@ bitnet_status bitnet_gemv_launch(int mode, GemvArgs a, int num_sms, cudaStream_t
   if (p.smem > 227 * 1024) return BITNET_ERR_UNSUPPORTED;
   a.rows_per_stage = p.rows_per_stage;
   a.stages = p.stages;
+  a.wk = p.wk;
   cudaError_t e = cudaErrorInvalidValue;
 #define BITNET_GEMV_CASE(MODE_)                                                       \
   if (mode == MODE_) {                                                                \
