@@ -382,7 +382,7 @@ def profile_case(case):
         for _ in range(4):
             B.bitnet_linear(p, g, x)
     else:
-        H, I, M = 8192, INTER * 4 + 1024, 2048
+        H, I, M = 8192, 28672, 2048
         x = torch.from_numpy(inputs.activations((M, H), seed=0).view(np.int16)).to(dev)
         ws = [B.bitnet_pack_weights(torch.from_numpy(inputs.weights(n, k, seed=2000 + i)).to(dev))
               for i, (n, k) in enumerate(((I, H), (I, H), (H, I)))]
