@@ -17,7 +17,8 @@ bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* ga
                                   cudaStream_t stream);
 bitnet_status bitnet_gemv_launch(int mode, GemvArgs a, int num_sms, cudaStream_t stream);
 bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
-                                 const uint8_t* w1, GemmArgs a, int bn, cudaStream_t stream);
+                                 const uint8_t* w1, GemmArgs a, int bn, int num_sms,
+                                 cudaStream_t stream);
 int bitnet_gemm_pick_bn(int M);
 
 namespace {
@@ -267,7 +268,7 @@ bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N
     a.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc);
     if (cudaMemsetAsync(a.acc_ws0, 0, (size_t)M * N * 4, s) != cudaSuccess) return BITNET_ERR_CUDA;
   }
-  return bitnet_gemm_launch(0 /*linear*/, xq, packed, nullptr, a, bn, s);
+  return bitnet_gemm_launch(0 /*linear*/, xq, packed, nullptr, a, bn, d.num_sms, s);
 }
 
 size_t bitnet_ffn_workspace_size(int64_t M, int64_t H, int64_t I) {
@@ -340,7 +341,7 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
         cudaMemsetAsync(g.acc_ws1, 0, (size_t)M * I * 4, s) != cudaSuccess)
       return BITNET_ERR_CUDA;
   }
-  st = bitnet_gemm_launch(1 /*glu*/, xq1, gate, up, g, bn, s);
+  st = bitnet_gemm_launch(1 /*glu*/, xq1, gate, up, g, bn, d.num_sms, s);
   if (st != BITNET_OK) return st;
   st = bitnet_quant_launch(hbuf, true, norm2_w, M, I, xq2, I, true, s2, rs2, ss2, dbg.xq2, s);
   if (st != BITNET_OK) return st;
@@ -354,7 +355,7 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
     dn.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
     if (cudaMemsetAsync(dn.acc_ws0, 0, (size_t)M * H * 4, s) != cudaSuccess) return BITNET_ERR_CUDA;
   }
-  return bitnet_gemm_launch(2 /*down*/, xq2, down, nullptr, dn, bn, s);
+  return bitnet_gemm_launch(2 /*down*/, xq2, down, nullptr, dn, bn, d.num_sms, s);
 }
 
 bitnet_status bitnet_last_device_status(void* stream) {

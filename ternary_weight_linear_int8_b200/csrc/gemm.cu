@@ -52,7 +52,7 @@ struct GemmArgs {
 
 constexpr int kBM = 128;                 // features per tile (MMA M)
 constexpr int kBK = 128;                 // K elements (bytes) per stage
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;        // 10 warps: TMA, MMA, 4 unpack, 4 epilogue
 
 template <int BN, int NMAT>
 struct GemmCfg {
@@ -60,9 +60,11 @@ struct GemmCfg {
   static constexpr int kA = kBM * kBK;                // one unpacked weight tile
   static constexpr int kP = kBM * (kBK / 4);          // one packed weight tile
   static constexpr int kStage = kB + NMAT * (kA + kP);
-  static constexpr int kStages0 = (220 * 1024) / kStage;
+  static constexpr int kStages0 = (218 * 1024) / kStage;
   static constexpr int kStages = kStages0 > 6 ? 6 : (kStages0 < 2 ? 2 : kStages0);
-  static constexpr int kCols0 = NMAT * BN;
+  // accumulator sets in TMEM (512 columns): two when they fit
+  static constexpr int kAcc = (2 * NMAT * BN <= 512) ? 2 : 1;
+  static constexpr int kCols0 = kAcc * NMAT * BN;
   static constexpr int kTmemCols = kCols0 <= 32 ? 32 : kCols0 <= 64 ? 64 : kCols0 <= 128 ? 128
                                  : kCols0 <= 256 ? 256 : 512;
   static constexpr int kAux = 1024;                   // barriers + tmem slot
@@ -124,12 +126,17 @@ __device__ __forceinline__ void epi_sync() {
   asm volatile("bar.sync 2, 128;" ::: "memory");
 }
 
+// Persistent: each CTA walks work units (feature tile, token tile, K split)
+// with stride gridDim.x.  The stage ring and its barrier phases run on across
+// units; TMEM holds NACC accumulator sets so the epilogue warps drain unit i
+// while the MMA warp already accumulates unit i + 1.
 template <int MODE, int BN, int NMAT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw0,
                 const __grid_constant__ CUtensorMap tw1, const GemmArgs a) {
   using C = GemmCfg<BN, NMAT>;
   constexpr int S = C::kStages;
+  constexpr int NACC = C::kAcc;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles
   const uint32_t raw = smem_u32(smem_raw);
@@ -138,19 +145,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tma_full = reinterpret_cast<uint64_t*>(aux);
   uint64_t* a_full = tma_full + S;
   uint64_t* mma_done = a_full + S;
-  uint64_t* accum_full = mma_done + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_full + 1);
+  uint64_t* acc_full = mma_done + S;         // [NACC]
+  uint64_t* acc_empty = acc_full + NACC;     // [NACC]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + NACC);
   float* tok_d0 = reinterpret_cast<float*>(aux + C::kAux);
   float* tok_d1 = tok_d0 + BN;
   float* tok_f = tok_d1 + BN;
   int* tok_rs = reinterpret_cast<int*>(tok_f + BN);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_tile = blockIdx.x, m_tile = blockIdx.y;
+  const int n_tiles = (a.N + kBM - 1) / kBM;
+  const int m_tiles = (a.M + BN - 1) / BN;
+  const int units = n_tiles * m_tiles * a.ksplit;
   const int kst = (a.K + kBK - 1) / kBK;
-  const int k0 = (int)(((int64_t)blockIdx.z * kst) / a.ksplit);
-  const int k1 = (int)(((int64_t)(blockIdx.z + 1) * kst) / a.ksplit);
-  const int nk = k1 - k0;
+
+  // unit -> (n_tile, m_tile, kz); feature tiles vary fastest so that the
+  // CTAs running at one time share token tiles in L2
+  auto decode_unit = [&](int unit, int& nt, int& mt, int& k0, int& nk) {
+    nt = unit % n_tiles;
+    const int rest = unit / n_tiles;
+    mt = rest % m_tiles;
+    const int kz = rest / m_tiles;
+    k0 = (int)(((int64_t)kz * kst) / a.ksplit);
+    nk = (int)(((int64_t)(kz + 1) * kst) / a.ksplit) - k0;
+  };
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -158,7 +176,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&a_full[s], 4);
       mbar_init(&mma_done[s], 1);
     }
-    mbar_init(accum_full, 1);
+    for (int b = 0; b < NACC; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
     fence_mbar_init();
     prefetch_tmap(&tx);
     prefetch_tmap(&tw0);
@@ -183,141 +204,154 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint64_t pol_w = policy_evict_normal();
       const uint64_t pol_x = policy_evict_last();
       const uint32_t bytes = (uint32_t)(C::kB + NMAT * C::kP);
-      // weights do not depend on the previous kernel: prefetch the first
-      // stages before waiting for it, then add the activation tiles.
-      const int pre = nk < S ? nk : S;
-      for (int u = 0; u < pre; ++u) {
-        uint8_t* st = smem + (size_t)u * C::kStage;
-        const int kx = (k0 + u) * kBK;
-        mbar_arrive_expect_tx(&tma_full[u], bytes);
-        tma_load_2d(st + C::kB + NMAT * C::kA, &tw0, &tma_full[u], kx / 4, n_tile * kBM, pol_w);
-        if (NMAT == 2)
-          tma_load_2d(st + C::kB + NMAT * C::kA + C::kP, &tw1, &tma_full[u], kx / 4,
-                      n_tile * kBM, pol_w);
-      }
-      pdl_wait();
-      for (int u = 0; u < pre; ++u) {
-        uint8_t* st = smem + (size_t)u * C::kStage;
-        tma_load_2d(st, &tx, &tma_full[u], (k0 + u) * kBK, m_tile * BN, pol_x);
-      }
-      for (int u = pre; u < nk; ++u) {
-        const int s = u % S;
-        if (!mbar_wait(&mma_done[s], ((u / S) - 1) & 1)) break;
-        uint8_t* st = smem + (size_t)s * C::kStage;
-        const int kx = (k0 + u) * kBK;
-        mbar_arrive_expect_tx(&tma_full[s], bytes);
-        tma_load_2d(st, &tx, &tma_full[s], kx, m_tile * BN, pol_x);
-        tma_load_2d(st + C::kB + NMAT * C::kA, &tw0, &tma_full[s], kx / 4, n_tile * kBM, pol_w);
-        if (NMAT == 2)
-          tma_load_2d(st + C::kB + NMAT * C::kA + C::kP, &tw1, &tma_full[s], kx / 4,
-                      n_tile * kBM, pol_w);
+      bool waited = false;
+      int u = 0;                               // running stage counter
+      for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
+        int nt, mt, k0, nk;
+        decode_unit(unit, nt, mt, k0, nk);
+        for (int kk = 0; kk < nk; ++kk, ++u) {
+          const int s = u % S;
+          if (u >= S && !mbar_wait(&mma_done[s], ((u / S) - 1) & 1)) { u = -1; break; }
+          uint8_t* st = smem + (size_t)s * C::kStage;
+          const int kx = (k0 + kk) * kBK;
+          mbar_arrive_expect_tx(&tma_full[s], bytes);
+          // weights never depend on the previous kernel: load them first
+          tma_load_2d(st + C::kB + NMAT * C::kA, &tw0, &tma_full[s], kx / 4, nt * kBM, pol_w);
+          if (NMAT == 2)
+            tma_load_2d(st + C::kB + NMAT * C::kA + C::kP, &tw1, &tma_full[s], kx / 4, nt * kBM,
+                        pol_w);
+          if (!waited) { pdl_wait(); waited = true; }
+          tma_load_2d(st, &tx, &tma_full[s], kx, mt * BN, pol_x);
+        }
+        if (u < 0) break;
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
       bool ok = true;
-      for (int u = 0; u < nk && ok; ++u) {
-        const int s = u % S;
-        const uint32_t ph = (u / S) & 1;
-        ok = mbar_wait(&a_full[s], ph) && mbar_wait(&tma_full[s], ph);
-        if (!ok) break;
+      int u = 0, i = 0;
+      for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x, ++i) {
+        int nt, mt, k0, nk;
+        decode_unit(unit, nt, mt, k0, nk);
+        const int ab = i % NACC;
+        if (i >= NACC && !mbar_wait(&acc_empty[ab], ((i / NACC) - 1) & 1)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t dt = tmem + (uint32_t)(ab * NMAT * BN);
+        for (int kk = 0; kk < nk; ++kk, ++u) {
+          const int s = u % S;
+          const uint32_t ph = (u / S) & 1;
+          ok = mbar_wait(&a_full[s], ph) && mbar_wait(&tma_full[s], ph);
+          if (!ok) break;
+          tc_fence_after();
+          uint8_t* st = smem + (size_t)s * C::kStage;
+          const uint64_t bdesc = sw128_desc(smem_u32(st));
+#pragma unroll
+          for (int mat = 0; mat < NMAT; ++mat) {
+            const uint64_t adesc = sw128_desc(smem_u32(st + C::kB + mat * C::kA));
+#pragma unroll
+            for (int q = 0; q < kBK / 32; ++q) {
+              // advance 32 bytes of K inside the swizzle atom: +2 in 16-byte units
+              tc_mma_i8(dt + mat * BN, adesc + 2 * q, bdesc + 2 * q, C::kIdesc,
+                        (kk > 0 || q > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit(&mma_done[s]);
+        }
+        tc_commit(&acc_full[ab]);
+      }
+    }
+  } else if (warp < 6) {
+    // ---------------------------------------------------- unpack warps
+    const int ut = tid - 64;                 // 0..127: one weight row each
+    int u = 0;
+    bool ok = true;
+    for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
+      int nt, mt, k0, nk;
+      decode_unit(unit, nt, mt, k0, nk);
+      for (int kk = 0; kk < nk; ++kk, ++u) {
+        const int s = u % S;
+        if (!mbar_wait(&tma_full[s], (u / S) & 1)) { ok = false; break; }
         uint8_t* st = smem + (size_t)s * C::kStage;
-        const uint64_t bdesc = sw128_desc(smem_u32(st));
 #pragma unroll
         for (int mat = 0; mat < NMAT; ++mat) {
-          const uint64_t adesc = sw128_desc(smem_u32(st + C::kB + mat * C::kA));
+          const uint4* pk = reinterpret_cast<const uint4*>(st + C::kB + NMAT * C::kA +
+                                                           mat * C::kP + ut * (kBK / 4));
+          const uint4 p0 = pk[0], p1 = pk[1];
+          const uint32_t wv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+          uint8_t* arow = st + C::kB + mat * C::kA + ut * kBK;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 32; ++kk) {
-            // advance 32 bytes of K inside the swizzle atom: +2 in 16-byte units
-            tc_mma_i8(tmem + mat * BN, adesc + 2 * kk, bdesc + 2 * kk, C::kIdesc,
-                      (u > 0 || kk > 0) ? 1u : 0u);
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t w = wv[j];
+            const uint4 o = make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u,
+                                       (w >> 4) & 0x03030303u, (w >> 6) & 0x03030303u);
+            *reinterpret_cast<uint4*>(arow + ((j ^ (ut & 7)) << 4)) = o;
           }
         }
-        tc_commit(&mma_done[s]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[s]);
       }
-      tc_commit(accum_full);
     }
   } else {
-    // ------------------------------------- unpack (then epilogue) warps
-    const int ut = tid - 64;                 // 0..127: one weight row each
-    bool ok = true;
-    for (int u = 0; u < nk; ++u) {
-      const int s = u % S;
-      if (!mbar_wait(&tma_full[s], (u / S) & 1)) { ok = false; break; }
-      uint8_t* st = smem + (size_t)s * C::kStage;
-#pragma unroll
-      for (int mat = 0; mat < NMAT; ++mat) {
-        const uint4* pk = reinterpret_cast<const uint4*>(st + C::kB + NMAT * C::kA + mat * C::kP +
-                                                         ut * (kBK / 4));
-        const uint4 p0 = pk[0], p1 = pk[1];
-        const uint32_t wv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        uint8_t* arow = st + C::kB + mat * C::kA + ut * kBK;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t w = wv[j];
-          const uint4 o = make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u,
-                                     (w >> 4) & 0x03030303u, (w >> 6) & 0x03030303u);
-          *reinterpret_cast<uint4*>(arow + ((j ^ (ut & 7)) << 4)) = o;
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[s]);
-    }
-
     // --------------------------------------------------------- epilogue
     pdl_wait();
-    const int et = ut;                       // 0..127
-    for (int c = et; c < BN; c += 128) {
-      const int tok = m_tile * BN + c;
-      float d0 = 0.f, d1 = 0.f, f = 0.f;
-      int rs = 0;
-      if (tok < a.M) {
-        const float s = a.scale[tok];
-        d0 = __fdiv_rn(*a.gamma0, s);
-        if (MODE == gGlu) d1 = __fdiv_rn(*a.gamma1, s);
-        rs = a.rowsum[tok];
-        if (MODE == gDown) {
-          const double eps = (double)a.eps;
-          const double r1 = 1.0 / sqrt(a.sumsq_x[tok] / (double)a.H + eps);
-          const double r1_3 = r1 * r1 * r1;
-          const double r2 = 1.0 / sqrt(r1_3 * r1_3 * (a.sumsq_h[tok] / (double)a.K) + eps);
-          f = (float)(r1_3 * r2);
+    const int et = tid - 192;                // 0..127
+    const int lb = 32 * (warp & 3);          // TMEM lanes this warp may access
+    int i = 0;
+    for (int unit = blockIdx.x; unit < units; unit += gridDim.x, ++i) {
+      int nt, mt, k0, nk;
+      decode_unit(unit, nt, mt, k0, nk);
+      const int ab = i % NACC;
+      if (a.ksplit == 1) {
+        epi_sync();                          // previous unit's scalars are consumed
+        for (int c = et; c < BN; c += 128) {
+          const int tok = mt * BN + c;
+          float d0 = 0.f, d1 = 0.f, f = 0.f;
+          int rs = 0;
+          if (tok < a.M) {
+            const float s = a.scale[tok];
+            d0 = __fdiv_rn(*a.gamma0, s);
+            if (MODE == gGlu) d1 = __fdiv_rn(*a.gamma1, s);
+            rs = a.rowsum[tok];
+            if (MODE == gDown) {
+              const double eps = (double)a.eps;
+              const double r1 = 1.0 / sqrt(a.sumsq_x[tok] / (double)a.H + eps);
+              const double r1_3 = r1 * r1 * r1;
+              const double r2 = 1.0 / sqrt(r1_3 * r1_3 * (a.sumsq_h[tok] / (double)a.K) + eps);
+              f = (float)(r1_3 * r2);
+            }
+          }
+          tok_d0[c] = d0;
+          tok_d1[c] = d1;
+          tok_f[c] = f;
+          tok_rs[c] = rs;
         }
+        epi_sync();
       }
-      tok_d0[c] = d0;
-      tok_d1[c] = d1;
-      tok_f[c] = f;
-      tok_rs[c] = rs;
-    }
-    epi_sync();
-    if (ok && !mbar_wait(accum_full, 0)) ok = false;
-    tc_fence_after();
-    if (ok) {
-      const int lb = 32 * (warp & 3);        // TMEM lanes this warp may access
-      const int n = n_tile * kBM + lb + lane;
-      const uint32_t tbase = tmem + ((uint32_t)lb << 16);
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      const bool ok = mbar_wait(&acc_full[ab], (i / NACC) & 1);
+      tc_fence_after();
+      const int n = nt * kBM + lb + lane;
+      const uint32_t tbase = tmem + ((uint32_t)lb << 16) + (uint32_t)(ab * NMAT * BN);
+      for (int c0 = 0; c0 < BN && ok; c0 += 32) {
         uint32_t v0[32], v1[32];
         tmem_ld32(tbase + c0, v0);
         if (NMAT == 2) tmem_ld32(tbase + BN + c0, v1);
         if (n < a.N) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int c = c0 + i;
-            const int tok = m_tile * BN + c;
+          for (int q = 0; q < 32; ++q) {
+            const int c = c0 + q;
+            const int tok = mt * BN + c;
             if (tok >= a.M) continue;
             const int64_t o = (int64_t)tok * a.N + n;
             if (a.ksplit > 1) {
-              atomicAdd(&a.acc_ws0[o], (int)v0[i]);
-              if (NMAT == 2) atomicAdd(&a.acc_ws1[o], (int)v1[i]);
+              atomicAdd(&a.acc_ws0[o], (int)v0[q]);
+              if (NMAT == 2) atomicAdd(&a.acc_ws1[o], (int)v1[q]);
               continue;
             }
-            const int ac = (int)v0[i] - tok_rs[c];
+            const int ac = (int)v0[q] - tok_rs[c];
             if (MODE == gGlu) {
-              const int au = (int)v1[i] - tok_rs[c];
+              const int au = (int)v1[q] - tok_rs[c];
               const float g = __fmul_rn(__int2float_rn(ac), tok_d0[c]);
               const float uu = __fmul_rn(__int2float_rn(au), tok_d1[c]);
               const float rg = fmaxf(g, 0.0f);
@@ -334,13 +368,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    // every MMA has completed once accum_full has (it is committed last)
-    mbar_wait(accum_full, 0);
+    // every MMA has completed once the last accumulator set was committed
+    // and drained (the epilogue waited on it); wait on the final commit too
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
@@ -465,7 +502,8 @@ int bitnet_gemm_pick_bn(int M) {
 // Launch the tensor-core kernel (and, with ksplit > 1, its finaliser).
 // xq: [M, K] int8 in the permuted K order; w0/w1: packed [N, K/4].
 bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
-                                 const uint8_t* w1, GemmArgs a, int bn, cudaStream_t stream) {
+                                 const uint8_t* w1, GemmArgs a, int bn, int num_sms,
+                                 cudaStream_t stream) {
   CUtensorMap tx, tw0, tw1;
   const int nmat = mode == gGlu ? 2 : 1;
   if (!make_map_u8(&tx, xq, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, kBK, (uint32_t)bn, true))
@@ -480,7 +518,8 @@ bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
   } else {
     tw1 = tw0;
   }
-  dim3 grid((a.N + kBM - 1) / kBM, (a.M + bn - 1) / bn, a.ksplit);
+  const int64_t units = (int64_t)((a.N + kBM - 1) / kBM) * ((a.M + bn - 1) / bn) * a.ksplit;
+  dim3 grid((unsigned)(units < num_sms ? units : num_sms));
   cudaError_t e = cudaErrorInvalidValue;
 #define BITNET_GEMM_BN(MODE_, NMAT_)                                              \
   switch (bn) {                                                                   \

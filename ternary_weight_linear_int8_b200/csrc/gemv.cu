@@ -105,8 +105,10 @@ __device__ __forceinline__ void load_gain16(const float* g, int64_t idx, float (
   }
 }
 
-template <int MODE, int MT>
+template <int MODE, int MT, int MM>
 __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
+  // MM: token count rounded up to 1, 2, 4 or 8 (loops over tokens unroll to
+  // MM, keeping the code small for single-token decode)
   constexpr int NMAT = (MODE == kGlu) ? 2 : 1;
   constexpr int NR = 4 * NMAT;             // values per lane per row block
   constexpr bool kF32Src = (MODE == kDown);
@@ -177,16 +179,16 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
     *reinterpret_cast<uint4*>(xperm + i) = make_uint4(0, 0, 0, 0);
 
   // pass 1: per-token absmax of src*gain (and, for Down, sums of squares)
-  float am[kMaxTok];
-  double ss[kMaxTok], sx[kMaxTok];
+  float am[MM];
+  double ss[MM], sx[MM];
 #pragma unroll
-  for (int m = 0; m < kMaxTok; ++m) { am[m] = 0.f; ss[m] = 0.0; sx[m] = 0.0; }
+  for (int m = 0; m < MM; ++m) { am[m] = 0.f; ss[m] = 0.0; sx[m] = 0.0; }
 #pragma unroll 2
   for (int g = tid; g < Kw; g += NT) {
     float gn[16];
     if (a.gain) load_gain16(a.gain, (int64_t)g * 16, gn);
 #pragma unroll
-    for (int m = 0; m < kMaxTok; ++m) {
+    for (int m = 0; m < MM; ++m) {
       if (m < M) {
         float v[16];
         load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, v);
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
 #pragma unroll 2
     for (int g = tid; g < (a.H >> 4); g += NT) {
 #pragma unroll
-      for (int m = 0; m < kMaxTok; ++m)
+      for (int m = 0; m < MM; ++m)
         if (m < M) {
           float v[16];
           load_group16<false>(a.xnorm, (int64_t)m * a.H + g * 16, v);
@@ -213,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
     }
   }
 #pragma unroll
-  for (int m = 0; m < kMaxTok; ++m) {
+  for (int m = 0; m < MM; ++m) {
     if (m < M) {
       const float w = warp_max(am[m]);
       if (lane == 0) red_f[warp * kMaxTok + m] = w;
@@ -228,22 +230,29 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
     }
   }
   consumer_sync();
+  // every thread derives the token scales from the 8 warp maxima itself
+  // (same values, same order -> identical in every thread)
+  float sc[MM];
+#pragma unroll
+  for (int m = 0; m < MM; ++m) {
+    float amax = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) amax = fmaxf(amax, red_f[w * kMaxTok + m]);
+    sc[m] = qscale(amax);
+  }
   if (tid < M) {
     const int m = tid;
-    float amax = 0.f;
-    double s1 = 0.0, s2 = 0.0;
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      amax = fmaxf(amax, red_f[w * kMaxTok + m]);
-      if (MODE == kDown) {
-        s1 += red_d[(w * kMaxTok + m) * 2 + 0];
-        s2 += red_d[(w * kMaxTok + m) * 2 + 1];
-      }
-    }
-    const float s = qscale(amax);
-    tok_s[m] = s;
+    float s = sc[0];
+#pragma unroll
+    for (int mm = 1; mm < MM; ++mm) if (mm == m) s = sc[mm];
     tok_d0[m] = __fdiv_rn(*a.gamma0, s);
     if (MODE == kGlu) tok_d1[m] = __fdiv_rn(*a.gamma1, s);
     if (MODE == kDown) {
+      double s1 = 0.0, s2 = 0.0;
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        s1 += red_d[(w * kMaxTok + m) * 2 + 0];
+        s2 += red_d[(w * kMaxTok + m) * 2 + 1];
+      }
       const double eps = (double)a.eps;
       const double r1 = 1.0 / sqrt(s2 / (double)a.H + eps);
       const double r1_3 = r1 * r1 * r1;
@@ -251,19 +260,18 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
       tok_f[m] = (float)(r1_3 * r2);
     }
   }
-  consumer_sync();
   // pass 2: quantise into the permuted layout, one group of 16 per step
-  int rs[kMaxTok];
+  int rs[MM];
 #pragma unroll
-  for (int m = 0; m < kMaxTok; ++m) rs[m] = 0;
+  for (int m = 0; m < MM; ++m) rs[m] = 0;
 #pragma unroll 2
   for (int g = tid; g < Kw; g += NT) {
     float gn[16];
     if (a.gain) load_gain16(a.gain, (int64_t)g * 16, gn);
 #pragma unroll
-    for (int m = 0; m < kMaxTok; ++m) {
+    for (int m = 0; m < MM; ++m) {
       if (m < M) {
-        const float s = tok_s[m];
+        const float s = sc[m];
         float v[16];
         load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, v);
         int q[16];
@@ -288,19 +296,19 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
     }
   }
 #pragma unroll
-  for (int m = 0; m < kMaxTok; ++m) {
+  for (int m = 0; m < MM; ++m) {
     if (m < M) {
       const int t = warp_sum_i(rs[m]);
       if (lane == 0) red_i[warp * kMaxTok + m] = t;
     }
   }
   consumer_sync();
+  // the epilogue reads the row sums straight from the per-warp partials
   if (tid < M) {
     int t = 0;
     for (int w = 0; w < kConsumerWarps; ++w) t += red_i[w * kMaxTok + tid];
     tok_rs[tid] = t;
   }
-  consumer_sync();
 
   // ------------------------------------------------------------- main loop
   // A stage holds RS whole rows (of each matrix).  Work items are (block of
@@ -447,13 +455,13 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
   }
 }
 
-template <int MODE, int MT>
+template <int MODE, int MT, int MM>
 static cudaError_t launch_one(const GemvArgs& a, int grid, size_t smem, cudaStream_t stream) {
   static unsigned long long configured = 0;   // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(configured & (1ull << (dev & 63)))) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MODE, MT>,
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MODE, MT, MM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e != cudaSuccess) return e;
     configured |= 1ull << (dev & 63);
@@ -468,7 +476,7 @@ static cudaError_t launch_one(const GemvArgs& a, int grid, size_t smem, cudaStre
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<MODE, MT>, a);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<MODE, MT, MM>, a);
 }
 
 // Host-side planning: stage rows and ring depth under a shared-memory budget
@@ -541,9 +549,10 @@ bitnet_status bitnet_gemv_launch(int mode, GemvArgs a, int num_sms, cudaStream_t
   cudaError_t e = cudaErrorInvalidValue;
 #define BITNET_GEMV_CASE(MODE_)                                                       \
   if (mode == MODE_) {                                                                \
-    if (MT == 1) e = launch_one<MODE_, 1>(a, p.grid, p.smem, stream);                 \
-    else if (MT == 2) e = launch_one<MODE_, 2>(a, p.grid, p.smem, stream);            \
-    else e = launch_one<MODE_, 4>(a, p.grid, p.smem, stream);                         \
+    if (a.M == 1) e = launch_one<MODE_, 1, 1>(a, p.grid, p.smem, stream);             \
+    else if (a.M == 2) e = launch_one<MODE_, 2, 2>(a, p.grid, p.smem, stream);        \
+    else if (a.M <= 4) e = launch_one<MODE_, 4, 4>(a, p.grid, p.smem, stream);        \
+    else e = launch_one<MODE_, 4, 8>(a, p.grid, p.smem, stream);                      \
   }
   BITNET_GEMV_CASE(kLinear)
   BITNET_GEMV_CASE(kGlu)
