@@ -48,6 +48,7 @@ struct GemmArgs {
   float* h;                 // Glu [M,N]
   int32_t* acc_ws0;         // split-K accumulators [M,N]
   int32_t* acc_ws1;
+  int tma_store;            // 1: bf16 y written through the staged TMA store
 };
 
 constexpr int kBM = 128;                 // features per tile (MMA M)
@@ -60,7 +61,7 @@ struct GemmCfg {
   static constexpr int kA = kBM * kBK;                // one unpacked weight tile
   static constexpr int kP = kBM * (kBK / 4);          // one packed weight tile
   static constexpr int kStage = kB + NMAT * (kA + kP);
-  static constexpr int kStages0 = (218 * 1024) / kStage;
+  static constexpr int kStages0 = (218 * 1024 - ((NMAT == 1) ? 32 * 128 * 2 : 0)) / kStage;
   static constexpr int kStages = kStages0 > 6 ? 6 : (kStages0 < 2 ? 2 : kStages0);
   // accumulator sets in TMEM (512 columns): two when they fit
   static constexpr int kAcc = (2 * NMAT * BN <= 512) ? 2 : 1;
@@ -69,7 +70,10 @@ struct GemmCfg {
                                  : kCols0 <= 256 ? 256 : 512;
   static constexpr int kAux = 1024;                   // barriers + tmem slot
   static constexpr int kTok = BN * 16;                // per-token scalars
-  static constexpr size_t kSmem = 1024 /*align slack*/ + (size_t)kStages * kStage + kAux + kTok;
+  // bf16 output staging for the TMA store: 32 tokens x 128 features
+  static constexpr int kStaging = (NMAT == 1) ? 32 * kBM * 2 : 0;
+  static constexpr size_t kSmem =
+      1024 /*align slack*/ + (size_t)kStages * kStage + kAux + kTok + kStaging;
   // instruction descriptor: D s32, A s8, B s8, both K-major, N = BN, M = 128
   static constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) |
                                      ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
@@ -133,7 +137,8 @@ __device__ __forceinline__ void epi_sync() {
 template <int MODE, int BN, int NMAT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw0,
-                const __grid_constant__ CUtensorMap tw1, const GemmArgs a) {
+                const __grid_constant__ CUtensorMap tw1, const __grid_constant__ CUtensorMap ty,
+                const GemmArgs a) {
   using C = GemmCfg<BN, NMAT>;
   constexpr int S = C::kStages;
   constexpr int NACC = C::kAcc;
@@ -152,6 +157,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   float* tok_d1 = tok_d0 + BN;
   float* tok_f = tok_d1 + BN;
   int* tok_rs = reinterpret_cast<int*>(tok_f + BN);
+  uint8_t* staging = aux + C::kAux + C::kTok;     // [32 tokens][128 features] bf16
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_tiles = (a.N + kBM - 1) / kBM;
@@ -333,10 +339,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const int n = nt * kBM + lb + lane;
       const uint32_t tbase = tmem + ((uint32_t)lb << 16) + (uint32_t)(ab * NMAT * BN);
+      const bool exact_small = a.K <= 33024;  // |acc| < 2^22: integer-pipe conversion
+      const bool staged = (NMAT == 1) && a.ksplit == 1 && a.tma_store;
       for (int c0 = 0; c0 < BN && ok; c0 += 32) {
         uint32_t v0[32], v1[32];
         tmem_ld32(tbase + c0, v0);
         if (NMAT == 2) tmem_ld32(tbase + BN + c0, v1);
+        if (staged) {
+          // previous chunk's TMA store has finished reading the staging buffer
+          if (et == 0) bulk_wait_read0();
+          epi_sync();
+          const uint32_t sbase = smem_u32(staging) + 2u * (uint32_t)(lb + lane);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const int c = c0 + q;
+            const int ac = (int)v0[q] - tok_rs[c];
+            const float af = exact_small ? small_int_to_float(ac) : __int2float_rn(ac);
+            float y32 = __fmul_rn(af, tok_d0[c]);
+            if (MODE == gDown) y32 = __fmul_rn(y32, tok_f[c]);
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(sbase + (uint32_t)(q * kBM * 2)),
+                         "h"((unsigned short)f32_to_bf16_rne_bits(y32))
+                         : "memory");
+            if (a.y_f32 || a.acc0) {
+              const int tok = mt * BN + c;
+              if (tok < a.M && n < a.N) {
+                const int64_t o = (int64_t)tok * a.N + n;
+                if (a.y_f32) a.y_f32[o] = y32;
+                if (a.acc0) a.acc0[o] = ac;
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          epi_sync();
+          if (et == 0) {
+            tma_store_2d(&ty, staging, nt * kBM, mt * BN + c0);
+            bulk_commit();
+          }
+          continue;
+        }
         if (n < a.N) {
 #pragma unroll
           for (int q = 0; q < 32; ++q) {
@@ -350,18 +390,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               continue;
             }
             const int ac = (int)v0[q] - tok_rs[c];
+            const float af = exact_small ? small_int_to_float(ac) : __int2float_rn(ac);
             if (MODE == gGlu) {
               const int au = (int)v1[q] - tok_rs[c];
-              const float g = __fmul_rn(__int2float_rn(ac), tok_d0[c]);
-              const float uu = __fmul_rn(__int2float_rn(au), tok_d1[c]);
+              const float auf = exact_small ? small_int_to_float(au) : __int2float_rn(au);
+              const float g = __fmul_rn(af, tok_d0[c]);
+              const float uu = __fmul_rn(auf, tok_d1[c]);
               const float rg = fmaxf(g, 0.0f);
               a.h[o] = __fmul_rn(__fmul_rn(rg, rg), uu);
               if (a.acc0) a.acc0[o] = ac;
               if (a.acc1) a.acc1[o] = au;
             } else {
-              float y32 = __fmul_rn(__int2float_rn(ac), tok_d0[c]);
+              float y32 = __fmul_rn(af, tok_d0[c]);
               if (MODE == gDown) y32 = __fmul_rn(y32, tok_f[c]);
-              a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+              a.y[o] = (uint16_t)f32_to_bf16_rne_bits(y32);
               if (a.y_f32) a.y_f32[o] = y32;
               if (a.acc0) a.acc0[o] = ac;
             }
@@ -373,6 +415,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
     }
   }
+  if (tid == 192) bulk_wait0();              // outstanding TMA stores have landed
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -447,17 +490,19 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 2D uint8 tensor map: inner extent `inner` bytes, `rows` rows, row stride
-// `stride` bytes, box `box_inner` x `box_rows`.
-static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
-                        uint64_t stride, uint32_t box_inner, uint32_t box_rows, bool sw128) {
+// 2D tensor map: inner extent `inner` elements, `rows` rows, row stride
+// `stride` bytes, box `box_inner` x `box_rows` elements.
+static bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize,
+                        uint64_t inner, uint64_t rows, uint64_t stride, uint32_t box_inner,
+                        uint32_t box_rows, bool sw128) {
+  (void)esize;
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {stride};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t es[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides,
                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -466,8 +511,8 @@ static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64
 
 template <int MODE, int BN, int NMAT>
 static cudaError_t launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw0,
-                                 const CUtensorMap& tw1, const GemmArgs& a, dim3 grid,
-                                 cudaStream_t stream) {
+                                 const CUtensorMap& tw1, const CUtensorMap& ty, const GemmArgs& a,
+                                 dim3 grid, cudaStream_t stream) {
   using C = GemmCfg<BN, NMAT>;
   static int configured_dev_mask = 0;
   int dev = 0;
@@ -489,7 +534,7 @@ static cudaError_t launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw0,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_kernel<MODE, BN, NMAT>, tx, tw0, tw1, a);
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<MODE, BN, NMAT>, tx, tw0, tw1, ty, a);
 }
 
 int bitnet_gemm_pick_bn(int M) {
@@ -506,27 +551,37 @@ bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
                                  cudaStream_t stream) {
   CUtensorMap tx, tw0, tw1;
   const int nmat = mode == gGlu ? 2 : 1;
-  if (!make_map_u8(&tx, xq, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, kBK, (uint32_t)bn, true))
+  if (!make_map_2d(&tx, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.K, (uint64_t)a.M,
+                   (uint64_t)a.K, kBK, (uint32_t)bn, true))
     return BITNET_ERR_CUDA;
-  if (!make_map_u8(&tw0, w0, (uint64_t)a.K / 4, (uint64_t)a.N, (uint64_t)a.K / 4, kBK / 4, kBM,
-                   false))
+  if (!make_map_2d(&tw0, w0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.K / 4, (uint64_t)a.N,
+                   (uint64_t)a.K / 4, kBK / 4, kBM, false))
     return BITNET_ERR_CUDA;
   if (nmat == 2) {
-    if (!make_map_u8(&tw1, w1, (uint64_t)a.K / 4, (uint64_t)a.N, (uint64_t)a.K / 4, kBK / 4, kBM,
-                     false))
+    if (!make_map_2d(&tw1, w1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.K / 4, (uint64_t)a.N,
+                     (uint64_t)a.K / 4, kBK / 4, kBM, false))
       return BITNET_ERR_CUDA;
   } else {
     tw1 = tw0;
+  }
+  // bf16 output through TMA stores when the row pitch allows (N*2 % 16 == 0)
+  CUtensorMap ty = tw0;
+  a.tma_store = 0;
+  if (nmat == 1 && a.ksplit == 1 && a.N % 8 == 0 &&
+      (reinterpret_cast<uintptr_t>(a.y) & 15u) == 0) {
+    if (make_map_2d(&ty, a.y, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N, (uint64_t)a.M,
+                    (uint64_t)a.N * 2, kBM, 32, false))
+      a.tma_store = 1;
   }
   const int64_t units = (int64_t)((a.N + kBM - 1) / kBM) * ((a.M + bn - 1) / bn) * a.ksplit;
   dim3 grid((unsigned)(units < num_sms ? units : num_sms));
   cudaError_t e = cudaErrorInvalidValue;
 #define BITNET_GEMM_BN(MODE_, NMAT_)                                              \
   switch (bn) {                                                                   \
-    case 32: e = launch_gemm_t<MODE_, 32, NMAT_>(tx, tw0, tw1, a, grid, stream); break;   \
-    case 64: e = launch_gemm_t<MODE_, 64, NMAT_>(tx, tw0, tw1, a, grid, stream); break;   \
-    case 128: e = launch_gemm_t<MODE_, 128, NMAT_>(tx, tw0, tw1, a, grid, stream); break; \
-    default: e = launch_gemm_t<MODE_, 256, NMAT_>(tx, tw0, tw1, a, grid, stream); break;  \
+    case 32: e = launch_gemm_t<MODE_, 32, NMAT_>(tx, tw0, tw1, ty, a, grid, stream); break;   \
+    case 64: e = launch_gemm_t<MODE_, 64, NMAT_>(tx, tw0, tw1, ty, a, grid, stream); break;   \
+    case 128: e = launch_gemm_t<MODE_, 128, NMAT_>(tx, tw0, tw1, ty, a, grid, stream); break; \
+    default: e = launch_gemm_t<MODE_, 256, NMAT_>(tx, tw0, tw1, ty, a, grid, stream); break;  \
   }
   if (mode == gLinear) { BITNET_GEMM_BN(gLinear, 1) }
   else if (mode == gGlu) { BITNET_GEMM_BN(gGlu, 2) }

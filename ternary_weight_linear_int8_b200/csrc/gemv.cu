@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
   // robin; each item's per-row totals are added into shared-memory integer
   // accumulators (exact, order-free), and after a barrier the stage's
   // outputs are finished from them.
-  const uint4* x4 = reinterpret_cast<const uint4*>(xperm);
+  const uint32_t x_addr = smem_u32(xperm);
   bool ok = true;
   for (int c = 0; c < nchunks; ++c) {
     const int s = c % S;
@@ -325,17 +325,17 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
     const int nr = min(RS, n1 - r0);
     int* acc = acc_s + (c & 1) * acc_words;
     if (ok) {
-      const uint32_t* st = reinterpret_cast<const uint32_t*>(ring + (size_t)s * stage_bytes);
+      const uint32_t st_addr = smem_u32(ring + (size_t)s * stage_bytes);
       const int nitems = ((nr + 3) >> 2) * WK;
       for (int it = warp; it < nitems; it += kConsumerWarps) {
         const int b = it / WK, q = it - b * WK;
         const int j0 = (q * Kw) / WK, j1 = ((q + 1) * Kw) / WK;
-        const uint32_t* rowp[NR];
+        uint32_t rowa[NR];             // shared-window byte address of each row
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
           const int row = (NMAT == 2) ? (r >> 1) : r;
           const int mat = (NMAT == 2) ? (r & 1) : 0;
-          rowp[r] = st + (mat * RS + 4 * b + row) * Kw;
+          rowa[r] = st_addr + (uint32_t)((mat * RS + 4 * b + row) * Kb);
         }
         for (int tg = 0; tg < M; tg += MT) {
           int acc_r[NR][MT];
@@ -347,15 +347,15 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
 #pragma unroll
             for (int p = 0; p < 4; ++p) acc4[r][p] = 0;
           }
-          const uint4* xt = x4 + tg * Kw;
+          const uint32_t xt_addr = x_addr + (uint32_t)(tg * K);
 #pragma unroll 2
           for (int j = j0 + lane; j < j1; j += 32) {
             uint32_t w[NR];
 #pragma unroll
-            for (int r = 0; r < NR; ++r) w[r] = rowp[r][j];
+            for (int r = 0; r < NR; ++r) w[r] = lds_u32(rowa[r] + 4u * j);
             uint4 xv[MT];
 #pragma unroll
-            for (int t = 0; t < MT; ++t) xv[t] = xt[t * Kw + j];
+            for (int t = 0; t < MT; ++t) xv[t] = lds_v4(xt_addr + (uint32_t)(t * K) + 16u * j);
 #pragma unroll
             for (int r = 0; r < NR; ++r) {
               if constexpr (MT == 1) {
