@@ -70,7 +70,7 @@ struct GemmCfg {
                                  : kCols0 <= 256 ? 256 : 512;
   static constexpr int kAux = 1024;                   // barriers + tmem slot
   static constexpr int kTok = BN * 16;                // per-token scalars
-  // bf16 output staging for the TMA store: 32 tokens x 128 features
+  // bf16 output staging for the TMA stores: 4 warps x 2 buffers x (16 tokens x 32 features)
   static constexpr int kStaging = (NMAT == 1) ? 32 * kBM * 2 : 0;
   static constexpr size_t kSmem =
       1024 /*align slack*/ + (size_t)kStages * kStage + kAux + kTok + kStaging;
@@ -346,34 +346,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld32(tbase + c0, v0);
         if (NMAT == 2) tmem_ld32(tbase + BN + c0, v1);
         if (staged) {
-          // previous chunk's TMA store has finished reading the staging buffer
-          if (et == 0) bulk_wait_read0();
-          epi_sync();
-          const uint32_t sbase = smem_u32(staging) + 2u * (uint32_t)(lb + lane);
+          // Each warp stages its 32 features x 16 tokens (1 KB) and stores it
+          // with one TMA store; two buffers per warp, so a buffer is reused
+          // only after the store issued two half-chunks earlier has read it.
+          const uint32_t wbuf = smem_u32(staging) + (uint32_t)((warp & 3) * 2048);
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int c = c0 + q;
-            const int ac = (int)v0[q] - tok_rs[c];
-            const float af = exact_small ? small_int_to_float(ac) : __int2float_rn(ac);
-            float y32 = __fmul_rn(af, tok_d0[c]);
-            if (MODE == gDown) y32 = __fmul_rn(y32, tok_f[c]);
-            asm volatile("st.shared.u16 [%0], %1;" ::"r"(sbase + (uint32_t)(q * kBM * 2)),
-                         "h"((unsigned short)f32_to_bf16_rne_bits(y32))
-                         : "memory");
-            if (a.y_f32 || a.acc0) {
-              const int tok = mt * BN + c;
-              if (tok < a.M && n < a.N) {
-                const int64_t o = (int64_t)tok * a.N + n;
-                if (a.y_f32) a.y_f32[o] = y32;
-                if (a.acc0) a.acc0[o] = ac;
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t buf = wbuf + (uint32_t)(((c0 >> 4) + hh) & 1) * 1024u;
+            if (lane == 0) bulk_wait_read1();
+            __syncwarp();
+#pragma unroll
+            for (int qq = 0; qq < 16; ++qq) {
+              const int q = hh * 16 + qq;
+              const int c = c0 + q;
+              const int ac = (int)v0[q] - tok_rs[c];
+              const float af = exact_small ? small_int_to_float(ac) : __int2float_rn(ac);
+              float y32 = __fmul_rn(af, tok_d0[c]);
+              if (MODE == gDown) y32 = __fmul_rn(y32, tok_f[c]);
+              asm volatile("st.shared.u16 [%0], %1;" ::"r"(buf + (uint32_t)(qq * 64 + lane * 2)),
+                           "h"((unsigned short)f32_to_bf16_rne_bits(y32))
+                           : "memory");
+              if (a.y_f32 || a.acc0) {
+                const int tok = mt * BN + c;
+                if (tok < a.M && n < a.N) {
+                  const int64_t o = (int64_t)tok * a.N + n;
+                  if (a.y_f32) a.y_f32[o] = y32;
+                  if (a.acc0) a.acc0[o] = ac;
+                }
               }
             }
-          }
-          fence_proxy_async_smem();
-          epi_sync();
-          if (et == 0) {
-            tma_store_2d(&ty, staging, nt * kBM, mt * BN + c0);
-            bulk_commit();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&ty, staging + (buf - smem_u32(staging)), nt * kBM + lb,
+                           mt * BN + c0 + 16 * hh);
+              bulk_commit();
+            }
           }
           continue;
         }
@@ -415,7 +423,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
     }
   }
-  if (tid == 192) bulk_wait0();              // outstanding TMA stores have landed
+  if (warp >= 6 && lane == 0) bulk_wait0();  // this warp's TMA stores have landed
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -570,7 +578,7 @@ bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
   if (nmat == 1 && a.ksplit == 1 && a.N % 8 == 0 &&
       (reinterpret_cast<uintptr_t>(a.y) & 15u) == 0) {
     if (make_map_2d(&ty, a.y, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N, (uint64_t)a.M,
-                    (uint64_t)a.N * 2, kBM, 32, false))
+                    (uint64_t)a.N * 2, 32, 16, false))
       a.tma_store = 1;
   }
   const int64_t units = (int64_t)((a.N + kBM - 1) / kBM) * ((a.M + bn - 1) / bn) * a.ksplit;

@@ -1,4 +1,4 @@
-// Per-token absmax int8 activation quantisation (one CTA per token).
+// Per-token absmax int8 activation quantisation (one warp per token).
 //
 // youngju.dev "BitNet論文分析：1-Bit LLMの時代", section "Absmean量子化関数",
 // BitLinear_b158.activation_quant: per-token absmax scale, round, clamp.
@@ -24,112 +24,144 @@ struct QuantArgs {
   int8_t* xq_natural;     // optional extra natural-layout copy (debug), [M,K]
 };
 
+// 8 consecutive source values as floats (one 16-byte load of bf16, two of fp32).
+template <bool kF32>
+__device__ __forceinline__ void load8(const void* src, int64_t idx, float (&v)[8]) {
+  if (kF32) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(src) + idx);
+    const float4 a = p[0], b = p[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 t = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(src) + idx);
+    const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+  }
+}
+template <bool kF32>
+__device__ __forceinline__ void load4(const void* src, int64_t idx, float (&v)[4]) {
+  if (kF32) {
+    const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + idx);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  } else {
+    const uint2 t = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(src) + idx);
+    v[0] = __uint_as_float(t.x << 16);
+    v[1] = __uint_as_float(t.x & 0xffff0000u);
+    v[2] = __uint_as_float(t.y << 16);
+    v[3] = __uint_as_float(t.y & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
+         ((uint32_t)(d & 0xff) << 24);
+}
+
+// One warp per token: two passes over the row (the second mostly from L1),
+// reductions by shuffles only.  kPerm needs K % 16 == 0.
 template <bool kF32, bool kPerm>
 __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
-  __shared__ float red_f[8];
-  __shared__ int red_i[8];
-  __shared__ double red_d[8];
-  const int64_t m = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t K = a.K;
+  const int lane = threadIdx.x & 31;
+  const int64_t m = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   pdl_wait();
-  // pass 1: absmax of src*gain (and the sum of squares of src)
-  float amax = 0.f;
-  double ss = 0.0;
-  for (int64_t k = (int64_t)tid * 4; k < K; k += 256 * 4) {
-    float v[4];
-    if (kF32) {
-      const float4 t = *reinterpret_cast<const float4*>(
-          static_cast<const float*>(a.src) + m * K + k);
-      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-    } else {
-      const uint2 t = *reinterpret_cast<const uint2*>(
-          static_cast<const uint16_t*>(a.src) + m * K + k);
-      v[0] = __uint_as_float(t.x << 16);
-      v[1] = __uint_as_float(t.x & 0xffff0000u);
-      v[2] = __uint_as_float(t.y << 16);
-      v[3] = __uint_as_float(t.y & 0xffff0000u);
-    }
+  if (m < a.M) {
+    const int64_t K = a.K;
+    const int64_t base = m * K;
+    // rows start 16-byte aligned only when K % 8 == 0 (bf16) ; otherwise use
+    // 4-element chunks (8-byte bf16 loads, 4-byte code stores) throughout
+    const bool v8 = (K & 7) == 0;
+    const int64_t K8 = v8 ? K : 0;
+    // pass 1: absmax of src * gain, sum of squares of src
+    float amax = 0.f;
+    double ss = 0.0;
+#pragma unroll 4
+    for (int64_t k = (int64_t)lane * 8; k < K8; k += 256) {
+      float v[8];
+      load8<kF32>(a.src, base + k, v);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (a.sumsq) ss += (double)v[c] * (double)v[c];
-      const float g = a.gain ? __fmul_rn(v[c], a.gain[k + c]) : v[c];
-      amax = fmaxf(amax, fabsf(g));
-    }
-  }
-  amax = warp_max(amax);
-  if (a.sumsq) ss = warp_sum_d(ss);
-  if (lane == 0) { red_f[warp] = amax; red_d[warp] = ss; }
-  __syncthreads();
-  if (tid < 32) {
-    float v = lane < 8 ? red_f[lane] : 0.f;
-    v = warp_max(v);
-    double d = lane < 8 ? red_d[lane] : 0.0;
-    if (a.sumsq) d = warp_sum_d(d);
-    if (lane == 0) { red_f[0] = v; red_d[0] = d; }
-  }
-  __syncthreads();
-  const float s = qscale(red_f[0]);
-  // pass 2: quantise (re-reading the row, now in L1/L2)
-  int rs = 0;
-  const int64_t step = kPerm ? 16 : 4;
-  for (int64_t k = (int64_t)tid * step; k < K; k += 256 * step) {
-    int q[16];
-#pragma unroll
-    for (int c4 = 0; c4 < (kPerm ? 4 : 1); ++c4) {
-      const int64_t kk = k + 4 * c4;
-      float v[4];
-      if (kF32) {
-        const float4 t = *reinterpret_cast<const float4*>(
-            static_cast<const float*>(a.src) + m * K + kk);
-        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-      } else {
-        const uint2 t = *reinterpret_cast<const uint2*>(
-            static_cast<const uint16_t*>(a.src) + m * K + kk);
-        v[0] = __uint_as_float(t.x << 16);
-        v[1] = __uint_as_float(t.x & 0xffff0000u);
-        v[2] = __uint_as_float(t.y << 16);
-        v[3] = __uint_as_float(t.y & 0xffff0000u);
+      for (int c = 0; c < 8; ++c) {
+        if (a.sumsq) ss += (double)v[c] * (double)v[c];
+        const float g = a.gain ? __fmul_rn(v[c], a.gain[k + c]) : v[c];
+        amax = fmaxf(amax, fabsf(g));
       }
+    }
+    for (int64_t k = K8 + (int64_t)lane * 4; k < K; k += 128) {
+      float v[4];
+      load4<kF32>(a.src, base + k, v);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const float g = a.gain ? __fmul_rn(v[c], a.gain[kk + c]) : v[c];
-        q[4 * c4 + c] = quant_code(g, s);
-        rs += q[4 * c4 + c];
+        if (a.sumsq) ss += (double)v[c] * (double)v[c];
+        const float g = a.gain ? __fmul_rn(v[c], a.gain[k + c]) : v[c];
+        amax = fmaxf(amax, fabsf(g));
       }
     }
+    amax = warp_max(amax);
+    if (a.sumsq) ss = warp_sum_d(ss);
+    const float s = qscale(amax);
+    // pass 2: quantise
+    int rs = 0;
     if (kPerm) {
-      // slot 4*t + b holds natural index 4*b + t
-      uint32_t w[4];
+      for (int64_t k = (int64_t)lane * 16; k < K; k += 512) {
+        float v0[8], v1[8];
+        load8<kF32>(a.src, base + k, v0);
+        load8<kF32>(a.src, base + k + 8, v1);
+        int q[16];
 #pragma unroll
-      for (int t = 0; t < 4; ++t)
-        w[t] = (uint32_t)(q[t] & 0xff) | ((uint32_t)(q[4 + t] & 0xff) << 8) |
-               ((uint32_t)(q[8 + t] & 0xff) << 16) | ((uint32_t)(q[12 + t] & 0xff) << 24);
-      *reinterpret_cast<uint4*>(a.xq + m * a.ld_q + k) = make_uint4(w[0], w[1], w[2], w[3]);
-      if (a.xq_natural) {
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const uint32_t n = (uint32_t)(q[4 * c4] & 0xff) | ((uint32_t)(q[4 * c4 + 1] & 0xff) << 8) |
-                             ((uint32_t)(q[4 * c4 + 2] & 0xff) << 16) |
-                             ((uint32_t)(q[4 * c4 + 3] & 0xff) << 24);
-          *reinterpret_cast<uint32_t*>(a.xq_natural + m * K + k + 4 * c4) = n;
+        for (int c = 0; c < 8; ++c) {
+          const float g0 = a.gain ? __fmul_rn(v0[c], a.gain[k + c]) : v0[c];
+          const float g1 = a.gain ? __fmul_rn(v1[c], a.gain[k + 8 + c]) : v1[c];
+          q[c] = quant_code(g0, s);
+          q[8 + c] = quant_code(g1, s);
         }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) rs += q[c];
+        // slot 4*t + b holds natural index 4*b + t
+        *reinterpret_cast<uint4*>(a.xq + m * a.ld_q + k) =
+            make_uint4(pack4(q[0], q[4], q[8], q[12]), pack4(q[1], q[5], q[9], q[13]),
+                       pack4(q[2], q[6], q[10], q[14]), pack4(q[3], q[7], q[11], q[15]));
+        if (a.xq_natural)
+          *reinterpret_cast<uint4*>(a.xq_natural + m * K + k) =
+              make_uint4(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]),
+                         pack4(q[8], q[9], q[10], q[11]), pack4(q[12], q[13], q[14], q[15]));
       }
     } else {
-      const uint32_t n = (uint32_t)(q[0] & 0xff) | ((uint32_t)(q[1] & 0xff) << 8) |
-                         ((uint32_t)(q[2] & 0xff) << 16) | ((uint32_t)(q[3] & 0xff) << 24);
-      *reinterpret_cast<uint32_t*>(a.xq + m * a.ld_q + k) = n;
+#pragma unroll 4
+      for (int64_t k = (int64_t)lane * 8; k < K8; k += 256) {
+        float v[8];
+        load8<kF32>(a.src, base + k, v);
+        int q[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float g = a.gain ? __fmul_rn(v[c], a.gain[k + c]) : v[c];
+          q[c] = quant_code(g, s);
+          rs += q[c];
+        }
+        *reinterpret_cast<uint2*>(a.xq + m * a.ld_q + k) =
+            make_uint2(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]));
+      }
+      for (int64_t k = K8 + (int64_t)lane * 4; k < K; k += 128) {
+        float v[4];
+        load4<kF32>(a.src, base + k, v);
+        int q[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float g = a.gain ? __fmul_rn(v[c], a.gain[k + c]) : v[c];
+          q[c] = quant_code(g, s);
+          rs += q[c];
+        }
+        *reinterpret_cast<uint32_t*>(a.xq + m * a.ld_q + k) = pack4(q[0], q[1], q[2], q[3]);
+      }
     }
-  }
-  rs = warp_sum_i(rs);
-  if (lane == 0) red_i[warp] = rs;
-  __syncthreads();
-  if (tid == 0) {
-    int t = 0;
-    for (int w = 0; w < 8; ++w) t += red_i[w];
-    a.scale[m] = s;
-    if (a.rowsum) a.rowsum[m] = t;
-    if (a.sumsq) a.sumsq[m] = red_d[0];
+    rs = warp_sum_i(rs);
+    if (lane == 0) {
+      a.scale[m] = s;
+      if (a.rowsum) a.rowsum[m] = rs;
+      if (a.sumsq) a.sumsq[m] = ss;
+    }
   }
   pdl_launch_dependents();
 }
@@ -145,7 +177,7 @@ bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* ga
                                   cudaStream_t stream) {
   QuantArgs a{src, gain, M, K, xq, ld_q, scale, rowsum, sumsq, xq_natural};
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)M);
+  cfg.gridDim = dim3((unsigned)((M + 7) / 8));
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
