@@ -186,6 +186,38 @@ BITNET_API bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int
                          size_t workspace_bytes, void* stream);
 
 /*
+ * BitLinear without a caller workspace, for callers that cannot allocate
+ * device memory: code that issues work while a CUDA stream is being
+ * captured into a graph (a cudaMalloc there is not part of the capture),
+ * services that reserve a fixed memory budget at start-up and allocate
+ * nothing afterwards, and plug-ins running inside another framework whose
+ * allocator they cannot reach.  The pages describe no such variant; it has no
+ * counterpart there.
+ *
+ * Computes exactly what bitnet_linear computes (same kernels, same results,
+ * no y_f32 / acc outputs).  The scratch that bitnet_linear takes from the
+ * workspace argument comes instead from one fixed array of
+ * BITNET_NOALLOC_SCRATCH_BYTES in device memory that the library defines;
+ * every GPU that loads the library holds that array until the process exits.
+ * The function itself calls no allocator (no cudaMalloc, cudaFree or
+ * allocating library routine).
+ *   - Shapes whose scratch would exceed the array (see
+ *     bitnet_linear_workspace_size) return BITNET_ERR_WORKSPACE and enqueue
+ *     nothing.
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (once per device, with that device current); make
+ *     that first call before capturing any stream.
+ *   - All calls share the one array, which keeps the last call's contents;
+ *     whatever must start at zero is cleared by the call itself.  Calls that
+ *     may overlap on the GPU (other streams, other host threads) race on the
+ *     array: the caller must order them, e.g. on one stream.
+ */
+#define BITNET_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+BITNET_API bitnet_status bitnet_linear_noalloc(const uint8_t* packed, const float* gamma, int64_t N,
+                                               int64_t K, const uint16_t* x, int64_t M,
+                                               uint16_t* y, void* stream);
+
+/*
  * Synchronise `stream`, then return and clear the device status word of the
  * current device: BITNET_OK, BITNET_ERR_TIMEOUT (a bounded wait expired; the
  * affected outputs are unspecified) or BITNET_ERR_NONFINITE.  A failing

@@ -40,6 +40,7 @@ SIGNATURES = {
     "bitnet_ffn": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _F,
                                   _P, _P, _P, _SZ, _P]),
     "bitnet_last_device_status": (ctypes.c_int, [_P]),
+    "bitnet_linear_noalloc": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I64, _P, _P]),
 }
 
 
@@ -216,6 +217,23 @@ def bitnet_ffn(x: torch.Tensor, w: FfnWeights, eps: float = 1e-5, y=None, debug:
                           _ptr(ws), nb, _stream())
     _check("bitnet_ffn", st)
     return y, dbg
+
+
+def bitnet_linear_noalloc(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, y=None):
+    """BitLinear using the library's fixed device scratch array instead of a
+    workspace (for callers that cannot allocate).  Returns y bf16 [M,N]."""
+    _dev(packed, "packed")
+    _dev(gamma, "gamma")
+    _bits16(x, "x")
+    N, Kb = packed.shape
+    M, K = x.shape
+    if K != 4 * Kb:
+        raise ValueError("x and packed disagree on K")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    st = lib().bitnet_linear_noalloc(_ptr(packed), _ptr(gamma), N, K, _ptr(x), M, _ptr(y),
+                                     _stream())
+    _check("bitnet_linear_noalloc", st)
+    return y
 
 
 def bitnet_last_device_status() -> int:

@@ -6,3 +6,4 @@
 #include "gemv.cu"
 #include "gemm.cu"
 #include "api.cu"
+#include "noalloc.cu"
