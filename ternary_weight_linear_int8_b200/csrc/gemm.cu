@@ -350,6 +350,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // with one TMA store; two buffers per warp, so a buffer is reused
           // only after the store issued two half-chunks earlier has read it.
           const uint32_t wbuf = smem_u32(staging) + (uint32_t)((warp & 3) * 2048);
+          // per-token scalars of this chunk, into registers (broadcast loads)
+          float d0r[32], fr[32];
+          int rsr[32];
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const uint4 dv = lds_v4(smem_u32(tok_d0 + c0 + 4 * q4));
+            const uint4 rv = lds_v4(smem_u32(tok_rs + c0 + 4 * q4));
+            d0r[4 * q4] = __uint_as_float(dv.x); d0r[4 * q4 + 1] = __uint_as_float(dv.y);
+            d0r[4 * q4 + 2] = __uint_as_float(dv.z); d0r[4 * q4 + 3] = __uint_as_float(dv.w);
+            rsr[4 * q4] = (int)rv.x; rsr[4 * q4 + 1] = (int)rv.y;
+            rsr[4 * q4 + 2] = (int)rv.z; rsr[4 * q4 + 3] = (int)rv.w;
+            if (MODE == gDown) {
+              const uint4 fv = lds_v4(smem_u32(tok_f + c0 + 4 * q4));
+              fr[4 * q4] = __uint_as_float(fv.x); fr[4 * q4 + 1] = __uint_as_float(fv.y);
+              fr[4 * q4 + 2] = __uint_as_float(fv.z); fr[4 * q4 + 3] = __uint_as_float(fv.w);
+            }
+          }
+          const bool dbg = (a.y_f32 != nullptr) || (a.acc0 != nullptr);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const uint32_t buf = wbuf + (uint32_t)(((c0 >> 4) + hh) & 1) * 1024u;
@@ -358,16 +376,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int qq = 0; qq < 16; ++qq) {
               const int q = hh * 16 + qq;
-              const int c = c0 + q;
-              const int ac = (int)v0[q] - tok_rs[c];
+              const int ac = (int)v0[q] - rsr[q];
               const float af = exact_small ? small_int_to_float(ac) : __int2float_rn(ac);
-              float y32 = __fmul_rn(af, tok_d0[c]);
-              if (MODE == gDown) y32 = __fmul_rn(y32, tok_f[c]);
+              float y32 = __fmul_rn(af, d0r[q]);
+              if (MODE == gDown) y32 = __fmul_rn(y32, fr[q]);
               asm volatile("st.shared.u16 [%0], %1;" ::"r"(buf + (uint32_t)(qq * 64 + lane * 2)),
-                           "h"((unsigned short)f32_to_bf16_rne_bits(y32))
-                           : "memory");
-              if (a.y_f32 || a.acc0) {
-                const int tok = mt * BN + c;
+                           "h"((unsigned short)f32_to_bf16_rne_bits(y32)));
+              if (dbg) {
+                const int tok = mt * BN + c0 + q;
                 if (tok < a.M && n < a.N) {
                   const int64_t o = (int64_t)tok * a.N + n;
                   if (a.y_f32) a.y_f32[o] = y32;

@@ -45,7 +45,7 @@ struct GemvArgs {
   int wk;                 // K-slices per 4-row block
 };
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 16;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxTok = 8;
 
@@ -106,7 +106,7 @@ __device__ __forceinline__ void load_gain16(const float* g, int64_t idx, float (
 }
 
 template <int MODE, int MT, int MM>
-__global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
   // MM: token count rounded up to 1, 2, 4 or 8 (loops over tokens unroll to
   // MM, keeping the code small for single-token decode)
   constexpr int NMAT = (MODE == kGlu) ? 2 : 1;
@@ -121,13 +121,13 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
   float* tok_d1 = tok_d0 + kMaxTok;
   float* tok_f = tok_d1 + kMaxTok;
   int* tok_rs = reinterpret_cast<int*>(tok_f + kMaxTok);
-  float* red_f = reinterpret_cast<float*>(smem + 384);          // [8 warps][8 tok]
-  int* red_i = reinterpret_cast<int*>(smem + 640);              // [8][8]
-  double* red_d = reinterpret_cast<double*>(smem + 1024);       // [8][8][2]
+  float* red_f = reinterpret_cast<float*>(smem + 512);          // [16 warps][8 tok]
+  int* red_i = reinterpret_cast<int*>(smem + 1024);             // [16][8]
+  double* red_d = reinterpret_cast<double*>(smem + 2048);       // [16][8][2]
   const int M = a.M, K = a.K, N = a.N;
   const int Mpad = ((M + MT - 1) / MT) * MT;
   const int RS = a.rows_per_stage, S = a.stages, WK = a.wk;
-  uint8_t* xperm = smem + 2048;
+  uint8_t* xperm = smem + 4096;
   const int xbytes = ((Mpad * K + 127) / 128) * 128;
   // per-stage integer accumulators [2 parity][NMAT][RS][kMaxTok]
   int* acc_s = reinterpret_cast<int*>(xperm + xbytes);
@@ -178,25 +178,54 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
   for (int i = M * K + tid * 16; i < Mpad * K; i += NT * 16)
     *reinterpret_cast<uint4*>(xperm + i) = make_uint4(0, 0, 0, 0);
 
-  // pass 1: per-token absmax of src*gain (and, for Down, sums of squares)
+  // pass 1: per-token absmax of src*gain (and, for Down, sums of squares).
+  // With one or two tokens and at most KEEPG groups of 16 per thread the
+  // values stay in registers for pass 2 instead of being loaded again.
+  constexpr int KEEPG = (MM == 1) ? 2 : 1;
+  const bool keep = (MM <= 2) && Kw <= KEEPG * NT;
+  float vk[KEEPG][MM][16];
   float am[MM];
   double ss[MM], sx[MM];
 #pragma unroll
   for (int m = 0; m < MM; ++m) { am[m] = 0.f; ss[m] = 0.0; sx[m] = 0.0; }
+  if (keep) {
+#pragma unroll
+    for (int gi = 0; gi < KEEPG; ++gi) {
+      const int g = tid + gi * NT;
+      if (g < Kw) {
+        float gn[16];
+        if (a.gain) load_gain16(a.gain, (int64_t)g * 16, gn);
+#pragma unroll
+        for (int m = 0; m < MM; ++m) {
+          if (m < M) {
+            load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, vk[gi][m]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float v = vk[gi][m][i];
+              const float vg = a.gain ? __fmul_rn(v, gn[i]) : v;
+              am[m] = fmaxf(am[m], fabsf(vg));
+              if (MODE == kDown) ss[m] += (double)v * (double)v;
+            }
+          }
+        }
+      }
+    }
+  } else {
 #pragma unroll 2
-  for (int g = tid; g < Kw; g += NT) {
-    float gn[16];
-    if (a.gain) load_gain16(a.gain, (int64_t)g * 16, gn);
+    for (int g = tid; g < Kw; g += NT) {
+      float gn[16];
+      if (a.gain) load_gain16(a.gain, (int64_t)g * 16, gn);
 #pragma unroll
-    for (int m = 0; m < MM; ++m) {
-      if (m < M) {
-        float v[16];
-        load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, v);
+      for (int m = 0; m < MM; ++m) {
+        if (m < M) {
+          float v[16];
+          load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, v);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float vg = a.gain ? __fmul_rn(v[i], gn[i]) : v[i];
-          am[m] = fmaxf(am[m], fabsf(vg));
-          if (MODE == kDown) ss[m] += (double)v[i] * (double)v[i];
+          for (int i = 0; i < 16; ++i) {
+            const float vg = a.gain ? __fmul_rn(v[i], gn[i]) : v[i];
+            am[m] = fmaxf(am[m], fabsf(vg));
+            if (MODE == kDown) ss[m] += (double)v[i] * (double)v[i];
+          }
         }
       }
     }
@@ -264,33 +293,49 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvArgs a) {
   int rs[MM];
 #pragma unroll
   for (int m = 0; m < MM; ++m) rs[m] = 0;
+  auto quant_group = [&](int g, int m, const float (&v)[16], const float (&gn)[16]) {
+    const float s = sc[m];
+    int q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float vg = a.gain ? __fmul_rn(v[i], gn[i]) : v[i];
+      q[i] = quant_code(vg, s);
+      rs[m] += q[i];
+    }
+    uint32_t w[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      w[t] = (uint32_t)(q[t] & 0xff) | ((uint32_t)(q[4 + t] & 0xff) << 8) |
+             ((uint32_t)(q[8 + t] & 0xff) << 16) | ((uint32_t)(q[12 + t] & 0xff) << 24);
+    *reinterpret_cast<uint4*>(xperm + (int64_t)m * K + g * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (a.xq_dbg && blockIdx.x == 0) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) a.xq_dbg[(int64_t)m * K + g * 16 + i] = (int8_t)q[i];
+    }
+  };
+  if (keep) {
+#pragma unroll
+    for (int gi = 0; gi < KEEPG; ++gi) {
+      const int g = tid + gi * NT;
+      if (g < Kw) {
+        float gn[16];
+        if (a.gain) load_gain16(a.gain, (int64_t)g * 16, gn);
+#pragma unroll
+        for (int m = 0; m < MM; ++m)
+          if (m < M) quant_group(g, m, vk[gi][m], gn);
+      }
+    }
+  } else {
 #pragma unroll 2
-  for (int g = tid; g < Kw; g += NT) {
-    float gn[16];
-    if (a.gain) load_gain16(a.gain, (int64_t)g * 16, gn);
+    for (int g = tid; g < Kw; g += NT) {
+      float gn[16];
+      if (a.gain) load_gain16(a.gain, (int64_t)g * 16, gn);
 #pragma unroll
-    for (int m = 0; m < MM; ++m) {
-      if (m < M) {
-        const float s = sc[m];
-        float v[16];
-        load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, v);
-        int q[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float vg = a.gain ? __fmul_rn(v[i], gn[i]) : v[i];
-          q[i] = quant_code(vg, s);
-          rs[m] += q[i];
-        }
-        uint32_t w[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          w[t] = (uint32_t)(q[t] & 0xff) | ((uint32_t)(q[4 + t] & 0xff) << 8) |
-                 ((uint32_t)(q[8 + t] & 0xff) << 16) | ((uint32_t)(q[12 + t] & 0xff) << 24);
-        *reinterpret_cast<uint4*>(xperm + (int64_t)m * K + g * 16) =
-            make_uint4(w[0], w[1], w[2], w[3]);
-        if (a.xq_dbg && blockIdx.x == 0) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) a.xq_dbg[(int64_t)m * K + g * 16 + i] = (int8_t)q[i];
+      for (int m = 0; m < MM; ++m) {
+        if (m < M) {
+          float v[16];
+          load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, v);
+          quant_group(g, m, v, gn);
         }
       }
     }
@@ -505,23 +550,25 @@ static GemvPlan plan_gemv(int M, int N, int K, int nmat, int num_sms, int MT) {
   GemvPlan p{};
   const int Mpad = ((M + MT - 1) / MT) * MT;
   const size_t xbytes = (((size_t)Mpad * K + 127) / 128) * 128;
-  const size_t budget = 112 * 1024;
+  const size_t budget = 200 * 1024;
   const size_t row_bytes = (size_t)(K / 4) * nmat;
   int blocks = (N + 3) / 4;
   p.grid = blocks < num_sms ? blocks : num_sms;
   const int rows_per_cta = (N + p.grid - 1) / p.grid;
-  int rs = (int)((32 * 1024) / row_bytes);
-  rs = rs / 4 * 4;
-  if (rs < 4) rs = 4;
-  const int rows_cap = (rows_per_cta + 3) / 4 * 4;
-  if (rs > rows_cap) rs = rows_cap;
+  // stages of at most 48 KB, as few as cover the CTA's rows, equally sized
+  int rs_max = (int)((48 * 1024) / row_bytes) / 4 * 4;
+  if (rs_max < 4) rs_max = 4;
+  const int nch = (rows_per_cta + rs_max - 1) / rs_max;
+  int rs = (rows_per_cta + nch - 1) / nch;
+  rs = (rs + 3) / 4 * 4;
   const size_t acc_bytes = ((2 * (size_t)nmat * rs * kMaxTok * 4 + 127) / 128) * 128;
-  const size_t head = 2048 + xbytes + acc_bytes;
+  const size_t head = 4096 + xbytes + acc_bytes;
   const size_t ring = budget > head + 2 * (size_t)rs * row_bytes ? budget - head
                                                                   : 2 * (size_t)rs * row_bytes;
   int st = (int)(ring / ((size_t)rs * row_bytes));
   if (st > 8) st = 8;
   if (st < 2) st = 2;
+  if (st > nch) st = nch < 2 ? 2 : nch;
   p.rows_per_stage = rs;
   p.stages = st;
   p.wk = pick_wk(rs / 4, K / 16);
