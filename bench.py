@@ -148,6 +148,25 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(value, device=None):
+    """Max of a per-rank float over all ranks (identity without a process
+    group).  Every rank must call it at the same point."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world, units_per_rank, seconds_max):
+    """Whole-job throughput: every rank processed units_per_rank in at most
+    seconds_max (the slowest rank's time)."""
+    return world * units_per_rank / seconds_max
+
+
 # -------------------------------------------------------- CPU reference arm
 def oracle_decode_sample(n_layers, seed_base=0):
     """Pack a few decode layers with the oracle (untimed) and return them."""
@@ -407,7 +426,7 @@ def run_ours(args, world, rank, local):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=dev)
         barrier = dist.barrier
     B.lib()
@@ -427,11 +446,7 @@ def run_ours(args, world, rank, local):
     sampler.start()
     ms, t0, t1 = time_graph(torch, graph, stream, args.steps, args.warmup, barrier)
     clocks = sampler.stop(t0, t1)
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, dev)
     # the graph's output equals an eager chain, bit for bit
     y_graph = bufs[1].clone()
     chain_calls(B, packs, x, bufs)
@@ -442,7 +457,7 @@ def run_ours(args, world, rank, local):
     n_launch = len(packs)
     step_s = ms / args.steps * 1e-3
     packed_bytes = sum(p.numel() for p, _ in packs)
-    value = world * packed_bytes / step_s / 1e9
+    value = weak_scaling_value(world, packed_bytes, step_s) / 1e9
     # roofline for the decode kernel: algorithmic bytes per launch / avg launch time
     alg_bytes = packed_bytes / n_launch + 2 * HIDDEN + 2 * INTER + 4
     launch_s = step_s / n_launch
@@ -473,13 +488,8 @@ def run_ours(args, world, rank, local):
             yh.copy_(out.view(torch.int16), non_blocking=True)
         e1.record(stream)
         e1.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e = {"value": world * packed_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+    e2e = {"value": weak_scaling_value(world, packed_bytes, e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
            "ms_per_step": e2e_ms,
            "how": "pinned host x -> device, 60 eager bitnet_linear calls through the Python "
