@@ -53,7 +53,7 @@ struct GemmArgs {
 
 constexpr int kBM = 128;                 // features per tile (MMA M)
 constexpr int kBK = 128;                 // K elements (bytes) per stage
-constexpr int kGemmThreads = 320;        // 10 warps: TMA, MMA, 4 unpack, 4 epilogue
+constexpr int kGemmThreads = 448;        // 14 warps: TMA, MMA, 4 unpack, 8 epilogue
 
 template <int BN, int NMAT>
 struct GemmCfg {
@@ -68,9 +68,9 @@ struct GemmCfg {
   static constexpr int kCols0 = kAcc * NMAT * BN;
   static constexpr int kTmemCols = kCols0 <= 32 ? 32 : kCols0 <= 64 ? 64 : kCols0 <= 128 ? 128
                                  : kCols0 <= 256 ? 256 : 512;
-  static constexpr int kAux = 1024;                   // barriers + tmem slot
-  static constexpr int kTok = BN * 16;                // per-token scalars
-  // bf16 output staging for the TMA stores: 4 warps x 2 buffers x (16 tokens x 32 features)
+  static constexpr int kAux = 512;                    // barriers + tmem slot
+  static constexpr int kTok = BN * 12;                // per-token scalars: d0, rowsum, d1-or-f
+  // bf16 output staging for the TMA stores: 8 warps x 2 buffers x (8 tokens x 32 features)
   static constexpr int kStaging = (NMAT == 1) ? 32 * kBM * 2 : 0;
   static constexpr size_t kSmem =
       1024 /*align slack*/ + (size_t)kStages * kStage + kAux + kTok + kStaging;
@@ -127,7 +127,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void epi_sync() {
-  asm volatile("bar.sync 2, 128;" ::: "memory");
+  asm volatile("bar.sync 2, 256;" ::: "memory");
 }
 
 // Persistent: each CTA walks work units (feature tile, token tile, K split)
@@ -154,10 +154,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_empty = acc_full + NACC;     // [NACC]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + NACC);
   float* tok_d0 = reinterpret_cast<float*>(aux + C::kAux);
-  float* tok_d1 = tok_d0 + BN;
-  float* tok_f = tok_d1 + BN;
-  int* tok_rs = reinterpret_cast<int*>(tok_f + BN);
-  uint8_t* staging = aux + C::kAux + C::kTok;     // [32 tokens][128 features] bf16
+  int* tok_rs = reinterpret_cast<int*>(tok_d0 + BN);
+  float* tok_x1 = reinterpret_cast<float*>(tok_rs + BN);   // Glu: gamma_up / s; Down: r1^3 r2
+  float* tok_d1 = tok_x1;
+  float* tok_f = tok_x1;
+  uint8_t* staging = aux + C::kAux + C::kTok;     // 8 warps x 2 x [8 tokens][32 features] bf16
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_tiles = (a.N + kBM - 1) / kBM;
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < NACC; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], 8);
     }
     fence_mbar_init();
     prefetch_tmap(&tx);
@@ -301,9 +302,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // --------------------------------------------------------- epilogue
+    // 8 warps: warp w reads TMEM lanes 32*(w%4).. (its quadrant of features)
+    // and one half of the token columns.
     pdl_wait();
-    const int et = tid - 192;                // 0..127
-    const int lb = 32 * (warp & 3);          // TMEM lanes this warp may access
+    const int ew = warp - 6;                 // 0..7
+    const int et = tid - 192;                // 0..255
+    const int lb = 32 * (warp & 3);
+    const int half = ew >> 2;
+    const int cbeg = (BN >= 64) ? half * (BN / 2) : 0;
+    const int cend = (BN >= 64) ? cbeg + BN / 2 : (half == 0 ? BN : 0);
     int i = 0;
     for (int unit = blockIdx.x; unit < units; unit += gridDim.x, ++i) {
       int nt, mt, k0, nk;
@@ -311,27 +318,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int ab = i % NACC;
       if (a.ksplit == 1) {
         epi_sync();                          // previous unit's scalars are consumed
-        for (int c = et; c < BN; c += 128) {
+        for (int c = et; c < BN; c += 256) {
           const int tok = mt * BN + c;
-          float d0 = 0.f, d1 = 0.f, f = 0.f;
+          float d0 = 0.f, x1 = 0.f;
           int rs = 0;
           if (tok < a.M) {
             const float s = a.scale[tok];
             d0 = __fdiv_rn(*a.gamma0, s);
-            if (MODE == gGlu) d1 = __fdiv_rn(*a.gamma1, s);
+            if (MODE == gGlu) x1 = __fdiv_rn(*a.gamma1, s);
             rs = a.rowsum[tok];
             if (MODE == gDown) {
               const double eps = (double)a.eps;
               const double r1 = 1.0 / sqrt(a.sumsq_x[tok] / (double)a.H + eps);
               const double r1_3 = r1 * r1 * r1;
               const double r2 = 1.0 / sqrt(r1_3 * r1_3 * (a.sumsq_h[tok] / (double)a.K) + eps);
-              f = (float)(r1_3 * r2);
+              x1 = (float)(r1_3 * r2);
             }
           }
           tok_d0[c] = d0;
-          tok_d1[c] = d1;
-          tok_f[c] = f;
           tok_rs[c] = rs;
+          tok_x1[c] = x1;
         }
         epi_sync();
       }
@@ -341,49 +347,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t tbase = tmem + ((uint32_t)lb << 16) + (uint32_t)(ab * NMAT * BN);
       const bool exact_small = a.K <= 33024;  // |acc| < 2^22: integer-pipe conversion
       const bool staged = (NMAT == 1) && a.ksplit == 1 && a.tma_store;
-      for (int c0 = 0; c0 < BN && ok; c0 += 32) {
+      const bool dbg = (a.y_f32 != nullptr) || (a.acc0 != nullptr);
+      for (int c0 = cbeg; c0 < cend && ok; c0 += 32) {
         uint32_t v0[32], v1[32];
         tmem_ld32(tbase + c0, v0);
         if (NMAT == 2) tmem_ld32(tbase + BN + c0, v1);
         if (staged) {
-          // Each warp stages its 32 features x 16 tokens (1 KB) and stores it
-          // with one TMA store; two buffers per warp, so a buffer is reused
-          // only after the store issued two half-chunks earlier has read it.
-          const uint32_t wbuf = smem_u32(staging) + (uint32_t)((warp & 3) * 2048);
-          // per-token scalars of this chunk, into registers (broadcast loads)
-          float d0r[32], fr[32];
-          int rsr[32];
+          // each warp stages 8 tokens x its 32 features (512 B) per TMA store;
+          // two buffers per warp, reused once the store two steps back has
+          // finished reading
+          const uint32_t wbuf = smem_u32(staging) + (uint32_t)(ew * 1024);
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const uint4 dv = lds_v4(smem_u32(tok_d0 + c0 + 4 * q4));
-            const uint4 rv = lds_v4(smem_u32(tok_rs + c0 + 4 * q4));
-            d0r[4 * q4] = __uint_as_float(dv.x); d0r[4 * q4 + 1] = __uint_as_float(dv.y);
-            d0r[4 * q4 + 2] = __uint_as_float(dv.z); d0r[4 * q4 + 3] = __uint_as_float(dv.w);
-            rsr[4 * q4] = (int)rv.x; rsr[4 * q4 + 1] = (int)rv.y;
-            rsr[4 * q4 + 2] = (int)rv.z; rsr[4 * q4 + 3] = (int)rv.w;
+          for (int sub = 0; sub < 4; ++sub) {
+            const uint32_t buf = wbuf + (uint32_t)(sub & 1) * 512u;
+            const int cs = c0 + 8 * sub;
+            const uint4 dA = lds_v4(smem_u32(tok_d0 + cs)), dB = lds_v4(smem_u32(tok_d0 + cs + 4));
+            const uint4 rA = lds_v4(smem_u32(tok_rs + cs)), rB = lds_v4(smem_u32(tok_rs + cs + 4));
+            const float d8[8] = {__uint_as_float(dA.x), __uint_as_float(dA.y), __uint_as_float(dA.z),
+                                 __uint_as_float(dA.w), __uint_as_float(dB.x), __uint_as_float(dB.y),
+                                 __uint_as_float(dB.z), __uint_as_float(dB.w)};
+            const int r8[8] = {(int)rA.x, (int)rA.y, (int)rA.z, (int)rA.w,
+                               (int)rB.x, (int)rB.y, (int)rB.z, (int)rB.w};
+            float f8[8];
             if (MODE == gDown) {
-              const uint4 fv = lds_v4(smem_u32(tok_f + c0 + 4 * q4));
-              fr[4 * q4] = __uint_as_float(fv.x); fr[4 * q4 + 1] = __uint_as_float(fv.y);
-              fr[4 * q4 + 2] = __uint_as_float(fv.z); fr[4 * q4 + 3] = __uint_as_float(fv.w);
+              const uint4 fA = lds_v4(smem_u32(tok_f + cs)), fB = lds_v4(smem_u32(tok_f + cs + 4));
+              f8[0] = __uint_as_float(fA.x); f8[1] = __uint_as_float(fA.y);
+              f8[2] = __uint_as_float(fA.z); f8[3] = __uint_as_float(fA.w);
+              f8[4] = __uint_as_float(fB.x); f8[5] = __uint_as_float(fB.y);
+              f8[6] = __uint_as_float(fB.z); f8[7] = __uint_as_float(fB.w);
             }
-          }
-          const bool dbg = (a.y_f32 != nullptr) || (a.acc0 != nullptr);
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const uint32_t buf = wbuf + (uint32_t)(((c0 >> 4) + hh) & 1) * 1024u;
             if (lane == 0) bulk_wait_read1();
             __syncwarp();
 #pragma unroll
-            for (int qq = 0; qq < 16; ++qq) {
-              const int q = hh * 16 + qq;
-              const int ac = (int)v0[q] - rsr[q];
+            for (int qq = 0; qq < 8; ++qq) {
+              const int q = 8 * sub + qq;
+              const int ac = (int)v0[q] - r8[qq];
               const float af = exact_small ? small_int_to_float(ac) : __int2float_rn(ac);
-              float y32 = __fmul_rn(af, d0r[q]);
-              if (MODE == gDown) y32 = __fmul_rn(y32, fr[q]);
+              float y32 = __fmul_rn(af, d8[qq]);
+              if (MODE == gDown) y32 = __fmul_rn(y32, f8[qq]);
               asm volatile("st.shared.u16 [%0], %1;" ::"r"(buf + (uint32_t)(qq * 64 + lane * 2)),
                            "h"((unsigned short)f32_to_bf16_rne_bits(y32)));
               if (dbg) {
-                const int tok = mt * BN + c0 + q;
+                const int tok = mt * BN + cs + qq;
                 if (tok < a.M && n < a.N) {
                   const int64_t o = (int64_t)tok * a.N + n;
                   if (a.y_f32) a.y_f32[o] = y32;
@@ -394,8 +399,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&ty, staging + (buf - smem_u32(staging)), nt * kBM + lb,
-                           mt * BN + c0 + 16 * hh);
+              tma_store_2d(&ty, staging + (buf - smem_u32(staging)), nt * kBM + lb, mt * BN + cs);
               bulk_commit();
             }
           }
@@ -594,7 +598,7 @@ bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
   if (nmat == 1 && a.ksplit == 1 && a.N % 8 == 0 &&
       (reinterpret_cast<uintptr_t>(a.y) & 15u) == 0) {
     if (make_map_2d(&ty, a.y, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N, (uint64_t)a.M,
-                    (uint64_t)a.N * 2, 32, 16, false))
+                    (uint64_t)a.N * 2, 32, 8, false))
       a.tma_store = 1;
   }
   const int64_t units = (int64_t)((a.N + kBM - 1) / kBM) * ((a.M + bn - 1) / bn) * a.ksplit;
