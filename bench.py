@@ -393,7 +393,13 @@ def profile_case(case):
     from ternary_weight_linear_int8_b200 import bitnet as B
     from ternary_weight_linear_int8_b200 import inputs
     dev = torch.device("cuda", 0)
-    if case == "prefill":
+    if case == "gemv_big":
+        N, K = 28672, 8192
+        x = torch.from_numpy(inputs.activations((1, K), seed=0).view(np.int16)).to(dev)
+        p, g = B.bitnet_pack_weights(torch.from_numpy(inputs.weights(N, K, seed=2000)).to(dev))
+        for _ in range(4):
+            B.bitnet_linear(p, g, x)
+    elif case == "prefill":
         M, N, K = 4096, INTER, HIDDEN
         x = torch.from_numpy(inputs.activations((M, K), seed=0).view(np.int16)).to(dev)
         W = torch.from_numpy(inputs.weights(N, K, seed=1000)).to(dev)
@@ -547,7 +553,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--profile-case", choices=["prefill", "ffn2048"], default=None,
+    ap.add_argument("--profile-case", choices=["prefill", "ffn2048", "gemv_big"], default=None,
                     help="run a few calls of one workload for an ncu capture, print nothing")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -48,6 +48,7 @@ struct GemvArgs {
 constexpr int kConsumerWarps = 16;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxTok = 8;
+constexpr uint32_t kCopyChunk = 4096;   // bytes per bulk copy (a multiple of 16)
 
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
@@ -165,8 +166,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
         const uint32_t bytes = (uint32_t)nr * Kb;
         mbar_arrive_expect_tx(&full[s], bytes * NMAT);
         uint8_t* dst = ring + (size_t)s * stage_bytes;
-        bulk_g2s(dst, a.w0 + (int64_t)r0 * Kb, bytes, &full[s], pol);
-        if (NMAT == 2) bulk_g2s(dst + (size_t)RS * Kb, a.w1 + (int64_t)r0 * Kb, bytes, &full[s], pol);
+        // several 4 KB copies per stage keep more requests in flight than
+        // one large copy
+        for (uint32_t off = 0; off < bytes; off += kCopyChunk) {
+          const uint32_t nb = bytes - off < kCopyChunk ? bytes - off : kCopyChunk;
+          bulk_g2s(dst + off, a.w0 + (int64_t)r0 * Kb + off, nb, &full[s], pol);
+          if (NMAT == 2)
+            bulk_g2s(dst + (size_t)RS * Kb + off, a.w1 + (int64_t)r0 * Kb + off, nb, &full[s], pol);
+        }
       }
     }
     return;
