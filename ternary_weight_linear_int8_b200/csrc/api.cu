@@ -19,7 +19,7 @@ bitnet_status bitnet_gemv_launch(int mode, GemvArgs a, int num_sms, cudaStream_t
 bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
                                  const uint8_t* w1, GemmArgs a, int bn, int num_sms,
                                  cudaStream_t stream);
-int bitnet_gemm_pick_bn(int M);
+int bitnet_gemm_pick_bn(int M, int N, int num_sms);
 
 namespace {
 
@@ -258,7 +258,7 @@ bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N
   }
   st = bitnet_quant_launch(x, false, nullptr, M, K, xq, K, true, sc, rs, nullptr, nullptr, s);
   if (st != BITNET_OK) return st;
-  const int bn = bitnet_gemm_pick_bn((int)M);
+  const int bn = bitnet_gemm_pick_bn((int)M, (int)N, d.num_sms);
   GemmArgs a{};
   a.M = (int)M; a.N = (int)N; a.K = (int)K;
   a.ksplit = plan_ksplit(M, N, K, bn, d.num_sms);
@@ -328,7 +328,7 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
   float* hbuf = dbg.h ? dbg.h : h;
   st = bitnet_quant_launch(x, false, norm1_w, M, H, xq1, H, true, s1, rs1, ss1, dbg.xq1, s);
   if (st != BITNET_OK) return st;
-  const int bn = bitnet_gemm_pick_bn((int)M);
+  const int bn = bitnet_gemm_pick_bn((int)M, (int)I, d.num_sms);
   GemmArgs g{};
   g.M = (int)M; g.N = (int)I; g.K = (int)H;
   g.ksplit = plan_ksplit(M, I, H, bn, d.num_sms);
@@ -346,8 +346,9 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
   st = bitnet_quant_launch(hbuf, true, norm2_w, M, I, xq2, I, true, s2, rs2, ss2, dbg.xq2, s);
   if (st != BITNET_OK) return st;
   GemmArgs dn{};
+  const int bn_d = bitnet_gemm_pick_bn((int)M, (int)H, d.num_sms);
   dn.M = (int)M; dn.N = (int)H; dn.K = (int)I;
-  dn.ksplit = plan_ksplit(M, H, I, bn, d.num_sms);
+  dn.ksplit = plan_ksplit(M, H, I, bn_d, d.num_sms);
   dn.scale = s2; dn.rowsum = rs2; dn.gamma0 = gamma_down;
   dn.sumsq_h = ss2; dn.sumsq_x = ss1; dn.H = (int)H; dn.eps = eps;
   dn.y = y; dn.y_f32 = dbg.y_f32; dn.acc0 = dbg.acc_down;
@@ -355,7 +356,7 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
     dn.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
     if (cudaMemsetAsync(dn.acc_ws0, 0, (size_t)M * H * 4, s) != cudaSuccess) return BITNET_ERR_CUDA;
   }
-  return bitnet_gemm_launch(2 /*down*/, xq2, down, nullptr, dn, bn, d.num_sms, s);
+  return bitnet_gemm_launch(2 /*down*/, xq2, down, nullptr, dn, bn_d, d.num_sms, s);
 }
 
 bitnet_status bitnet_last_device_status(void* stream) {

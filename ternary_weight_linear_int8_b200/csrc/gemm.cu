@@ -565,11 +565,27 @@ static cudaError_t launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw0,
   return cudaLaunchKernelEx(&cfg, gemm_kernel<MODE, BN, NMAT>, tx, tw0, tw1, ty, a);
 }
 
-int bitnet_gemm_pick_bn(int M) {
+// Token-tile width: small M takes the smallest tile that covers it; large M
+// picks among 256, 192 and 128 the width whose tile count fills the last
+// wave of the persistent grid best (ties to the wider tile).
+int bitnet_gemm_pick_bn(int M, int N, int num_sms) {
   if (M <= 32) return 32;
   if (M <= 64) return 64;
   if (M <= 128) return 128;
-  return 256;
+  const int cand[3] = {256, 192, 128};
+  int best = 256;
+  double best_score = -1.0;
+  for (int i = 0; i < 3; ++i) {
+    const int bn = cand[i];
+    const long long mt = (M + bn - 1) / bn;
+    const long long units = (long long)((N + kBM - 1) / kBM) * mt;
+    const double waves = (double)units / num_sms;
+    const double fill = waves / (double)((units + num_sms - 1) / num_sms);
+    const double pad = (double)M / (double)(mt * bn);
+    const double score = fill * pad * (bn == 256 ? 1.0 : (bn == 192 ? 0.985 : 0.96));
+    if (score > best_score + 1e-9) { best_score = score; best = bn; }
+  }
+  return best;
 }
 
 // Launch the tensor-core kernel (and, with ksplit > 1, its finaliser).
@@ -609,6 +625,7 @@ bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
     case 32: e = launch_gemm_t<MODE_, 32, NMAT_>(tx, tw0, tw1, ty, a, grid, stream); break;   \
     case 64: e = launch_gemm_t<MODE_, 64, NMAT_>(tx, tw0, tw1, ty, a, grid, stream); break;   \
     case 128: e = launch_gemm_t<MODE_, 128, NMAT_>(tx, tw0, tw1, ty, a, grid, stream); break; \
+    case 192: e = launch_gemm_t<MODE_, 192, NMAT_>(tx, tw0, tw1, ty, a, grid, stream); break; \
     default: e = launch_gemm_t<MODE_, 256, NMAT_>(tx, tw0, tw1, ty, a, grid, stream); break;  \
   }
   if (mode == gLinear) { BITNET_GEMM_BN(gLinear, 1) }

@@ -127,7 +127,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
   double* red_d = reinterpret_cast<double*>(smem + 2048);       // [16][8][2]
   const int M = a.M, K = a.K, N = a.N;
   const int Mpad = ((M + MT - 1) / MT) * MT;
-  const int RS = a.rows_per_stage, S = a.stages, WK = a.wk;
+  const int RS = a.rows_per_stage, S = a.stages, WK = a.wk;   // WK is a power of two
+  const int wk_log2 = __ffs(WK) - 1;
   uint8_t* xperm = smem + 4096;
   const int xbytes = ((Mpad * K + 127) / 128) * 128;
   // per-stage integer accumulators [2 parity][NMAT][RS][kMaxTok]
@@ -380,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
       const uint32_t st_addr = smem_u32(ring + (size_t)s * stage_bytes);
       const int nitems = ((nr + 3) >> 2) * WK;
       for (int it = warp; it < nitems; it += kConsumerWarps) {
-        const int b = it / WK, q = it - b * WK;
+        const int b = it >> wk_log2, q = it & (WK - 1);
         const int j0 = (q * Kw) / WK, j1 = ((q + 1) * Kw) / WK;
         uint32_t rowa[NR];             // shared-window byte address of each row
 #pragma unroll
@@ -538,8 +539,8 @@ struct GemvPlan {
   size_t smem;
 };
 
-// K-slices per row block: balance (blocks x slices) items over the 8 warps
-// against the per-item reduction cost (about half a 32-word step).
+// K-slices per row block: balance (blocks x slices) items over the warps
+// against the fixed cost of an item (reduction, shared atomics, set-up).
 static int pick_wk(int nb, int Kw) {
   int best = 1;
   double best_cost = 1e30;
@@ -547,7 +548,7 @@ static int pick_wk(int nb, int Kw) {
     if (wk > 1 && Kw / wk < 8) break;
     const double rounds = (double)((nb * wk + kConsumerWarps - 1) / kConsumerWarps);
     const double iters = (double)((Kw / wk + 31) / 32);
-    const double cost = rounds * (iters + 0.5);
+    const double cost = rounds * (iters + 2.0);   // per-item reduction ~ two 32-word steps
     if (cost < best_cost - 1e-9) { best_cost = cost; best = wk; }
   }
   return best;
