@@ -328,7 +328,8 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
   float* hbuf = dbg.h ? dbg.h : h;
   st = bitnet_quant_launch(x, false, norm1_w, M, H, xq1, H, true, s1, rs1, ss1, dbg.xq1, s);
   if (st != BITNET_OK) return st;
-  const int bn = bitnet_gemm_pick_bn((int)M, (int)I, d.num_sms);
+  // gate and up share the activation tile: keep it at the full 256 tokens
+  const int bn = M > 128 ? 256 : bitnet_gemm_pick_bn((int)M, (int)I, d.num_sms);
   GemmArgs g{};
   g.M = (int)M; g.N = (int)I; g.K = (int)H;
   g.ksplit = plan_ksplit(M, I, H, bn, d.num_sms);

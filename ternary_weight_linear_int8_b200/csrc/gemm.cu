@@ -582,7 +582,9 @@ int bitnet_gemm_pick_bn(int M, int N, int num_sms) {
     const double waves = (double)units / num_sms;
     const double fill = waves / (double)((units + num_sms - 1) / num_sms);
     const double pad = (double)M / (double)(mt * bn);
-    const double score = fill * pad * (bn == 256 ? 1.0 : (bn == 192 ? 0.985 : 0.96));
+    // narrower tiles move more shared-memory bytes per MMA: only worth it
+    // when they fill the last wave much better
+    const double score = fill * pad * (bn == 256 ? 1.0 : (bn == 192 ? 0.85 : 0.75));
     if (score > best_score + 1e-9) { best_score = score; best = bn; }
   }
   return best;

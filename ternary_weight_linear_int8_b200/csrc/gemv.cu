@@ -111,7 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
   // MM: token count rounded up to 1, 2, 4 or 8 (loops over tokens unroll to
   // MM, keeping the code small for single-token decode)
   constexpr int NMAT = (MODE == kGlu) ? 2 : 1;
-  constexpr int NR = 4 * NMAT;             // values per lane per row block
+  constexpr int RB = (NMAT == 2) ? 4 : 8;  // rows per block (per matrix)
+  constexpr int NR = 8;                    // values per lane per block: RB rows x NMAT
   constexpr bool kF32Src = (MODE == kDown);
   constexpr int NT = kConsumerWarps * 32;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -379,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
     int* acc = acc_s + (c & 1) * acc_words;
     if (ok) {
       const uint32_t st_addr = smem_u32(ring + (size_t)s * stage_bytes);
-      const int nitems = ((nr + 3) >> 2) * WK;
+      const int nitems = ((nr + RB - 1) / RB) * WK;
       for (int it = warp; it < nitems; it += kConsumerWarps) {
         const int b = it >> wk_log2, q = it & (WK - 1);
         const int j0 = (q * Kw) / WK, j1 = ((q + 1) * Kw) / WK;
@@ -388,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
         for (int r = 0; r < NR; ++r) {
           const int row = (NMAT == 2) ? (r >> 1) : r;
           const int mat = (NMAT == 2) ? (r & 1) : 0;
-          rowa[r] = st_addr + (uint32_t)((mat * RS + 4 * b + row) * Kb);
+          rowa[r] = st_addr + (uint32_t)((mat * RS + RB * b + row) * Kb);
         }
         for (int tg = 0; tg < M; tg += MT) {
           int acc_r[NR][MT];
@@ -443,31 +444,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
             int v[NR];
 #pragma unroll
             for (int r = 0; r < NR; ++r) v[r] = acc_r[r][t];
-            int tot;
-            int row, mat;
-            bool writer;
-            if constexpr (NR == 4) {
-              int h2[2], h1[1];
-              halve<4>(v, h2, 16, lane);
-              halve<2>(h2, h1, 8, lane);
-              tot = h1[0];
-              tot += __shfl_xor_sync(0xffffffffu, tot, 4);
-              tot += __shfl_xor_sync(0xffffffffu, tot, 2);
-              tot += __shfl_xor_sync(0xffffffffu, tot, 1);
-              row = lane >> 3; mat = 0; writer = (lane & 7) == 0;
-            } else {
-              int h4[4], h2[2], h1[1];
-              halve<8>(v, h4, 16, lane);
-              halve<4>(h4, h2, 8, lane);
-              halve<2>(h2, h1, 4, lane);
-              tot = h1[0];
-              tot += __shfl_xor_sync(0xffffffffu, tot, 2);
-              tot += __shfl_xor_sync(0xffffffffu, tot, 1);
-              row = lane >> 3; mat = (lane >> 2) & 1; writer = (lane & 3) == 0;
-            }
+            // butterfly over the 8 values: lane l ends with value l >> 2
+            int h4[4], h2[2], h1[1];
+            halve<8>(v, h4, 16, lane);
+            halve<4>(h4, h2, 8, lane);
+            halve<2>(h2, h1, 4, lane);
+            int tot = h1[0];
+            tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+            tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+            const int vi = lane >> 2;
+            const int row = (NMAT == 2) ? (vi >> 1) : vi;
+            const int mat = (NMAT == 2) ? (vi & 1) : 0;
+            const bool writer = (lane & 3) == 0;
             const int m = tg + t;
-            if (writer && m < M && 4 * b + row < nr)
-              atomicAdd(&acc[(mat * RS + 4 * b + row) * kMaxTok + m], tot);
+            if (writer && m < M && RB * b + row < nr)
+              atomicAdd(&acc[(mat * RS + RB * b + row) * kMaxTok + m], tot);
           }
         }
       }
@@ -563,12 +554,13 @@ static GemvPlan plan_gemv(int M, int N, int K, int nmat, int num_sms, int MT) {
   int blocks = (N + 3) / 4;
   p.grid = blocks < num_sms ? blocks : num_sms;
   const int rows_per_cta = (N + p.grid - 1) / p.grid;
-  // stages of at most 48 KB, as few as cover the CTA's rows, equally sized
-  int rs_max = (int)((48 * 1024) / row_bytes) / 4 * 4;
-  if (rs_max < 4) rs_max = 4;
+  // stages of at most 56 KB, as few as cover the CTA's rows, equally sized
+  const int rb = nmat == 2 ? 4 : 8;       // rows per work block
+  int rs_max = (int)((56 * 1024) / row_bytes) / rb * rb;
+  if (rs_max < rb) rs_max = rb;
   const int nch = (rows_per_cta + rs_max - 1) / rs_max;
   int rs = (rows_per_cta + nch - 1) / nch;
-  rs = (rs + 3) / 4 * 4;
+  rs = (rs + rb - 1) / rb * rb;
   const size_t acc_bytes = ((2 * (size_t)nmat * rs * kMaxTok * 4 + 127) / 128) * 128;
   const size_t head = 4096 + xbytes + acc_bytes;
   const size_t ring = budget > head + 2 * (size_t)rs * row_bytes ? budget - head
@@ -579,7 +571,7 @@ static GemvPlan plan_gemv(int M, int N, int K, int nmat, int num_sms, int MT) {
   if (st > nch) st = nch < 2 ? 2 : nch;
   p.rows_per_stage = rs;
   p.stages = st;
-  p.wk = pick_wk(rs / 4, K / 16);
+  p.wk = pick_wk(rs / rb, K / 16);
   p.smem = head + (size_t)st * rs * row_bytes;
   return p;
 }
