@@ -106,13 +106,14 @@ __device__ __forceinline__ void load_gain16(const float* g, int64_t idx, float (
   }
 }
 
-template <int MODE, int MT, int MM>
+template <int MODE, int MT, int MM, int RB>
 __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
   // MM: token count rounded up to 1, 2, 4 or 8 (loops over tokens unroll to
   // MM, keeping the code small for single-token decode)
   constexpr int NMAT = (MODE == kGlu) ? 2 : 1;
-  constexpr int RB = (NMAT == 2) ? 4 : 8;  // rows per block (per matrix)
-  constexpr int NR = 8;                    // values per lane per block: RB rows x NMAT
+  // RB: rows per work block (per matrix); NR values per lane per block
+  constexpr int NR = RB * NMAT;
+  static_assert(NR == 4 || NR == 8, "4 or 8 values per block");
   constexpr bool kF32Src = (MODE == kDown);
   constexpr int NT = kConsumerWarps * 32;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -444,18 +445,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
             int v[NR];
 #pragma unroll
             for (int r = 0; r < NR; ++r) v[r] = acc_r[r][t];
-            // butterfly over the 8 values: lane l ends with value l >> 2
-            int h4[4], h2[2], h1[1];
-            halve<8>(v, h4, 16, lane);
-            halve<4>(h4, h2, 8, lane);
-            halve<2>(h2, h1, 4, lane);
-            int tot = h1[0];
-            tot += __shfl_xor_sync(0xffffffffu, tot, 2);
-            tot += __shfl_xor_sync(0xffffffffu, tot, 1);
-            const int vi = lane >> 2;
-            const int row = (NMAT == 2) ? (vi >> 1) : vi;
-            const int mat = (NMAT == 2) ? (vi & 1) : 0;
-            const bool writer = (lane & 3) == 0;
+            int tot, row, mat;
+            bool writer;
+            if constexpr (NR == 4) {
+              // butterfly over 4 values: lane l ends with row l >> 3
+              int h2[2], h1[1];
+              halve<4>(v, h2, 16, lane);
+              halve<2>(h2, h1, 8, lane);
+              tot = h1[0];
+              tot += __shfl_xor_sync(0xffffffffu, tot, 4);
+              tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+              tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+              row = lane >> 3; mat = 0; writer = (lane & 7) == 0;
+            } else {
+              // butterfly over 8 values: lane l ends with value l >> 2
+              int h4[4], h2[2], h1[1];
+              halve<8>(v, h4, 16, lane);
+              halve<4>(h4, h2, 8, lane);
+              halve<2>(h2, h1, 4, lane);
+              tot = h1[0];
+              tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+              tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+              const int vi = lane >> 2;
+              row = (NMAT == 2) ? (vi >> 1) : vi;
+              mat = (NMAT == 2) ? (vi & 1) : 0;
+              writer = (lane & 3) == 0;
+            }
             const int m = tg + t;
             if (writer && m < M && RB * b + row < nr)
               atomicAdd(&acc[(mat * RS + RB * b + row) * kMaxTok + m], tot);
@@ -499,13 +514,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
   }
 }
 
-template <int MODE, int MT, int MM>
+template <int MODE, int MT, int MM, int RB>
 static cudaError_t launch_one(const GemvArgs& a, int grid, size_t smem, cudaStream_t stream) {
   static unsigned long long configured = 0;   // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(configured & (1ull << (dev & 63)))) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MODE, MT, MM>,
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MODE, MT, MM, RB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e != cudaSuccess) return e;
     configured |= 1ull << (dev & 63);
@@ -520,7 +535,7 @@ static cudaError_t launch_one(const GemvArgs& a, int grid, size_t smem, cudaStre
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<MODE, MT, MM>, a);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<MODE, MT, MM, RB>, a);
 }
 
 // Host-side planning: stage rows and ring depth under a shared-memory budget
@@ -545,6 +560,12 @@ static int pick_wk(int nb, int Kw) {
   return best;
 }
 
+// Rows per work block: 8 for a single matrix with long rows and one token
+// (the activation loads and the reduction are shared by more rows), else 4.
+static int gemv_rows_per_block(int M, int K, int nmat) {
+  return (nmat == 1 && M == 1 && K >= 8192) ? 8 : 4;
+}
+
 static GemvPlan plan_gemv(int M, int N, int K, int nmat, int num_sms, int MT) {
   GemvPlan p{};
   const int Mpad = ((M + MT - 1) / MT) * MT;
@@ -555,7 +576,7 @@ static GemvPlan plan_gemv(int M, int N, int K, int nmat, int num_sms, int MT) {
   p.grid = blocks < num_sms ? blocks : num_sms;
   const int rows_per_cta = (N + p.grid - 1) / p.grid;
   // stages of at most 56 KB, as few as cover the CTA's rows, equally sized
-  const int rb = nmat == 2 ? 4 : 8;       // rows per work block
+  const int rb = gemv_rows_per_block(M, K, nmat);
   int rs_max = (int)((56 * 1024) / row_bytes) / rb * rb;
   if (rs_max < rb) rs_max = rb;
   const int nch = (rows_per_cta + rs_max - 1) / rs_max;
@@ -593,13 +614,15 @@ bitnet_status bitnet_gemv_launch(int mode, GemvArgs a, int num_sms, cudaStream_t
   a.rows_per_stage = p.rows_per_stage;
   a.stages = p.stages;
   a.wk = p.wk;
+  const int rb = gemv_rows_per_block(a.M, a.K, nmat);
   cudaError_t e = cudaErrorInvalidValue;
 #define BITNET_GEMV_CASE(MODE_)                                                       \
   if (mode == MODE_) {                                                                \
-    if (a.M == 1) e = launch_one<MODE_, 1, 1>(a, p.grid, p.smem, stream);             \
-    else if (a.M == 2) e = launch_one<MODE_, 2, 2>(a, p.grid, p.smem, stream);        \
-    else if (a.M <= 4) e = launch_one<MODE_, 4, 4>(a, p.grid, p.smem, stream);        \
-    else e = launch_one<MODE_, 4, 8>(a, p.grid, p.smem, stream);                      \
+    if (a.M == 1 && rb == 8) e = launch_one<MODE_, 1, 1, (MODE_ == kGlu ? 4 : 8)>(a, p.grid, p.smem, stream); \
+    else if (a.M == 1) e = launch_one<MODE_, 1, 1, 4>(a, p.grid, p.smem, stream);     \
+    else if (a.M == 2) e = launch_one<MODE_, 2, 2, 4>(a, p.grid, p.smem, stream);     \
+    else if (a.M <= 4) e = launch_one<MODE_, 4, 4, 4>(a, p.grid, p.smem, stream);     \
+    else e = launch_one<MODE_, 4, 8, 4>(a, p.grid, p.smem, stream);                   \
   }
   BITNET_GEMV_CASE(kLinear)
   BITNET_GEMV_CASE(kGlu)
