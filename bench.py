@@ -4,10 +4,12 @@
 Headline workload (one "step"): 2B-class decode, M = 1 token, a chain of 30
 layers x {up [6912,2560], down [2560,6912]} = 60 distinct packed matrices
 (265 MB of packed weights, larger than the 126 MB L2), each BitLinear fed the
-previous one's bf16 output, captured in one CUDA graph (kernels use
-programmatic dependent launch).  Per step the path runs activation quant
+previous one's bf16 output: one bitnet_linear_chain call (one cooperative
+launch of the decode kernel running the 60 layers with a grid barrier between
+them), captured in a CUDA graph.  Per step the path runs activation quant
 (fused), the ternary int8 matmul and the dequant/bf16 store for all 60
-matrices.  value = packed-weight bytes streamed / device time (GB/s).
+matrices.  value = packed-weight bytes streamed / device time (GB/s).  The
+same chain as 60 separate bitnet_linear calls is reported alongside.
 
 Secondary figures (same JSON line, "secondary"): prefill GEMM TOPS at M=4096,
 batched decode M in {4,16,64}, and the 100B-class FFN block at M=1 and 2048.
@@ -263,12 +265,31 @@ def build_decode_chain(B, inputs, torch, dev, n_layers=2 * LAYERS):
 
 
 def chain_calls(B, packs, x, bufs):
+    """The chain as one bitnet_linear call per layer."""
     cur = x
     for l, (p, g) in enumerate(packs):
         out = bufs[l % 2]
         B.bitnet_linear(p, g, cur, y=out)
         cur = out
     return cur
+
+
+class ChainProgram:
+    """The chain as one bitnet_linear_chain call (outputs ping-pong in bufs)."""
+
+    def __init__(self, B, torch, packs, bufs, dev):
+        self.B = B
+        self.P = [p for p, _ in packs]
+        self.G = [g for _, g in packs]
+        self.ys = [bufs[l % 2] for l in range(len(packs))]
+        M = bufs[0].shape[0]
+        nb = B.bitnet_linear_chain_workspace_size([p.shape[0] for p in self.P],
+                                                  [p.shape[1] * 4 for p in self.P], M)
+        self.ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+
+    def __call__(self, x):
+        self.B.bitnet_linear_chain(self.P, self.G, x, ys=self.ys, workspace=self.ws)
+        return self.ys[-1]
 
 
 def capture(torch, fn, stream):
@@ -329,27 +350,28 @@ def secondary_measurements(B, inputs, torch, dev, stream, pk):
                                         "includes": "activation quant kernel + tcgen05 GEMM"}
         del g
     del xs, yu, yd, wsu, wsd
-    # batched decode: the same 60-layer chain with M tokens
+    # batched decode: the same 60-layer chain with M tokens (M = 1: as 60
+    # separate bitnet_linear calls, for comparison with the one-launch chain)
     packs = pk["_packs"]
-    for M in (4, 16, 64):
+    for M in (1, 4, 16, 64):
         x = torch.from_numpy(inputs.activations((M, HIDDEN), seed=0, outliers=True).view(np.int16)).to(dev)
         bufs = [torch.empty((M, INTER), dtype=torch.bfloat16, device=dev),
                 torch.empty((M, HIDDEN), dtype=torch.bfloat16, device=dev)]
-        wsb = torch.empty(max(B.bitnet_linear_workspace_size(M, INTER, HIDDEN),
-                              B.bitnet_linear_workspace_size(M, HIDDEN, INTER), 16),
-                          dtype=torch.uint8, device=dev)
+        if M == 1:
+            def run():
+                chain_calls(B, packs, x, bufs)
+        else:
+            prog = ChainProgram(B, torch, packs, bufs, dev)
 
-        def run():
-            cur = x
-            for l, (p, g_) in enumerate(packs):
-                B.bitnet_linear(p, g_, cur, y=bufs[l % 2], workspace=wsb)
-                cur = bufs[l % 2]
+            def run():
+                prog(x)
         g = capture(torch, run, stream)
         ms, _, _ = time_graph(torch, g, stream, 20, 3)
         t = ms / 20 * 1e-3
         nbytes = sum(p.numel() for p, _ in packs)
         ops = 2.0 * M * sum(p.numel() * 4 for p, _ in packs)
-        out[f"decode_chain_M{M}"] = {"GB/s": round(nbytes / t / 1e9, 1),
+        key = "decode_chain_M1_separate_calls" if M == 1 else f"decode_chain_M{M}"
+        out[key] = {"GB/s": round(nbytes / t / 1e9, 1),
                                      "TOPS": round(ops / t / 1e12, 2),
                                      "frac_hbm": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4),
                                      "us_per_step": round(t * 1e6, 1)}
@@ -447,32 +469,35 @@ def run_ours(args, world, rank, local):
     bufs = [torch.empty((1, INTER), dtype=torch.bfloat16, device=dev),
             torch.empty((1, HIDDEN), dtype=torch.bfloat16, device=dev)]
     torch.cuda.synchronize()
-    graph = capture(torch, lambda: chain_calls(B, packs, x, bufs), stream)
+    program = ChainProgram(B, torch, packs, bufs, dev)
+    graph = capture(torch, lambda: program(x), stream)
     sampler = ClockSampler(local)
     sampler.start()
     ms, t0, t1 = time_graph(torch, graph, stream, args.steps, args.warmup, barrier)
     clocks = sampler.stop(t0, t1)
     ms = max_over_ranks(ms, dev)
-    # the graph's output equals an eager chain, bit for bit
+    # the graph's output equals 60 eager bitnet_linear calls, bit for bit
     y_graph = bufs[1].clone()
     chain_calls(B, packs, x, bufs)
     torch.cuda.synchronize()
     check_ok = bool(torch.equal(y_graph.view(torch.int16), bufs[1].view(torch.int16)))
     status = B.bitnet_last_device_status()
 
-    n_launch = len(packs)
+    n_mat = len(packs)
     step_s = ms / args.steps * 1e-3
     packed_bytes = sum(p.numel() for p, _ in packs)
     value = weak_scaling_value(world, packed_bytes, step_s) / 1e9
-    # roofline for the decode kernel: algorithmic bytes per launch / avg launch time
-    alg_bytes = packed_bytes / n_launch + 2 * HIDDEN + 2 * INTER + 4
-    launch_s = step_s / n_launch
+    # roofline for the decode kernel: one launch per step runs all 60 layers;
+    # algorithmic bytes = packed weights + each layer's bf16 input and output
+    # + the gammas
+    alg_bytes = packed_bytes + n_mat // 2 * 2 * (2 * HIDDEN + 2 * INTER) + 4 * n_mat
+    launch_s = step_s
     achieved = alg_bytes / launch_s / 1e9
-    traffic = profile_traffic("gemv_decode_2b_m1.md")
+    traffic = profile_traffic("decode_program_2b_m1.md")
 
     # --------------------------------------------------- e2e through the API
-    # per step: pinned host x -> device, 60 bitnet_linear calls through the
-    # binding (eager, no graph), device -> pinned host y
+    # per step: pinned host x -> device, one bitnet_linear_chain call through
+    # the binding (eager, no graph), device -> pinned host y
     xh = torch.from_numpy(x_host.view(np.int16)).pin_memory()
     yh = torch.empty((1, HIDDEN), dtype=torch.int16).pin_memory()
     xd = torch.empty((1, HIDDEN), dtype=torch.int16, device=dev)
@@ -480,7 +505,7 @@ def run_ours(args, world, rank, local):
     with torch.cuda.stream(stream):
         for _ in range(3):
             xd.copy_(xh, non_blocking=True)
-            out = chain_calls(B, packs, xd, bufs)
+            out = program(xd)
             yh.copy_(out.view(torch.int16), non_blocking=True)
         torch.cuda.synchronize()
         if barrier:
@@ -490,7 +515,7 @@ def run_ours(args, world, rank, local):
         e0.record(stream)
         for _ in range(e2e_steps):
             xd.copy_(xh, non_blocking=True)
-            out = chain_calls(B, packs, xd, bufs)
+            out = program(xd)
             yh.copy_(out.view(torch.int16), non_blocking=True)
         e1.record(stream)
         e1.synchronize()
@@ -498,8 +523,8 @@ def run_ours(args, world, rank, local):
     e2e = {"value": weak_scaling_value(world, packed_bytes, e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
            "ms_per_step": e2e_ms,
-           "how": "pinned host x -> device, 60 eager bitnet_linear calls through the Python "
-                  "binding, device -> pinned host y; CUDA events"}
+           "how": "pinned host x -> device, one eager bitnet_linear_chain call (60 layers) "
+                  "through the Python binding, device -> pinned host y; CUDA events"}
 
     secondary = None
     if not args.no_secondary and rank == 0:
@@ -517,19 +542,20 @@ def run_ours(args, world, rank, local):
             "data": "synthetic",
             "config": {"workload": "2B-class decode GEMV chain, M=1: 30 layers x (up [6912,2560], "
                                    "down [2560,6912]) = 60 distinct 2-bit packed matrices, "
-                                   "each fed the previous bf16 output; one CUDA graph per step",
-                       "M": 1, "matrices": n_launch, "packed_bytes_per_step": packed_bytes,
+                                   "each fed the previous bf16 output; one bitnet_linear_chain "
+                                   "call (one cooperative launch) per step, in a CUDA graph",
+                       "M": 1, "matrices": n_mat, "packed_bytes_per_step": packed_bytes,
                        "l2": "inputs larger than L2 (265 MB packed weights > 126 MB L2), no flush",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
-                         "traffic": traffic, "kernel": "gemv_kernel<Linear,1>",
+                         "traffic": traffic, "kernel": "decode_kernel, 60-layer program",
                          "peak_source": pk["source"],
                          "algorithmic_bytes_per_launch": alg_bytes,
                          "launch_us": round(launch_s * 1e6, 3)},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": n_launch * args.steps,
+            "gpu_launches": args.steps,
             "clocks": clocks,
             "device_status": B.bitnet_status_string(status),
             "graph_equals_eager": check_ok,

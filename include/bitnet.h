@@ -175,7 +175,11 @@ typedef struct {
  * means all ones.  eps >= 0.  y [M,H] bf16 bits written.
  * workspace >= bitnet_ffn_workspace_size(M, H, I) bytes.
  * debug  NULL or a host struct of optional device outputs (see above).
- * Requires M >= 1, H % 64 == 0, I % 64 == 0, H, I >= 64.
+ * Requires M >= 1, H % 64 == 0, I % 64 == 0, H, I >= 64.  With M <= 8 and
+ * M_pad * max(H, I) <= 65536 (M_pad = M rounded up to 1, 2 or a multiple of
+ * 4) the whole block is one cooperative launch of the decode kernel (one CTA
+ * per SM, a grid barrier between gate/up and down); larger M runs the
+ * activation quantiser and the tensor-core kernel per step.
  */
 BITNET_API size_t bitnet_ffn_workspace_size(int64_t M, int64_t H, int64_t I);
 BITNET_API bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
@@ -184,6 +188,44 @@ BITNET_API bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int
                          const uint8_t* down, const float* gamma_down, float eps,
                          uint16_t* y, const bitnet_ffn_debug* debug, void* workspace,
                          size_t workspace_bytes, void* stream);
+
+/*
+ * A chain of BitLinear layers, each fed the previous one's output:
+ *   y[0] = BitLinear(packed[0], gamma[0])(x),
+ *   y[l] = BitLinear(packed[l], gamma[l])(y[l-1])   for l = 1 .. L-1,
+ * every layer computed exactly as bitnet_linear computes it (same codes,
+ * accumulators and bf16 outputs).  [A] section "モデル構造": the model is a
+ * decoder-only Transformer whose nn.Linear layers are all BitLinear, so a
+ * decode step runs them one after the other; the pages define no call that
+ * runs several layers, this one only schedules them.
+ *
+ * Runs of consecutive layers in the decode kernel's range (M <= 8,
+ * K % 64 == 0, M_pad * K <= 65536) execute as one cooperative launch of up
+ * to 64 layers: the weights of later layers stream into shared memory while
+ * earlier layers compute, and the CTAs meet at a grid barrier between
+ * layers.  Other layers run as bitnet_linear calls.
+ *
+ * L        number of layers, >= 1.
+ * packed, gamma, N, K, y   HOST arrays of L entries; packed[l], gamma[l] and
+ *          y[l] are device pointers.  Layer l maps [M, K[l]] to [M, N[l]];
+ *          K[l] == N[l-1] for l >= 1.  The arrays are read during the call
+ *          only.
+ * x        [M, K[0]] bf16 bits, device.   y[l]  [M, N[l]] bf16 bits, written.
+ * A layer's output may not overlap its input (y[l] vs y[l-1], y[0] vs x):
+ * BITNET_ERR_INVALID_ARG.  Ping-pong buffers (y[l] == y[l-2]) are fine.
+ * workspace  >= bitnet_linear_chain_workspace_size(L, N, K, M) bytes, device
+ *          (contents need not be initialised; the call uses its first 256
+ *          bytes as the grid-barrier counter).
+ * Other requirements and errors as bitnet_linear, per layer; all layers are
+ * validated before anything is enqueued.
+ */
+BITNET_API size_t bitnet_linear_chain_workspace_size(int64_t L, const int64_t* N,
+                                                     const int64_t* K, int64_t M);
+BITNET_API bitnet_status bitnet_linear_chain(int64_t L, const uint8_t* const* packed,
+                                             const float* const* gamma, const int64_t* N,
+                                             const int64_t* K, const uint16_t* x, int64_t M,
+                                             uint16_t* const* y, void* workspace,
+                                             size_t workspace_bytes, void* stream);
 
 /*
  * BitLinear without a caller workspace, for callers that cannot allocate

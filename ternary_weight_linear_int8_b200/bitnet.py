@@ -41,6 +41,8 @@ SIGNATURES = {
                                   _P, _P, _P, _SZ, _P]),
     "bitnet_last_device_status": (ctypes.c_int, [_P]),
     "bitnet_linear_noalloc": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I64, _P, _P]),
+    "bitnet_linear_chain_workspace_size": (_SZ, [_I64, _P, _P, _I64]),
+    "bitnet_linear_chain": (ctypes.c_int, [_I64, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
 }
 
 
@@ -217,6 +219,46 @@ def bitnet_ffn(x: torch.Tensor, w: FfnWeights, eps: float = 1e-5, y=None, debug:
                           _ptr(ws), nb, _stream())
     _check("bitnet_ffn", st)
     return y, dbg
+
+
+def _host_arrays(packs, gammas, ys, x):
+    L = len(packs)
+    Ns = (ctypes.c_int64 * L)(*[int(p.shape[0]) for p in packs])
+    Ks = (ctypes.c_int64 * L)(*[int(p.shape[1]) * 4 for p in packs])
+    P = (ctypes.c_void_p * L)(*[p.data_ptr() for p in packs])
+    G = (ctypes.c_void_p * L)(*[g.data_ptr() for g in gammas])
+    Y = (ctypes.c_void_p * L)(*[y.data_ptr() for y in ys])
+    return L, Ns, Ks, P, G, Y
+
+
+def bitnet_linear_chain_workspace_size(Ns, Ks, M: int) -> int:
+    L = len(Ns)
+    n = (ctypes.c_int64 * L)(*Ns)
+    k = (ctypes.c_int64 * L)(*Ks)
+    return lib().bitnet_linear_chain_workspace_size(L, n, k, M)
+
+
+def bitnet_linear_chain(packs, gammas, x: torch.Tensor, ys=None, workspace=None):
+    """Layers l = 0..L-1: y[l] = BitLinear(packs[l], gammas[l])(y[l-1]), y[-1] = x.
+    `ys` (optional) are the output tensors, one per layer; a layer's output
+    may not be its own input (ping-pong buffers are fine).  Returns ys."""
+    _bits16(x, "x")
+    if len(packs) != len(gammas) or not packs:
+        raise ValueError("packs and gammas must be non-empty lists of equal length")
+    M = x.shape[0]
+    for p, g in zip(packs, gammas):
+        _dev(p, "packed")
+        _dev(g, "gamma")
+    if ys is None:
+        ys = [torch.empty((M, p.shape[0]), dtype=torch.bfloat16, device=x.device) for p in packs]
+    for y in ys:
+        _bits16(y, "y")
+    L, Ns, Ks, P, G, Y = _host_arrays(packs, gammas, ys, x)
+    nb = lib().bitnet_linear_chain_workspace_size(L, Ns, Ks, M)
+    ws = _workspace(nb, x.device, workspace)
+    st = lib().bitnet_linear_chain(L, P, G, Ns, Ks, _ptr(x), M, Y, _ptr(ws), nb, _stream())
+    _check("bitnet_linear_chain", st)
+    return ys
 
 
 def bitnet_linear_noalloc(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, y=None):

@@ -15,7 +15,8 @@ bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* ga
                                   int64_t K, int8_t* xq, int64_t ld_q, bool perm, float* scale,
                                   int32_t* rowsum, double* sumsq, int8_t* xq_natural,
                                   cudaStream_t stream);
-bitnet_status bitnet_gemv_launch(int mode, GemvArgs a, int num_sms, cudaStream_t stream);
+bitnet_status bitnet_decode_launch(const DecodeOp* ops, int nops, int M, unsigned int* bar,
+                                   int num_sms, cudaStream_t stream);
 bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
                                  const uint8_t* w1, GemmArgs a, int bn, int num_sms,
                                  cudaStream_t stream);
@@ -125,13 +126,17 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
 
 struct FfnWs {
   bool gemv;
-  size_t h, xq1, s1, rs1, ss1, xq2, s2, rs2, ss2, acc0, acc1, total;
+  size_t bar, h, xq1, s1, rs1, ss1, xq2, s2, rs2, ss2, acc0, acc1, total;
 };
 
 FfnWs ffn_ws_layout(int64_t M, int64_t H, int64_t I) {
   FfnWs w{};
   w.gemv = gemv_fits(M, H) && gemv_fits(M, I);
   size_t off = 0;
+  if (w.gemv) {   // grid-barrier word of the one-launch decode program
+    w.bar = off;
+    off += 256;
+  }
   w.h = off;
   off += al256((size_t)M * I * 4);
   if (!w.gemv) {
@@ -236,12 +241,13 @@ bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N
   cudaStream_t s = as_stream(stream);
   const LinearPath p = linear_path(M, K);
   if (p == kPathGemv) {
-    GemvArgs a{};
+    DecodeOp a{};
+    a.mode = kLinear;
     a.w0 = packed; a.gamma0 = gamma;
-    a.N = (int)N; a.K = (int)K; a.M = (int)M;
+    a.N = (int)N; a.K = (int)K;
     a.x = x;
     a.y = y; a.y_f32 = y_f32; a.acc0 = acc;
-    return bitnet_gemv_launch(kLinear, a, d.num_sms, s);
+    return bitnet_decode_launch(&a, 1, (int)M, nullptr, d.num_sms, s);
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int8_t* xq = reinterpret_cast<int8_t*>(ws + L.xq);
@@ -302,20 +308,24 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* h = reinterpret_cast<float*>(ws + L.h);
   if (L.gemv) {
-    GemvArgs g{};
+    // one launch: gate/up, grid barrier, down (down's weights stream in
+    // while gate/up finishes)
+    DecodeOp ops[2] = {};
+    DecodeOp& g = ops[0];
+    g.mode = kGlu;
     g.w0 = gate; g.gamma0 = gamma_gate; g.w1 = up; g.gamma1 = gamma_up;
-    g.N = (int)I; g.K = (int)H; g.M = (int)M;
+    g.N = (int)I; g.K = (int)H;
     g.x = x; g.gain = norm1_w;
     g.h = dbg.h ? dbg.h : h;
     g.acc0 = dbg.acc_gate; g.acc1 = dbg.acc_up; g.xq_dbg = dbg.xq1;
-    st = bitnet_gemv_launch(kGlu, g, d.num_sms, s);
-    if (st != BITNET_OK) return st;
-    GemvArgs dn{};
+    DecodeOp& dn = ops[1];
+    dn.mode = kDown;
     dn.w0 = down; dn.gamma0 = gamma_down;
-    dn.N = (int)H; dn.K = (int)I; dn.M = (int)M;
+    dn.N = (int)H; dn.K = (int)I;
     dn.x = g.h; dn.gain = norm2_w; dn.xnorm = x; dn.H = (int)H; dn.eps = eps;
     dn.y = y; dn.y_f32 = dbg.y_f32; dn.acc0 = dbg.acc_down; dn.xq_dbg = dbg.xq2;
-    return bitnet_gemv_launch(kDown, dn, d.num_sms, s);
+    unsigned int* bar = reinterpret_cast<unsigned int*>(ws + L.bar);
+    return bitnet_decode_launch(ops, 2, (int)M, bar, d.num_sms, s);
   }
   int8_t* xq1 = reinterpret_cast<int8_t*>(ws + L.xq1);
   float* s1 = reinterpret_cast<float*>(ws + L.s1);
@@ -358,6 +368,82 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
     if (cudaMemsetAsync(dn.acc_ws0, 0, (size_t)M * H * 4, s) != cudaSuccess) return BITNET_ERR_CUDA;
   }
   return bitnet_gemm_launch(2 /*down*/, xq2, down, nullptr, dn, bn_d, d.num_sms, s);
+}
+
+size_t bitnet_linear_chain_workspace_size(int64_t L, const int64_t* N, const int64_t* K,
+                                          int64_t M) {
+  if (L < 1 || !N || !K || M < 1) return 0;
+  size_t lin = 0;
+  for (int64_t l = 0; l < L; ++l) {
+    if (N[l] < 1 || K[l] < 4) return 0;
+    const size_t b = linear_ws_layout(M, N[l], K[l]).total;
+    if (b > lin) lin = b;
+  }
+  return 256 + lin;   // grid-barrier word, then bitnet_linear's scratch
+}
+
+bitnet_status bitnet_linear_chain(int64_t L, const uint8_t* const* packed,
+                                  const float* const* gamma, const int64_t* N, const int64_t* K,
+                                  const uint16_t* x, int64_t M, uint16_t* const* y,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (L < 1 || !packed || !gamma || !N || !K || !x || !y) return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || M > 0x7fffffff) return BITNET_ERR_SHAPE;
+  if (!aligned16(x)) return BITNET_ERR_ALIGN;
+  for (int64_t l = 0; l < L; ++l) {
+    if (!packed[l] || !gamma[l] || !y[l]) return BITNET_ERR_INVALID_ARG;
+    if (N[l] < 1 || K[l] < 4 || K[l] % 4 != 0 || K[l] > 524288 || N[l] > 0x7fffffff)
+      return BITNET_ERR_SHAPE;
+    if (l > 0 && K[l] != N[l - 1]) return BITNET_ERR_SHAPE;
+    if (!aligned16(packed[l]) || !aligned16(y[l]) || ((uintptr_t)gamma[l] & 3u))
+      return BITNET_ERR_ALIGN;
+    // a layer's output may not overlap its own input (the CTAs of one
+    // launch read the input while others already write the output)
+    const uintptr_t in = reinterpret_cast<uintptr_t>(l == 0 ? x : y[l - 1]);
+    const uintptr_t out = reinterpret_cast<uintptr_t>(y[l]);
+    const uintptr_t in_end = in + (uintptr_t)(M * K[l] * 2);
+    const uintptr_t out_end = out + (uintptr_t)(M * N[l] * 2);
+    if (in < out_end && out < in_end) return BITNET_ERR_INVALID_ARG;
+  }
+  const size_t need = bitnet_linear_chain_workspace_size(L, N, K, M);
+  if (!workspace || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  unsigned int* bar = reinterpret_cast<unsigned int*>(ws);
+  DecodeOp ops[kMaxProgramOps];
+  int64_t l = 0;
+  while (l < L) {
+    if (!gemv_fits(M, K[l])) {
+      // a layer outside the decode kernel's range: one bitnet_linear call
+      st = bitnet_linear(packed[l], gamma[l], N[l], K[l], l == 0 ? x : y[l - 1], M, y[l],
+                         nullptr, nullptr, ws + 256, workspace_bytes - 256, stream);
+      if (st != BITNET_OK) return st;
+      ++l;
+      continue;
+    }
+    // the longest run of decode-range layers (at most kMaxProgramOps) as
+    // one program
+    int n = 0;
+    while (l + n < L && n < kMaxProgramOps && gemv_fits(M, K[l + n])) {
+      DecodeOp& o = ops[n];
+      o = DecodeOp{};
+      o.mode = kLinear;
+      o.w0 = packed[l + n];
+      o.gamma0 = gamma[l + n];
+      o.N = (int)N[l + n];
+      o.K = (int)K[l + n];
+      o.x = (l + n == 0) ? x : y[l + n - 1];
+      o.y = y[l + n];
+      ++n;
+    }
+    st = bitnet_decode_launch(ops, n, (int)M, bar, d.num_sms, s);
+    if (st != BITNET_OK) return st;
+    l += n;
+  }
+  return BITNET_OK;
 }
 
 bitnet_status bitnet_last_device_status(void* stream) {

@@ -9,49 +9,99 @@
 // plane t = word & (0x03030303 << 2t) holds, byte b, the code of k = 4b + t
 // times 4^t, and the activations sit in shared memory in the matching order.
 //
-// Layout of work: one CTA per SM-slot owns a contiguous range of output rows;
-// warp 8 is the producer (bulk copies of whole rows, a few stages ahead);
-// warps 0..7 each take blocks of 4 rows, lane l reading words l, l+32, ... of
-// each row, then a butterfly reduction across the warp leaves row r's total
-// in lane 8r.
+// A launch runs a decode program: one or more BitLinear steps ("ops") in
+// order, each reading what the one before it wrote (a chain of layers, or
+// the FFN block's gate/up step followed by its down step).  Weights never
+// depend on activations, so the producer warp streams the weights of all
+// ops back to back, as far ahead as the ring allows, while the consumer
+// warps run the ops one after the other; between two ops every CTA waits at
+// a grid barrier (a counter in global memory that each CTA bumps once its
+// outputs are written).  A program of more than one op is a cooperative
+// launch with one CTA per SM, so all CTAs are resident together.
 //
-// Programmatic dependent launch: the producer starts streaming weights
-// before griddepcontrol.wait, the consumers wait before reading activations.
+// Layout of work within an op: each CTA owns a contiguous range of output
+// rows; warp 16 is the producer (bulk copies of whole rows, a few stages
+// ahead); warps 0..15 take (block of RB rows, K-slice) items, lane l reading
+// words l, l+32, ... of each row, then a butterfly reduction across the warp
+// and shared-memory integer atomics combine the partial sums.
+//
+// Programmatic dependent launch (single-op programs): the producer starts
+// streaming weights before griddepcontrol.wait, the consumers wait before
+// reading activations.
 #include "common.cuh"
 
 namespace bitnet {
 
 enum GemvMode : int { kLinear = 0, kGlu = 1, kDown = 2 };
+constexpr int kModeLinear = 1 << kLinear;
+constexpr int kModeGlu = 1 << kGlu;
+constexpr int kModeDown = 1 << kDown;
 
-struct GemvArgs {
+// One BitLinear step of a decode program.
+struct DecodeOp {
   const uint8_t* w0;      // packed [N, K/4]   (Glu: gate)
   const float* gamma0;
   const uint8_t* w1;      // Glu: up
   const float* gamma1;
-  int N, K, M;
   const void* x;          // Linear/Glu: bf16 [M,K]; Down: fp32 h' [M,K]
   const float* gain;      // optional [K] (RMSNorm weight)
   const uint16_t* xnorm;  // Down: block input x [M,H] (for r1)
-  int H;
-  float eps;
   uint16_t* y;            // Linear/Down [M,N]
   float* y_f32;           // optional [M,N]
   int32_t* acc0;          // optional [M,N]
   int32_t* acc1;          // optional [M,N] (Glu up)
   float* h;               // Glu output h' [M,N]
   int8_t* xq_dbg;         // optional natural-layout x_q [M,K], written by CTA 0
-  int rows_per_stage;     // multiple of 4
-  int stages;             // 2..8
-  int wk;                 // K-slices per 4-row block
+  int N, K, H;
+  float eps;
+  int mode;
+  int rb;                 // rows per work block (4, or 8 for one long-row matrix)
+  int rows_per_stage;     // multiple of rb
+  int wk;                 // K-slices per row block (a power of two)
 };
 
-constexpr int kConsumerWarps = 16;
+constexpr int kMaxProgramOps = 64;
+
+template <int CAP>
+struct DecodeProgram {
+  int nops, M, stages;
+  uint32_t stage_bytes;   // bytes per ring stage (a multiple of 16)
+  uint32_t xbytes;        // bytes of the activation area (a multiple of 128)
+  uint32_t acc_words;     // integer accumulators per parity
+  unsigned int* bar;      // grid barrier counter, zero at launch (nops > 1)
+  DecodeOp op[CAP];
+};
+
+constexpr int kConsumerWarps = 15;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxTok = 8;
 constexpr uint32_t kCopyChunk = 4096;   // bytes per bulk copy (a multiple of 16)
 
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+
+// Grid barrier between the ops of a program.  Arrive: after the CTA's
+// consumer barrier (all its outputs written), one thread makes them visible
+// at GPU scope and bumps the counter.  Wait: one thread polls the counter
+// with acquire loads, bounded by kWaitLimitNs.
+__device__ __forceinline__ void grid_arrive(unsigned int* bar) {
+  __threadfence();
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
+}
+__device__ __forceinline__ bool grid_wait(const unsigned int* bar, unsigned int target) {
+  uint64_t t0 = 0;
+  for (int it = 0;; ++it) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+    if (v >= target) return true;
+    if (it == 0) {
+      t0 = globaltimer_ns();
+    } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(BITNET_ERR_TIMEOUT);
+      return false;
+    }
+  }
 }
 
 // Halving step of the butterfly: n values -> n/2, exchanging with lane ^ off.
@@ -66,27 +116,23 @@ __device__ __forceinline__ void halve(const int (&v)[N], int (&o)[N / 2], int of
   }
 }
 
-__device__ __forceinline__ float load_src(const void* x, bool f32, int64_t idx) {
-  if (f32) return static_cast<const float*>(x)[idx];
-  return bf16_bits_to_float(static_cast<const uint16_t*>(x)[idx]);
-}
-
 // 16 consecutive activations (one group) as floats: two 16-byte loads of
-// bf16 bits, or four of fp32.
+// bf16 bits, or four of fp32.  Loads go to L2 (.cg): in a program the
+// activations were written by other CTAs of the same launch.
 template <bool kF32>
 __device__ __forceinline__ void load_group16(const void* x, int64_t idx, float (&v)[16]) {
   if (kF32) {
     const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + idx);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 t = p[i];
+      const float4 t = __ldcg(p + i);
       v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
     }
   } else {
     const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + idx);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const uint4 t = p[i];
+      const uint4 t = __ldcg(p + i);
       const uint32_t w[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -106,8 +152,102 @@ __device__ __forceinline__ void load_gain16(const float* g, int64_t idx, float (
   }
 }
 
-template <int MODE, int MT, int MM, int RB>
-__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
+// Dynamic shared memory of the decode kernel: [0,128) full/empty mbarriers
+// (up to 8 stages each); [128,512) per-token scalars and the grid-barrier
+// flag; [512,4096) warp partials; then the permuted activations (xbytes),
+// the integer accumulators (2 parities x acc_words) and the ring (stages x
+// stage_bytes).  Fixed areas are addressed from the array itself, so they
+// cost no registers.
+extern __shared__ __align__(128) uint8_t g_decode_smem[];
+
+struct DecodeSmem {   // the variable part of the layout (from the program)
+  int S;
+  uint32_t stage_bytes, xbytes, acc_words;
+  __device__ __forceinline__ uint64_t* full() const {
+    return reinterpret_cast<uint64_t*>(g_decode_smem);
+  }
+  __device__ __forceinline__ uint64_t* empty() const { return full() + 8; }
+  __device__ __forceinline__ float* tok_d0() const {
+    return reinterpret_cast<float*>(g_decode_smem + 128 + 4 * kMaxTok);
+  }
+  __device__ __forceinline__ float* tok_d1() const { return tok_d0() + kMaxTok; }
+  __device__ __forceinline__ float* tok_f() const { return tok_d1() + kMaxTok; }
+  __device__ __forceinline__ int* tok_rs() const {
+    return reinterpret_cast<int*>(tok_f() + kMaxTok);
+  }
+  __device__ __forceinline__ volatile int* fail() const { return tok_rs() + kMaxTok; }
+  // output pointers of the running op (y, y_f32, acc0, acc1, h), [320,360)
+  __device__ __forceinline__ uint64_t* outp() const {
+    return reinterpret_cast<uint64_t*>(g_decode_smem + 320);
+  }
+  __device__ __forceinline__ float* red_f() const {   // [warps][8 tok]
+    return reinterpret_cast<float*>(g_decode_smem + 512);
+  }
+  __device__ __forceinline__ int* red_i() const {     // [warps][8]
+    return reinterpret_cast<int*>(g_decode_smem + 1024);
+  }
+  __device__ __forceinline__ double* red_d() const {  // [warps][8][2]
+    return reinterpret_cast<double*>(g_decode_smem + 2048);
+  }
+  __device__ __forceinline__ uint8_t* xperm() const { return g_decode_smem + 4096; }
+  __device__ __forceinline__ int* acc_s() const {
+    return reinterpret_cast<int*>(g_decode_smem + 4096 + xbytes);
+  }
+  __device__ __forceinline__ uint8_t* ring() const {
+    return g_decode_smem + 4096 + xbytes + ((2 * acc_words * 4 + 127) / 128) * 128;
+  }
+};
+
+__device__ __forceinline__ void op_rows(const DecodeOp& o, int& n0, int& n1) {
+  n0 = (int)(((int64_t)blockIdx.x * o.N) / gridDim.x);
+  n1 = (int)(((int64_t)(blockIdx.x + 1) * o.N) / gridDim.x);
+}
+
+// Producer (one thread): bulk copies of this CTA's rows of every op, in
+// program order, into the ring; `gc` counts stages over the whole program.
+template <int CAP>
+__device__ void produce(const DecodeProgram<CAP>& p, const DecodeSmem& sm) {
+  const uint64_t pol = policy_evict_first();
+  const int S = sm.S;
+  int gc = 0;
+  for (int i = 0; i < p.nops; ++i) {
+    const DecodeOp& o = p.op[i];
+    const bool two = o.mode == kGlu;
+    const int Kb = o.K >> 2;
+    int n0, n1;
+    op_rows(o, n0, n1);
+    const int RS = o.rows_per_stage;
+    const int nchunks = (n1 - n0 + RS - 1) / RS;
+    for (int c = 0; c < nchunks; ++c, ++gc) {
+      const int s = gc % S;
+      if (gc >= S && !mbar_wait(&sm.empty()[s], ((gc / S) - 1) & 1)) return;
+      const int r0 = n0 + c * RS;
+      const int nr = min(RS, n1 - r0);
+      const uint32_t bytes = (uint32_t)nr * Kb;
+      mbar_arrive_expect_tx(&sm.full()[s], two ? 2 * bytes : bytes);
+      uint8_t* dst = sm.ring() + (size_t)s * sm.stage_bytes;
+      // several 4 KB copies per stage keep more requests in flight than one
+      // large copy
+      for (uint32_t off = 0; off < bytes; off += kCopyChunk) {
+        const uint32_t nb = bytes - off < kCopyChunk ? bytes - off : kCopyChunk;
+        bulk_g2s(dst + off, o.w0 + (int64_t)r0 * Kb + off, nb, &sm.full()[s], pol);
+        if (two)
+          bulk_g2s(dst + (size_t)RS * Kb + off, o.w1 + (int64_t)r0 * Kb + off, nb,
+                   &sm.full()[s], pol);
+      }
+    }
+  }
+}
+
+// Consumers (warps 0..15): one op = prologue (quantise the op's input into
+// the permuted layout) + main loop over this CTA's stages of the op.
+// `ok` false: skip the arithmetic and the stores but keep the ring moving.
+// kReload: the op lives at a run-time index of the program; its output
+// pointers are parked in shared memory by the prologue and read back at each
+// stage's epilogue instead of being kept in registers through the main loop.
+template <int MODE, int MT, int MM, int RB, bool kReload>
+__device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const DecodeSmem& sm,
+                                       int& gc, const bool ok_in, bool& ring_ok) {
   // MM: token count rounded up to 1, 2, 4 or 8 (loops over tokens unroll to
   // MM, keeping the code small for single-token decode)
   constexpr int NMAT = (MODE == kGlu) ? 2 : 1;
@@ -116,75 +256,36 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
   static_assert(NR == 4 || NR == 8, "4 or 8 values per block");
   constexpr bool kF32Src = (MODE == kDown);
   constexpr int NT = kConsumerWarps * 32;
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* empty = full + 8;
-  float* tok_s = reinterpret_cast<float*>(smem + 128);
-  float* tok_d0 = tok_s + kMaxTok;
-  float* tok_d1 = tok_d0 + kMaxTok;
-  float* tok_f = tok_d1 + kMaxTok;
-  int* tok_rs = reinterpret_cast<int*>(tok_f + kMaxTok);
-  float* red_f = reinterpret_cast<float*>(smem + 512);          // [16 warps][8 tok]
-  int* red_i = reinterpret_cast<int*>(smem + 1024);             // [16][8]
-  double* red_d = reinterpret_cast<double*>(smem + 2048);       // [16][8][2]
-  const int M = a.M, K = a.K, N = a.N;
+  float* tok_d0 = sm.tok_d0();
+  float* tok_d1 = sm.tok_d1();
+  float* tok_f = sm.tok_f();
+  int* tok_rs = sm.tok_rs();
+  float* red_f = sm.red_f();
+  int* red_i = sm.red_i();
+  double* red_d = sm.red_d();
+  uint8_t* xperm = sm.xperm();
+  const int K = a.K, N = a.N;
   const int Mpad = ((M + MT - 1) / MT) * MT;
-  const int RS = a.rows_per_stage, S = a.stages, WK = a.wk;   // WK is a power of two
+  const int RS = a.rows_per_stage, S = sm.S, WK = a.wk;   // WK is a power of two
   const int wk_log2 = __ffs(WK) - 1;
-  uint8_t* xperm = smem + 4096;
-  const int xbytes = ((Mpad * K + 127) / 128) * 128;
-  // per-stage integer accumulators [2 parity][NMAT][RS][kMaxTok]
-  int* acc_s = reinterpret_cast<int*>(xperm + xbytes);
-  const int acc_words = NMAT * RS * kMaxTok;
-  const int acc_bytes = ((2 * acc_words * 4 + 127) / 128) * 128;
-  uint8_t* ring = xperm + xbytes + acc_bytes;
+  const int acc_words = (int)sm.acc_words;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Kb = K >> 2;                   // bytes per packed row
   const int Kw = K >> 4;                   // 32-bit words per packed row
-  const int n0 = (int)(((int64_t)blockIdx.x * N) / gridDim.x);
-  const int n1 = (int)(((int64_t)(blockIdx.x + 1) * N) / gridDim.x);
+  int n0, n1;
+  op_rows(a, n0, n1);
   const int nchunks = (n1 - n0 + RS - 1) / RS;
-  const int stage_bytes = RS * Kb * NMAT;
-
-  if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (tid == 0) pdl_launch_dependents();
-
-  if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      for (int c = 0; c < nchunks; ++c) {
-        const int s = c % S;
-        if (c >= S && !mbar_wait(&empty[s], ((c / S) - 1) & 1)) break;
-        const int r0 = n0 + c * RS;
-        const int nr = min(RS, n1 - r0);
-        const uint32_t bytes = (uint32_t)nr * Kb;
-        mbar_arrive_expect_tx(&full[s], bytes * NMAT);
-        uint8_t* dst = ring + (size_t)s * stage_bytes;
-        // several 4 KB copies per stage keep more requests in flight than
-        // one large copy
-        for (uint32_t off = 0; off < bytes; off += kCopyChunk) {
-          const uint32_t nb = bytes - off < kCopyChunk ? bytes - off : kCopyChunk;
-          bulk_g2s(dst + off, a.w0 + (int64_t)r0 * Kb + off, nb, &full[s], pol);
-          if (NMAT == 2)
-            bulk_g2s(dst + (size_t)RS * Kb + off, a.w1 + (int64_t)r0 * Kb + off, nb, &full[s], pol);
-        }
-      }
-    }
-    return;
-  }
 
   // -------------------------------------------------------------- prologue
-  for (int i = tid; i < 2 * acc_words; i += NT) acc_s[i] = 0;
-  pdl_wait();
+  if (kReload && tid == 0) {   // read back after the prologue's barriers
+    uint64_t* op_out = sm.outp();
+    op_out[0] = reinterpret_cast<uint64_t>(a.y);
+    op_out[1] = reinterpret_cast<uint64_t>(a.y_f32);
+    op_out[2] = reinterpret_cast<uint64_t>(a.acc0);
+    op_out[3] = reinterpret_cast<uint64_t>(a.acc1);
+    op_out[4] = reinterpret_cast<uint64_t>(a.h);
+  }
   for (int i = M * K + tid * 16; i < Mpad * K; i += NT * 16)
     *reinterpret_cast<uint4*>(xperm + i) = make_uint4(0, 0, 0, 0);
 
@@ -367,20 +468,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
 
   // ------------------------------------------------------------- main loop
   // A stage holds RS whole rows (of each matrix).  Work items are (block of
-  // 4 rows, K-slice) pairs, WK slices per block, dealt to the 8 warps round
+  // RB rows, K-slice) pairs, WK slices per block, dealt to the 16 warps round
   // robin; each item's per-row totals are added into shared-memory integer
   // accumulators (exact, order-free), and after a barrier the stage's
   // outputs are finished from them.
   const uint32_t x_addr = smem_u32(xperm);
-  bool ok = true;
-  for (int c = 0; c < nchunks; ++c) {
-    const int s = c % S;
-    if (ok && !mbar_wait(&full[s], (c / S) & 1)) ok = false;
+  for (int c = 0; c < nchunks; ++c, ++gc) {
+    const int s = gc % S;
+    if (ring_ok && !mbar_wait(&sm.full()[s], (gc / S) & 1)) ring_ok = false;
+    const bool ok = ok_in && ring_ok;
     const int r0 = n0 + c * RS;
     const int nr = min(RS, n1 - r0);
-    int* acc = acc_s + (c & 1) * acc_words;
+    int* acc = sm.acc_s() + (gc & 1) * acc_words;
     if (ok) {
-      const uint32_t st_addr = smem_u32(ring + (size_t)s * stage_bytes);
+      const uint32_t st_addr = smem_u32(sm.ring() + (size_t)s * sm.stage_bytes);
       const int nitems = ((nr + RB - 1) / RB) * WK;
       for (int it = warp; it < nitems; it += kConsumerWarps) {
         const int b = it >> wk_log2, q = it & (WK - 1);
@@ -479,9 +580,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    if (lane == 0) mbar_arrive(&sm.empty()[s]);
     consumer_sync();
-    // finish this stage's outputs; clear the accumulators for stage c + 2
+    // finish this stage's outputs; clear the accumulators for stage gc + 2
+    uint16_t* out_y;
+    float* out_y32;
+    int32_t* out_acc0;
+    int32_t* out_acc1;
+    float* out_h;
+    if constexpr (kReload) {
+      const volatile uint64_t* op_out = sm.outp();
+      out_y = reinterpret_cast<uint16_t*>(op_out[0]);
+      out_y32 = reinterpret_cast<float*>(op_out[1]);
+      out_acc0 = reinterpret_cast<int32_t*>(op_out[2]);
+      out_acc1 = reinterpret_cast<int32_t*>(op_out[3]);
+      out_h = reinterpret_cast<float*>(op_out[4]);
+    } else {
+      out_y = a.y;
+      out_y32 = a.y_f32;
+      out_acc0 = a.acc0;
+      out_acc1 = a.acc1;
+      out_h = a.h;
+    }
     for (int o = tid; o < nr * M; o += NT) {
       const int row = o / M, m = o - row * M;
       const int n = r0 + row;
@@ -496,31 +616,108 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvArgs a) {
         const float g = __fmul_rn(__int2float_rn(ag), tok_d0[m]);
         const float u = __fmul_rn(__int2float_rn(au), tok_d1[m]);
         const float rg = fmaxf(g, 0.0f);
-        if (ok) a.h[oo] = __fmul_rn(__fmul_rn(rg, rg), u);
-        if (ok && a.acc0) a.acc0[oo] = ag;
-        if (ok && a.acc1) a.acc1[oo] = au;
+        if (ok) out_h[oo] = __fmul_rn(__fmul_rn(rg, rg), u);
+        if (ok && out_acc0) out_acc0[oo] = ag;
+        if (ok && out_acc1) out_acc1[oo] = au;
       } else {
         const int ac = *p0 - rsum;
         *p0 = 0;
         float y32 = __fmul_rn(__int2float_rn(ac), tok_d0[m]);
         if (MODE == kDown) y32 = __fmul_rn(y32, tok_f[m]);
         if (ok) {
-          a.y[oo] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
-          if (a.y_f32) a.y_f32[oo] = y32;
-          if (a.acc0) a.acc0[oo] = ac;
+          out_y[oo] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+          if (out_y32) out_y32[oo] = y32;
+          if (out_acc0) out_acc0[oo] = ac;
         }
       }
     }
   }
 }
 
-template <int MODE, int MT, int MM, int RB>
-static cudaError_t launch_one(const GemvArgs& a, int grid, size_t smem, cudaStream_t stream) {
+
+template <int MT, int MM, int CAP, int MODES>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ DecodeProgram<CAP> p) {
+  DecodeSmem sm;
+  sm.S = p.stages;
+  sm.stage_bytes = p.stage_bytes;
+  sm.xbytes = p.xbytes;
+  sm.acc_words = p.acc_words;
+  volatile int* fail = sm.fail();
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < sm.S; ++s) {
+      mbar_init(&sm.full()[s], 1);
+      mbar_init(&sm.empty()[s], kConsumerWarps);
+    }
+    fence_mbar_init();
+    *fail = 0;
+  }
+  __syncthreads();
+  if (tid == 0) pdl_launch_dependents();
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0) produce(p, sm);
+    return;
+  }
+
+  for (int i = tid; i < 2 * (int)sm.acc_words; i += kConsumerWarps * 32) sm.acc_s()[i] = 0;
+  const int M = p.M;
+  int gc = 0;
+  bool ok = true, ring_ok = true;
+  if constexpr (MODES == (kModeGlu | kModeDown)) {
+    // the FFN block: gate/up, then down (fixed op indices keep the ops'
+    // fields as kernel-parameter operands)
+    pdl_wait();
+    run_op<kGlu, MT, MM, 4, false>(p.op[0], M, sm, gc, ok, ring_ok);
+    consumer_sync();   // every h' value of this CTA is written
+    if (tid == 0) grid_arrive(p.bar);
+    if (tid == 0 && !grid_wait(p.bar, gridDim.x)) *fail = 1;
+    consumer_sync();
+    if (*fail) ok = false;
+    if constexpr (MM == 1) {
+      if (p.op[1].rb == 8) run_op<kDown, MT, MM, 8, false>(p.op[1], M, sm, gc, ok, ring_ok);
+      else run_op<kDown, MT, MM, 4, false>(p.op[1], M, sm, gc, ok, ring_ok);
+    } else {
+      run_op<kDown, MT, MM, 4, false>(p.op[1], M, sm, gc, ok, ring_ok);
+    }
+  } else {
+    static_assert(MODES == kModeLinear, "programs are Linear chains or the FFN block");
+    const int nops = CAP == 1 ? 1 : p.nops;
+    for (int i = 0; i < nops; ++i) {
+      const DecodeOp& o = p.op[CAP == 1 ? 0 : i];
+      if (i == 0) {
+        pdl_wait();
+      } else {
+        if (tid == 0 && ok && !grid_wait(p.bar, (unsigned int)i * gridDim.x)) *fail = 1;
+        consumer_sync();
+        if (*fail) ok = false;
+      }
+      // 8-row blocks only where the op's fields are parameter operands (a
+      // single-op program); chains use 4-row blocks
+      if constexpr (MM == 1 && CAP == 1) {
+        if (o.rb == 8) run_op<kLinear, MT, MM, 8, false>(o, M, sm, gc, ok, ring_ok);
+        else run_op<kLinear, MT, MM, 4, false>(o, M, sm, gc, ok, ring_ok);
+      } else {
+        run_op<kLinear, MT, MM, 4, (CAP > 1)>(o, M, sm, gc, ok, ring_ok);
+      }
+      if (i + 1 < nops) {
+        consumer_sync();   // every output of this CTA for op i is written
+        if (tid == 0) grid_arrive(p.bar);
+      }
+    }
+  }
+}
+
+template <int MT, int MM, int CAP, int MODES>
+static cudaError_t launch_program(const DecodeProgram<CAP>& p, int grid, size_t smem,
+                                  cudaStream_t stream) {
   static unsigned long long configured = 0;   // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(configured & (1ull << (dev & 63)))) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MODE, MT, MM, RB>,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<MT, MM, CAP, MODES>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e != cudaSuccess) return e;
     configured |= 1ull << (dev & 63);
@@ -531,19 +728,28 @@ static cudaError_t launch_one(const GemvArgs& a, int grid, size_t smem, cudaStre
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  if (p.nops > 1) {
+    // the grid barrier needs every CTA resident: the launch fails instead
+    // of starting if they cannot be
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+  }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<MODE, MT, MM, RB>, a);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<MT, MM, CAP, MODES>, p);
 }
 
-// Host-side planning: stage rows and ring depth under a shared-memory budget
-// that leaves room for a second CTA per SM (the next kernel in the stream).
-struct GemvPlan {
-  int grid, rows_per_stage, stages, wk;
-  size_t smem;
-};
+template <int CAP, int MODES>
+static cudaError_t launch_by_tokens(const DecodeProgram<CAP>& p, int grid, size_t smem,
+                                    cudaStream_t stream) {
+  if (p.M == 1) return launch_program<1, 1, CAP, MODES>(p, grid, smem, stream);
+  if (p.M == 2) return launch_program<2, 2, CAP, MODES>(p, grid, smem, stream);
+  if (p.M <= 4) return launch_program<4, 4, CAP, MODES>(p, grid, smem, stream);
+  return launch_program<4, 8, CAP, MODES>(p, grid, smem, stream);
+}
 
 // K-slices per row block: balance (blocks x slices) items over the warps
 // against the fixed cost of an item (reduction, shared atomics, set-up).
@@ -566,67 +772,96 @@ static int gemv_rows_per_block(int M, int K, int nmat) {
   return (nmat == 1 && M == 1 && K >= 8192) ? 8 : 4;
 }
 
-static GemvPlan plan_gemv(int M, int N, int K, int nmat, int num_sms, int MT) {
-  GemvPlan p{};
+// Host-side planning of a program: per op the rows per stage (stages of at
+// most 56 KB, as few as cover the CTA's rows, equally sized), the work-block
+// height and the K-slicing; for the program the ring stage size (the largest
+// op's) and as many stages as a 200 KB budget holds (2..8).
+template <int CAP>
+static bitnet_status plan_program(DecodeProgram<CAP>& p, int num_sms, int* grid_out,
+                                  size_t* smem_out) {
+  const int M = p.M;
+  const int MT = M == 1 ? 1 : (M == 2 ? 2 : 4);
   const int Mpad = ((M + MT - 1) / MT) * MT;
-  const size_t xbytes = (((size_t)Mpad * K + 127) / 128) * 128;
+  int grid = num_sms;
+  if (p.nops == 1) {
+    const int blocks = (p.op[0].N + 3) / 4;
+    grid = blocks < num_sms ? blocks : num_sms;
+  }
+  size_t stage = 16, xbytes = 128, accw = 1;
+  int total_chunks = 0;
+  for (int i = 0; i < p.nops; ++i) {
+    DecodeOp& o = p.op[i];
+    const int nmat = o.mode == kGlu ? 2 : 1;
+    const size_t row_bytes = (size_t)(o.K / 4) * nmat;
+    // 8-row blocks: single-op programs and the FFN's down step only
+    const int rb = (p.nops > 1 && o.mode == kLinear) ? 4 : gemv_rows_per_block(M, o.K, nmat);
+    const int rows_per_cta = (o.N + grid - 1) / grid;
+    int rs_max = (int)((56 * 1024) / row_bytes) / rb * rb;
+    if (rs_max < rb) rs_max = rb;
+    const int nch = (rows_per_cta + rs_max - 1) / rs_max;
+    int rs = (rows_per_cta + nch - 1) / nch;
+    rs = (rs + rb - 1) / rb * rb;
+    o.rb = rb;
+    o.rows_per_stage = rs;
+    o.wk = pick_wk(rs / rb, o.K / 16);
+    if ((size_t)rs * row_bytes > stage) stage = (size_t)rs * row_bytes;
+    const size_t xb = (((size_t)Mpad * o.K + 127) / 128) * 128;
+    if (xb > xbytes) xbytes = xb;
+    if ((size_t)nmat * rs * kMaxTok > accw) accw = (size_t)nmat * rs * kMaxTok;
+    total_chunks += nch;
+  }
   const size_t budget = 200 * 1024;
-  const size_t row_bytes = (size_t)(K / 4) * nmat;
-  int blocks = (N + 3) / 4;
-  p.grid = blocks < num_sms ? blocks : num_sms;
-  const int rows_per_cta = (N + p.grid - 1) / p.grid;
-  // stages of at most 56 KB, as few as cover the CTA's rows, equally sized
-  const int rb = gemv_rows_per_block(M, K, nmat);
-  int rs_max = (int)((56 * 1024) / row_bytes) / rb * rb;
-  if (rs_max < rb) rs_max = rb;
-  const int nch = (rows_per_cta + rs_max - 1) / rs_max;
-  int rs = (rows_per_cta + nch - 1) / nch;
-  rs = (rs + rb - 1) / rb * rb;
-  const size_t acc_bytes = ((2 * (size_t)nmat * rs * kMaxTok * 4 + 127) / 128) * 128;
+  const size_t acc_bytes = ((2 * accw * 4 + 127) / 128) * 128;
   const size_t head = 4096 + xbytes + acc_bytes;
-  const size_t ring = budget > head + 2 * (size_t)rs * row_bytes ? budget - head
-                                                                  : 2 * (size_t)rs * row_bytes;
-  int st = (int)(ring / ((size_t)rs * row_bytes));
+  int st = budget > head + 2 * stage ? (int)((budget - head) / stage) : 2;
   if (st > 8) st = 8;
+  if (st > total_chunks) st = total_chunks;
   if (st < 2) st = 2;
-  if (st > nch) st = nch < 2 ? 2 : nch;
-  p.rows_per_stage = rs;
   p.stages = st;
-  p.wk = pick_wk(rs / rb, K / 16);
-  p.smem = head + (size_t)st * rs * row_bytes;
-  return p;
+  p.stage_bytes = (uint32_t)stage;
+  p.xbytes = (uint32_t)xbytes;
+  p.acc_words = (uint32_t)accw;
+  *grid_out = grid;
+  *smem_out = head + (size_t)st * stage;
+  return *smem_out > 227 * 1024 ? BITNET_ERR_UNSUPPORTED : BITNET_OK;
+}
+
+template <int CAP, int MODES>
+static bitnet_status run_program(const DecodeOp* ops, int nops, int M, unsigned int* bar,
+                                 int num_sms, cudaStream_t stream) {
+  DecodeProgram<CAP> p{};
+  p.nops = nops;
+  p.M = M;
+  p.bar = bar;
+  for (int i = 0; i < nops; ++i) p.op[i] = ops[i];
+  int grid = 0;
+  size_t smem = 0;
+  const bitnet_status st = plan_program(p, num_sms, &grid, &smem);
+  if (st != BITNET_OK) return st;
+  if (nops > 1 && cudaMemsetAsync(bar, 0, sizeof(unsigned int), stream) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  return launch_by_tokens<CAP, MODES>(p, grid, smem, stream) == cudaSuccess ? BITNET_OK
+                                                                            : BITNET_ERR_CUDA;
 }
 
 }  // namespace bitnet
 
 using namespace bitnet;
 
-size_t bitnet_gemv_smem_bytes(int M, int N, int K, int nmat, int num_sms) {
-  const int MT = M == 1 ? 1 : (M == 2 ? 2 : 4);
-  return plan_gemv(M, N, K, nmat, num_sms, MT).smem;
-}
-
-bitnet_status bitnet_gemv_launch(int mode, GemvArgs a, int num_sms, cudaStream_t stream) {
-  const int nmat = mode == kGlu ? 2 : 1;
-  const int MT = a.M == 1 ? 1 : (a.M == 2 ? 2 : 4);
-  const GemvPlan p = plan_gemv(a.M, a.N, a.K, nmat, num_sms, MT);
-  if (p.smem > 227 * 1024) return BITNET_ERR_UNSUPPORTED;
-  a.rows_per_stage = p.rows_per_stage;
-  a.stages = p.stages;
-  a.wk = p.wk;
-  const int rb = gemv_rows_per_block(a.M, a.K, nmat);
-  cudaError_t e = cudaErrorInvalidValue;
-#define BITNET_GEMV_CASE(MODE_)                                                       \
-  if (mode == MODE_) {                                                                \
-    if (a.M == 1 && rb == 8) e = launch_one<MODE_, 1, 1, (MODE_ == kGlu ? 4 : 8)>(a, p.grid, p.smem, stream); \
-    else if (a.M == 1) e = launch_one<MODE_, 1, 1, 4>(a, p.grid, p.smem, stream);     \
-    else if (a.M == 2) e = launch_one<MODE_, 2, 2, 4>(a, p.grid, p.smem, stream);     \
-    else if (a.M <= 4) e = launch_one<MODE_, 4, 4, 4>(a, p.grid, p.smem, stream);     \
-    else e = launch_one<MODE_, 4, 8, 4>(a, p.grid, p.smem, stream);                   \
-  }
-  BITNET_GEMV_CASE(kLinear)
-  BITNET_GEMV_CASE(kGlu)
-  BITNET_GEMV_CASE(kDown)
-#undef BITNET_GEMV_CASE
-  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+// Runs ops[0..nops) as one decode program.  Supported programs: one Linear
+// op; gate/up (Glu) followed by down (Down); up to kMaxProgramOps Linear ops.
+// `bar` (one zeroed word per launch, set here) is needed when nops > 1.
+bitnet_status bitnet_decode_launch(const DecodeOp* ops, int nops, int M, unsigned int* bar,
+                                   int num_sms, cudaStream_t stream) {
+  if (nops < 1 || nops > kMaxProgramOps || M < 1 || M > kMaxTok) return BITNET_ERR_UNSUPPORTED;
+  if (nops > 1 && !bar) return BITNET_ERR_INVALID_ARG;
+  bool all_linear = true;
+  for (int i = 0; i < nops; ++i) all_linear = all_linear && ops[i].mode == kLinear;
+  if (nops == 1 && all_linear)
+    return run_program<1, kModeLinear>(ops, nops, M, bar, num_sms, stream);
+  if (nops == 2 && ops[0].mode == kGlu && ops[1].mode == kDown)
+    return run_program<2, kModeGlu | kModeDown>(ops, nops, M, bar, num_sms, stream);
+  if (all_linear)
+    return run_program<kMaxProgramOps, kModeLinear>(ops, nops, M, bar, num_sms, stream);
+  return BITNET_ERR_UNSUPPORTED;
 }

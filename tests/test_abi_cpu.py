@@ -49,7 +49,7 @@ def test_workspace_sizes_are_host_only(L):
     assert L.bitnet_linear_workspace_size(4096, 6912, 2560) >= 4096 * 2560
     assert L.bitnet_linear_workspace_size(64, 2560, 6912) >= 64 * 6912 + 64 * 2560 * 4
     assert L.bitnet_linear_workspace_size(8, 400, 68) >= 8 * 68        # ragged K
-    assert L.bitnet_ffn_workspace_size(1, 8192, 28672) == 28672 * 4
+    assert L.bitnet_ffn_workspace_size(1, 8192, 28672) == 256 + 28672 * 4   # barrier + h'
     assert L.bitnet_ffn_workspace_size(2048, 8192, 28672) > 2048 * 28672 * 4
 
 
@@ -103,3 +103,52 @@ def test_pack_quant_ffn_validation(L):
     assert f(*a) == 3
     a = list(args); a[16] = 16
     assert f(*a) == 4
+
+
+def _chain_args(Ns, Ks, ys, x=FAKE):
+    n = len(Ns)
+    I64 = ctypes.c_int64 * n
+    VP = ctypes.c_void_p * n
+    return (n, VP(*([FAKE] * n)), VP(*([FAKE] * n)), I64(*Ns), I64(*Ks), x, VP(*ys))
+
+
+def test_chain_workspace_and_validation(L):
+    I64 = ctypes.c_int64 * 2
+    # decode-range chains need only the barrier word
+    assert L.bitnet_linear_chain_workspace_size(2, I64(6912, 2560), I64(2560, 6912), 1) == 256
+    big = L.bitnet_linear_chain_workspace_size(2, I64(6912, 2560), I64(2560, 6912), 4096)
+    assert big == 256 + L.bitnet_linear_workspace_size(4096, 2560, 6912)
+    assert L.bitnet_linear_chain_workspace_size(0, I64(1, 1), I64(4, 4), 1) == 0
+    y0, y1 = 0x100000, 0x200000
+    n, P, G, N, K, x, Y = _chain_args([6912, 2560], [2560, 6912], [y0, y1])
+    ws, nb = FAKE, 256
+
+    def call(**kw):
+        a = dict(n=n, P=P, G=G, N=N, K=K, x=x, M=1, Y=Y, ws=ws, nb=nb)
+        a.update(kw)
+        return L.bitnet_linear_chain(a["n"], a["P"], a["G"], a["N"], a["K"], a["x"], a["M"],
+                                     a["Y"], a["ws"], a["nb"], None)
+
+    assert call(n=0) == 1
+    assert call(P=None) == 1
+    assert call(x=None) == 1
+    assert call(M=0) == 2
+    # layer 1's K must equal layer 0's N
+    _, _, _, N2, K2, _, _ = _chain_args([6912, 2560], [2560, 6000], [y0, y1])
+    assert call(N=N2, K=K2) == 2
+    assert call(x=MIS) == 3
+    _, _, _, _, _, _, Ymis = _chain_args([6912, 2560], [2560, 6912], [y0, MIS])
+    assert call(Y=Ymis) == 3
+    # a layer's output overlapping its own input
+    _, _, _, _, _, _, Yal = _chain_args([6912, 2560], [2560, 6912], [FAKE + 64, y1])
+    assert call(Y=Yal) == 1
+    _, _, _, _, _, _, Yal2 = _chain_args([6912, 2560], [2560, 6912], [y0, y0 + 16])
+    assert call(Y=Yal2) == 1
+    # ping-pong (y[2] == y[0]) is allowed by the aliasing rule; here it fails
+    # only on the missing workspace
+    n3, P3, G3, N3, K3, x3, Y3 = _chain_args([6912, 2560, 6912], [2560, 6912, 2560],
+                                             [y0, y1, y0])
+    assert L.bitnet_linear_chain(n3, P3, G3, N3, K3, x3, 1, Y3, None, 0, None) == 4
+    assert call(ws=None) == 4
+    assert call(nb=255) == 4
+    assert call(ws=MIS) == 3
