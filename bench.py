@@ -4,12 +4,11 @@
 Headline workload (one "step"): 2B-class decode, M = 1 token, a chain of 30
 layers x {up [6912,2560], down [2560,6912]} = 60 distinct packed matrices
 (265 MB of packed weights, larger than the 126 MB L2), each BitLinear fed the
-previous one's bf16 output: one bitnet_linear_chain call (one cooperative
-launch of the decode kernel running the 60 layers with a grid barrier between
-them), captured in a CUDA graph.  Per step the path runs activation quant
-(fused), the ternary int8 matmul and the dequant/bf16 store for all 60
-matrices.  value = packed-weight bytes streamed / device time (GB/s).  The
-same chain as 60 separate bitnet_linear calls is reported alongside.
+previous one's bf16 output: one bitnet_linear_chain call (60 decode-kernel
+launches with programmatic dependent launch), captured in a CUDA graph.  Per
+step the path runs activation quant (fused), the ternary int8 matmul and the
+dequant/bf16 store for all 60 matrices.  value = packed-weight bytes
+streamed / device time (GB/s).
 
 Secondary figures (same JSON line, "secondary"): prefill GEMM TOPS at M=4096,
 batched decode M in {4,16,64}, and the 100B-class FFN block at M=1 and 2048.
@@ -274,7 +273,7 @@ def chain_calls(B, packs, x, bufs):
     return cur
 
 
-class ChainProgram:
+class ChainCall:
     """The chain as one bitnet_linear_chain call (outputs ping-pong in bufs)."""
 
     def __init__(self, B, torch, packs, bufs, dev):
@@ -350,28 +349,22 @@ def secondary_measurements(B, inputs, torch, dev, stream, pk):
                                         "includes": "activation quant kernel + tcgen05 GEMM"}
         del g
     del xs, yu, yd, wsu, wsd
-    # batched decode: the same 60-layer chain with M tokens (M = 1: as 60
-    # separate bitnet_linear calls, for comparison with the one-launch chain)
+    # batched decode: the same 60-layer chain with M tokens
     packs = pk["_packs"]
-    for M in (1, 4, 16, 64):
+    for M in (4, 16, 64):
         x = torch.from_numpy(inputs.activations((M, HIDDEN), seed=0, outliers=True).view(np.int16)).to(dev)
         bufs = [torch.empty((M, INTER), dtype=torch.bfloat16, device=dev),
                 torch.empty((M, HIDDEN), dtype=torch.bfloat16, device=dev)]
-        if M == 1:
-            def run():
-                chain_calls(B, packs, x, bufs)
-        else:
-            prog = ChainProgram(B, torch, packs, bufs, dev)
+        prog = ChainCall(B, torch, packs, bufs, dev)
 
-            def run():
-                prog(x)
+        def run():
+            prog(x)
         g = capture(torch, run, stream)
         ms, _, _ = time_graph(torch, g, stream, 20, 3)
         t = ms / 20 * 1e-3
         nbytes = sum(p.numel() for p, _ in packs)
         ops = 2.0 * M * sum(p.numel() * 4 for p, _ in packs)
-        key = "decode_chain_M1_separate_calls" if M == 1 else f"decode_chain_M{M}"
-        out[key] = {"GB/s": round(nbytes / t / 1e9, 1),
+        out[f"decode_chain_M{M}"] = {"GB/s": round(nbytes / t / 1e9, 1),
                                      "TOPS": round(ops / t / 1e12, 2),
                                      "frac_hbm": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4),
                                      "us_per_step": round(t * 1e6, 1)}
@@ -469,7 +462,7 @@ def run_ours(args, world, rank, local):
     bufs = [torch.empty((1, INTER), dtype=torch.bfloat16, device=dev),
             torch.empty((1, HIDDEN), dtype=torch.bfloat16, device=dev)]
     torch.cuda.synchronize()
-    program = ChainProgram(B, torch, packs, bufs, dev)
+    program = ChainCall(B, torch, packs, bufs, dev)
     graph = capture(torch, lambda: program(x), stream)
     sampler = ClockSampler(local)
     sampler.start()
@@ -487,13 +480,12 @@ def run_ours(args, world, rank, local):
     step_s = ms / args.steps * 1e-3
     packed_bytes = sum(p.numel() for p, _ in packs)
     value = weak_scaling_value(world, packed_bytes, step_s) / 1e9
-    # roofline for the decode kernel: one launch per step runs all 60 layers;
-    # algorithmic bytes = packed weights + each layer's bf16 input and output
-    # + the gammas
-    alg_bytes = packed_bytes + n_mat // 2 * 2 * (2 * HIDDEN + 2 * INTER) + 4 * n_mat
-    launch_s = step_s
+    # roofline for the decode kernel: algorithmic bytes per launch (packed
+    # weights + bf16 input and output + gamma) / average launch time
+    alg_bytes = packed_bytes / n_mat + 2 * HIDDEN + 2 * INTER + 4
+    launch_s = step_s / n_mat
     achieved = alg_bytes / launch_s / 1e9
-    traffic = profile_traffic("decode_program_2b_m1.md")
+    traffic = profile_traffic("decode_gemv_2b_m1.md")
 
     # --------------------------------------------------- e2e through the API
     # per step: pinned host x -> device, one bitnet_linear_chain call through
@@ -543,19 +535,19 @@ def run_ours(args, world, rank, local):
             "config": {"workload": "2B-class decode GEMV chain, M=1: 30 layers x (up [6912,2560], "
                                    "down [2560,6912]) = 60 distinct 2-bit packed matrices, "
                                    "each fed the previous bf16 output; one bitnet_linear_chain "
-                                   "call (one cooperative launch) per step, in a CUDA graph",
+                                   "call (60 launches) per step, in a CUDA graph",
                        "M": 1, "matrices": n_mat, "packed_bytes_per_step": packed_bytes,
                        "l2": "inputs larger than L2 (265 MB packed weights > 126 MB L2), no flush",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
-                         "traffic": traffic, "kernel": "decode_kernel, 60-layer program",
+                         "traffic": traffic, "kernel": "decode_kernel<Linear,1,1>",
                          "peak_source": pk["source"],
                          "algorithmic_bytes_per_launch": alg_bytes,
                          "launch_us": round(launch_s * 1e6, 3)},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": args.steps,
+            "gpu_launches": n_mat * args.steps,
             "clocks": clocks,
             "device_status": B.bitnet_status_string(status),
             "graph_equals_eager": check_ok,

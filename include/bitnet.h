@@ -177,9 +177,9 @@ typedef struct {
  * debug  NULL or a host struct of optional device outputs (see above).
  * Requires M >= 1, H % 64 == 0, I % 64 == 0, H, I >= 64.  With M <= 8 and
  * M_pad * max(H, I) <= 65536 (M_pad = M rounded up to 1, 2 or a multiple of
- * 4) the whole block is one cooperative launch of the decode kernel (one CTA
- * per SM, a grid barrier between gate/up and down); larger M runs the
- * activation quantiser and the tensor-core kernel per step.
+ * 4) the block runs as two decode-kernel launches (gate/up with the h'
+ * epilogue, then down); larger M runs the activation quantiser and the
+ * tensor-core kernel per step.
  */
 BITNET_API size_t bitnet_ffn_workspace_size(int64_t M, int64_t H, int64_t I);
 BITNET_API bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
@@ -199,11 +199,9 @@ BITNET_API bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int
  * decode step runs them one after the other; the pages define no call that
  * runs several layers, this one only schedules them.
  *
- * Runs of consecutive layers in the decode kernel's range (M <= 8,
- * K % 64 == 0, M_pad * K <= 65536) execute as one cooperative launch of up
- * to 64 layers: the weights of later layers stream into shared memory while
- * earlier layers compute, and the CTAs meet at a grid barrier between
- * layers.  Other layers run as bitnet_linear calls.
+ * The layers are launched one after the other on `stream`, each exactly as
+ * bitnet_linear launches it (decode kernels start streaming their weights
+ * while the layer before them finishes).
  *
  * L        number of layers, >= 1.
  * packed, gamma, N, K, y   HOST arrays of L entries; packed[l], gamma[l] and
@@ -214,8 +212,8 @@ BITNET_API bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int
  * A layer's output may not overlap its input (y[l] vs y[l-1], y[0] vs x):
  * BITNET_ERR_INVALID_ARG.  Ping-pong buffers (y[l] == y[l-2]) are fine.
  * workspace  >= bitnet_linear_chain_workspace_size(L, N, K, M) bytes, device
- *          (contents need not be initialised; the call uses its first 256
- *          bytes as the grid-barrier counter).
+ *          (the largest layer's bitnet_linear scratch, reused by every
+ *          layer; 0 bytes, and a NULL workspace, when no layer needs any).
  * Other requirements and errors as bitnet_linear, per layer; all layers are
  * validated before anything is enqueued.
  */

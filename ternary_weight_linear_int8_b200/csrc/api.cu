@@ -15,8 +15,7 @@ bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* ga
                                   int64_t K, int8_t* xq, int64_t ld_q, bool perm, float* scale,
                                   int32_t* rowsum, double* sumsq, int8_t* xq_natural,
                                   cudaStream_t stream);
-bitnet_status bitnet_decode_launch(const DecodeOp* ops, int nops, int M, unsigned int* bar,
-                                   int num_sms, cudaStream_t stream);
+bitnet_status bitnet_decode_launch(const DecodeOp& op, int M, int num_sms, cudaStream_t stream);
 bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
                                  const uint8_t* w1, GemmArgs a, int bn, int num_sms,
                                  cudaStream_t stream);
@@ -126,17 +125,13 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
 
 struct FfnWs {
   bool gemv;
-  size_t bar, h, xq1, s1, rs1, ss1, xq2, s2, rs2, ss2, acc0, acc1, total;
+  size_t h, xq1, s1, rs1, ss1, xq2, s2, rs2, ss2, acc0, acc1, total;
 };
 
 FfnWs ffn_ws_layout(int64_t M, int64_t H, int64_t I) {
   FfnWs w{};
   w.gemv = gemv_fits(M, H) && gemv_fits(M, I);
   size_t off = 0;
-  if (w.gemv) {   // grid-barrier word of the one-launch decode program
-    w.bar = off;
-    off += 256;
-  }
   w.h = off;
   off += al256((size_t)M * I * 4);
   if (!w.gemv) {
@@ -247,7 +242,7 @@ bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N
     a.N = (int)N; a.K = (int)K;
     a.x = x;
     a.y = y; a.y_f32 = y_f32; a.acc0 = acc;
-    return bitnet_decode_launch(&a, 1, (int)M, nullptr, d.num_sms, s);
+    return bitnet_decode_launch(a, (int)M, d.num_sms, s);
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int8_t* xq = reinterpret_cast<int8_t*>(ws + L.xq);
@@ -308,24 +303,24 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* h = reinterpret_cast<float*>(ws + L.h);
   if (L.gemv) {
-    // one launch: gate/up, grid barrier, down (down's weights stream in
-    // while gate/up finishes)
-    DecodeOp ops[2] = {};
-    DecodeOp& g = ops[0];
+    // two decode launches: gate/up (h'), then down; the down kernel streams
+    // its weights while gate/up finishes (programmatic dependent launch)
+    DecodeOp g{};
     g.mode = kGlu;
     g.w0 = gate; g.gamma0 = gamma_gate; g.w1 = up; g.gamma1 = gamma_up;
     g.N = (int)I; g.K = (int)H;
     g.x = x; g.gain = norm1_w;
     g.h = dbg.h ? dbg.h : h;
     g.acc0 = dbg.acc_gate; g.acc1 = dbg.acc_up; g.xq_dbg = dbg.xq1;
-    DecodeOp& dn = ops[1];
+    st = bitnet_decode_launch(g, (int)M, d.num_sms, s);
+    if (st != BITNET_OK) return st;
+    DecodeOp dn{};
     dn.mode = kDown;
     dn.w0 = down; dn.gamma0 = gamma_down;
     dn.N = (int)H; dn.K = (int)I;
     dn.x = g.h; dn.gain = norm2_w; dn.xnorm = x; dn.H = (int)H; dn.eps = eps;
     dn.y = y; dn.y_f32 = dbg.y_f32; dn.acc0 = dbg.acc_down; dn.xq_dbg = dbg.xq2;
-    unsigned int* bar = reinterpret_cast<unsigned int*>(ws + L.bar);
-    return bitnet_decode_launch(ops, 2, (int)M, bar, d.num_sms, s);
+    return bitnet_decode_launch(dn, (int)M, d.num_sms, s);
   }
   int8_t* xq1 = reinterpret_cast<int8_t*>(ws + L.xq1);
   float* s1 = reinterpret_cast<float*>(ws + L.s1);
@@ -373,13 +368,13 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
 size_t bitnet_linear_chain_workspace_size(int64_t L, const int64_t* N, const int64_t* K,
                                           int64_t M) {
   if (L < 1 || !N || !K || M < 1) return 0;
-  size_t lin = 0;
+  size_t lin = 0;   // the largest layer's bitnet_linear scratch (reused)
   for (int64_t l = 0; l < L; ++l) {
     if (N[l] < 1 || K[l] < 4) return 0;
     const size_t b = linear_ws_layout(M, N[l], K[l]).total;
     if (b > lin) lin = b;
   }
-  return 256 + lin;   // grid-barrier word, then bitnet_linear's scratch
+  return lin;
 }
 
 bitnet_status bitnet_linear_chain(int64_t L, const uint8_t* const* packed,
@@ -405,43 +400,19 @@ bitnet_status bitnet_linear_chain(int64_t L, const uint8_t* const* packed,
     if (in < out_end && out < in_end) return BITNET_ERR_INVALID_ARG;
   }
   const size_t need = bitnet_linear_chain_workspace_size(L, N, K, M);
-  if (!workspace || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  }
   DevInfo d;
   bitnet_status st = device_info(&d);
   if (st != BITNET_OK) return st;
-  cudaStream_t s = as_stream(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  unsigned int* bar = reinterpret_cast<unsigned int*>(ws);
-  DecodeOp ops[kMaxProgramOps];
-  int64_t l = 0;
-  while (l < L) {
-    if (!gemv_fits(M, K[l])) {
-      // a layer outside the decode kernel's range: one bitnet_linear call
-      st = bitnet_linear(packed[l], gamma[l], N[l], K[l], l == 0 ? x : y[l - 1], M, y[l],
-                         nullptr, nullptr, ws + 256, workspace_bytes - 256, stream);
-      if (st != BITNET_OK) return st;
-      ++l;
-      continue;
-    }
-    // the longest run of decode-range layers (at most kMaxProgramOps) as
-    // one program
-    int n = 0;
-    while (l + n < L && n < kMaxProgramOps && gemv_fits(M, K[l + n])) {
-      DecodeOp& o = ops[n];
-      o = DecodeOp{};
-      o.mode = kLinear;
-      o.w0 = packed[l + n];
-      o.gamma0 = gamma[l + n];
-      o.N = (int)N[l + n];
-      o.K = (int)K[l + n];
-      o.x = (l + n == 0) ? x : y[l + n - 1];
-      o.y = y[l + n];
-      ++n;
-    }
-    st = bitnet_decode_launch(ops, n, (int)M, bar, d.num_sms, s);
+  // one launch per layer, in order on the stream; each decode kernel starts
+  // streaming its weights while the previous layer finishes
+  for (int64_t l = 0; l < L; ++l) {
+    st = bitnet_linear(packed[l], gamma[l], N[l], K[l], l == 0 ? x : y[l - 1], M, y[l], nullptr,
+                       nullptr, workspace, workspace_bytes, stream);
     if (st != BITNET_OK) return st;
-    l += n;
   }
   return BITNET_OK;
 }

@@ -9,35 +9,26 @@
 // plane t = word & (0x03030303 << 2t) holds, byte b, the code of k = 4b + t
 // times 4^t, and the activations sit in shared memory in the matching order.
 //
-// A launch runs a decode program: one or more BitLinear steps ("ops") in
-// order, each reading what the one before it wrote (a chain of layers, or
-// the FFN block's gate/up step followed by its down step).  Weights never
-// depend on activations, so the producer warp streams the weights of all
-// ops back to back, as far ahead as the ring allows, while the consumer
-// warps run the ops one after the other; between two ops every CTA waits at
-// a grid barrier (a counter in global memory that each CTA bumps once its
-// outputs are written).  A program of more than one op is a cooperative
-// launch with one CTA per SM, so all CTAs are resident together.
+// Layout of work: one CTA per SM owns a contiguous range of output rows.
+// The last warp is the producer: bulk copies of whole rows into a ring of
+// stages, several stages ahead.  The consumer warps take (block of RB rows,
+// K-slice) items, dealt round robin and continuing from stage to stage; lane
+// l reads words l, l+32, ... of each row, a butterfly reduction across the
+// warp gives each row's partial sum, and either the warp finishes the row
+// itself (one slice per block) or shared-memory integer atomics and a
+// per-block counter let the warp that adds the last slice finish it.  No
+// stage waits for all warps.
 //
-// Layout of work within an op: each CTA owns a contiguous range of output
-// rows; warp 16 is the producer (bulk copies of whole rows, a few stages
-// ahead); warps 0..15 take (block of RB rows, K-slice) items, lane l reading
-// words l, l+32, ... of each row, then a butterfly reduction across the warp
-// and shared-memory integer atomics combine the partial sums.
-//
-// Programmatic dependent launch (single-op programs): the producer starts
-// streaming weights before griddepcontrol.wait, the consumers wait before
-// reading activations.
+// Programmatic dependent launch: the producer starts streaming weights
+// before griddepcontrol.wait, the consumers wait before reading activations,
+// so a kernel's weight stream overlaps the end of the kernel before it.
 #include "common.cuh"
 
 namespace bitnet {
 
 enum GemvMode : int { kLinear = 0, kGlu = 1, kDown = 2 };
-constexpr int kModeLinear = 1 << kLinear;
-constexpr int kModeGlu = 1 << kGlu;
-constexpr int kModeDown = 1 << kDown;
 
-// One BitLinear step of a decode program.
+// Arguments of one decode launch (one BitLinear, or one FFN step).
 struct DecodeOp {
   const uint8_t* w0;      // packed [N, K/4]   (Glu: gate)
   const float* gamma0;
@@ -60,18 +51,18 @@ struct DecodeOp {
   int wk;                 // K-slices per row block (a power of two)
 };
 
-constexpr int kMaxProgramOps = 64;
-
-template <int CAP>
-struct DecodeProgram {
-  int nops, M, stages;
+// Kernel parameters: the op and the shared-memory plan.
+struct DecodeParams {
+  DecodeOp op;
+  int M, stages;
   uint32_t stage_bytes;   // bytes per ring stage (a multiple of 16)
   uint32_t xbytes;        // bytes of the activation area (a multiple of 128)
-  uint32_t acc_words;     // integer accumulators per parity
-  unsigned int* bar;      // grid barrier counter, zero at launch (nops > 1)
-  DecodeOp op[CAP];
+  uint32_t acc_words;     // integer accumulators per ring stage
+  uint32_t cnt_words;     // per-block completion counters per ring stage
 };
 
+// 15 consumer warps + 1 producer: 4 warps per scheduler, so up to 128
+// registers per thread at one CTA per SM.
 constexpr int kConsumerWarps = 15;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxTok = 8;
@@ -79,29 +70,6 @@ constexpr uint32_t kCopyChunk = 4096;   // bytes per bulk copy (a multiple of 16
 
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-}
-
-// Grid barrier between the ops of a program.  Arrive: after the CTA's
-// consumer barrier (all its outputs written), one thread makes them visible
-// at GPU scope and bumps the counter.  Wait: one thread polls the counter
-// with acquire loads, bounded by kWaitLimitNs.
-__device__ __forceinline__ void grid_arrive(unsigned int* bar) {
-  __threadfence();
-  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
-}
-__device__ __forceinline__ bool grid_wait(const unsigned int* bar, unsigned int target) {
-  uint64_t t0 = 0;
-  for (int it = 0;; ++it) {
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
-    if (v >= target) return true;
-    if (it == 0) {
-      t0 = globaltimer_ns();
-    } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      record_error(BITNET_ERR_TIMEOUT);
-      return false;
-    }
-  }
 }
 
 // Halving step of the butterfly: n values -> n/2, exchanging with lane ^ off.
@@ -117,22 +85,21 @@ __device__ __forceinline__ void halve(const int (&v)[N], int (&o)[N / 2], int of
 }
 
 // 16 consecutive activations (one group) as floats: two 16-byte loads of
-// bf16 bits, or four of fp32.  Loads go to L2 (.cg): in a program the
-// activations were written by other CTAs of the same launch.
+// bf16 bits, or four of fp32.
 template <bool kF32>
 __device__ __forceinline__ void load_group16(const void* x, int64_t idx, float (&v)[16]) {
   if (kF32) {
     const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + idx);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 t = __ldcg(p + i);
+      const float4 t = p[i];
       v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
     }
   } else {
     const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + idx);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const uint4 t = __ldcg(p + i);
+      const uint4 t = p[i];
       const uint32_t w[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -153,16 +120,17 @@ __device__ __forceinline__ void load_gain16(const float* g, int64_t idx, float (
 }
 
 // Dynamic shared memory of the decode kernel: [0,128) full/empty mbarriers
-// (up to 8 stages each); [128,512) per-token scalars and the grid-barrier
-// flag; [512,4096) warp partials; then the permuted activations (xbytes),
-// the integer accumulators (2 parities x acc_words) and the ring (stages x
+// (up to 8 stages each); [128,512) per-token scalars; [512,4096) warp
+// partials; then the
+// permuted activations (xbytes), per ring stage the integer accumulators
+// (acc_words) and block counters (cnt_words), and the ring (stages x
 // stage_bytes).  Fixed areas are addressed from the array itself, so they
 // cost no registers.
 extern __shared__ __align__(128) uint8_t g_decode_smem[];
 
-struct DecodeSmem {   // the variable part of the layout (from the program)
+struct DecodeSmem {   // the variable part of the layout (from the plan)
   int S;
-  uint32_t stage_bytes, xbytes, acc_words;
+  uint32_t stage_bytes, xbytes, acc_words, cnt_words;
   __device__ __forceinline__ uint64_t* full() const {
     return reinterpret_cast<uint64_t*>(g_decode_smem);
   }
@@ -172,14 +140,6 @@ struct DecodeSmem {   // the variable part of the layout (from the program)
   }
   __device__ __forceinline__ float* tok_d1() const { return tok_d0() + kMaxTok; }
   __device__ __forceinline__ float* tok_f() const { return tok_d1() + kMaxTok; }
-  __device__ __forceinline__ int* tok_rs() const {
-    return reinterpret_cast<int*>(tok_f() + kMaxTok);
-  }
-  __device__ __forceinline__ volatile int* fail() const { return tok_rs() + kMaxTok; }
-  // output pointers of the running op (y, y_f32, acc0, acc1, h), [320,360)
-  __device__ __forceinline__ uint64_t* outp() const {
-    return reinterpret_cast<uint64_t*>(g_decode_smem + 320);
-  }
   __device__ __forceinline__ float* red_f() const {   // [warps][8 tok]
     return reinterpret_cast<float*>(g_decode_smem + 512);
   }
@@ -193,8 +153,12 @@ struct DecodeSmem {   // the variable part of the layout (from the program)
   __device__ __forceinline__ int* acc_s() const {
     return reinterpret_cast<int*>(g_decode_smem + 4096 + xbytes);
   }
+  __device__ __forceinline__ int* cnt_s() const {
+    return acc_s() + ((S * acc_words + 31) / 32) * 32;
+  }
   __device__ __forceinline__ uint8_t* ring() const {
-    return g_decode_smem + 4096 + xbytes + ((2 * acc_words * 4 + 127) / 128) * 128;
+    return g_decode_smem + 4096 + xbytes + ((S * acc_words + 31) / 32) * 128 +
+           ((S * cnt_words + 31) / 32) * 128;
   }
 };
 
@@ -203,51 +167,42 @@ __device__ __forceinline__ void op_rows(const DecodeOp& o, int& n0, int& n1) {
   n1 = (int)(((int64_t)(blockIdx.x + 1) * o.N) / gridDim.x);
 }
 
-// Producer (one thread): bulk copies of this CTA's rows of every op, in
-// program order, into the ring; `gc` counts stages over the whole program.
-template <int CAP>
-__device__ void produce(const DecodeProgram<CAP>& p, const DecodeSmem& sm) {
+// Producer (one thread): bulk copies of this CTA's rows into the ring.
+__device__ __forceinline__ void produce(const DecodeOp& o, const DecodeSmem& sm) {
   const uint64_t pol = policy_evict_first();
   const int S = sm.S;
-  int gc = 0;
-  for (int i = 0; i < p.nops; ++i) {
-    const DecodeOp& o = p.op[i];
-    const bool two = o.mode == kGlu;
-    const int Kb = o.K >> 2;
-    int n0, n1;
-    op_rows(o, n0, n1);
-    const int RS = o.rows_per_stage;
-    const int nchunks = (n1 - n0 + RS - 1) / RS;
-    for (int c = 0; c < nchunks; ++c, ++gc) {
-      const int s = gc % S;
-      if (gc >= S && !mbar_wait(&sm.empty()[s], ((gc / S) - 1) & 1)) return;
-      const int r0 = n0 + c * RS;
-      const int nr = min(RS, n1 - r0);
-      const uint32_t bytes = (uint32_t)nr * Kb;
-      mbar_arrive_expect_tx(&sm.full()[s], two ? 2 * bytes : bytes);
-      uint8_t* dst = sm.ring() + (size_t)s * sm.stage_bytes;
-      // several 4 KB copies per stage keep more requests in flight than one
-      // large copy
-      for (uint32_t off = 0; off < bytes; off += kCopyChunk) {
-        const uint32_t nb = bytes - off < kCopyChunk ? bytes - off : kCopyChunk;
-        bulk_g2s(dst + off, o.w0 + (int64_t)r0 * Kb + off, nb, &sm.full()[s], pol);
-        if (two)
-          bulk_g2s(dst + (size_t)RS * Kb + off, o.w1 + (int64_t)r0 * Kb + off, nb,
-                   &sm.full()[s], pol);
-      }
+  const bool two = o.mode == kGlu;
+  const int Kb = o.K >> 2;
+  int n0, n1;
+  op_rows(o, n0, n1);
+  const int RS = o.rows_per_stage;
+  const int nchunks = (n1 - n0 + RS - 1) / RS;
+  for (int c = 0; c < nchunks; ++c) {
+    const int s = c % S;
+    if (c >= S && !mbar_wait(&sm.empty()[s], ((c / S) - 1) & 1)) return;
+    const int r0 = n0 + c * RS;
+    const int nr = min(RS, n1 - r0);
+    const uint32_t bytes = (uint32_t)nr * Kb;
+    mbar_arrive_expect_tx(&sm.full()[s], two ? 2 * bytes : bytes);
+    uint8_t* dst = sm.ring() + (size_t)s * sm.stage_bytes;
+    // several 4 KB copies per stage keep more requests in flight than one
+    // large copy
+    for (uint32_t off = 0; off < bytes; off += kCopyChunk) {
+      const uint32_t nb = bytes - off < kCopyChunk ? bytes - off : kCopyChunk;
+      bulk_g2s(dst + off, o.w0 + (int64_t)r0 * Kb + off, nb, &sm.full()[s], pol);
+      if (two)
+        bulk_g2s(dst + (size_t)RS * Kb + off, o.w1 + (int64_t)r0 * Kb + off, nb, &sm.full()[s],
+                 pol);
     }
   }
 }
 
-// Consumers (warps 0..15): one op = prologue (quantise the op's input into
-// the permuted layout) + main loop over this CTA's stages of the op.
-// `ok` false: skip the arithmetic and the stores but keep the ring moving.
-// kReload: the op lives at a run-time index of the program; its output
-// pointers are parked in shared memory by the prologue and read back at each
-// stage's epilogue instead of being kept in registers through the main loop.
-template <int MODE, int MT, int MM, int RB, bool kReload>
+// Consumers: prologue (quantise the input into the permuted layout) and
+// main loop over this CTA's stages.  A failed wait (ring_ok false) skips the
+// arithmetic and the stores but keeps the ring moving.
+template <int MODE, int MT, int MM, int RB>
 __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const DecodeSmem& sm,
-                                       int& gc, const bool ok_in, bool& ring_ok) {
+                                       bool& ring_ok) {
   // MM: token count rounded up to 1, 2, 4 or 8 (loops over tokens unroll to
   // MM, keeping the code small for single-token decode)
   constexpr int NMAT = (MODE == kGlu) ? 2 : 1;
@@ -259,7 +214,6 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
   float* tok_d0 = sm.tok_d0();
   float* tok_d1 = sm.tok_d1();
   float* tok_f = sm.tok_f();
-  int* tok_rs = sm.tok_rs();
   float* red_f = sm.red_f();
   int* red_i = sm.red_i();
   double* red_d = sm.red_d();
@@ -276,15 +230,14 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
   int n0, n1;
   op_rows(a, n0, n1);
   const int nchunks = (n1 - n0 + RS - 1) / RS;
+  int gc = 0;   // stages consumed
 
   // -------------------------------------------------------------- prologue
-  if (kReload && tid == 0) {   // read back after the prologue's barriers
-    uint64_t* op_out = sm.outp();
-    op_out[0] = reinterpret_cast<uint64_t>(a.y);
-    op_out[1] = reinterpret_cast<uint64_t>(a.y_f32);
-    op_out[2] = reinterpret_cast<uint64_t>(a.acc0);
-    op_out[3] = reinterpret_cast<uint64_t>(a.acc1);
-    op_out[4] = reinterpret_cast<uint64_t>(a.h);
+  // gamma loads go out with the activation loads (their latencies overlap)
+  float gam0 = 0.f, gam1 = 0.f;
+  if (tid < M) {
+    gam0 = *a.gamma0;
+    if (MODE == kGlu) gam1 = *a.gamma1;
   }
   for (int i = M * K + tid * 16; i < Mpad * K; i += NT * 16)
     *reinterpret_cast<uint4*>(xperm + i) = make_uint4(0, 0, 0, 0);
@@ -292,6 +245,9 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
   // pass 1: per-token absmax of src*gain (and, for Down, sums of squares).
   // With one or two tokens and at most KEEPG groups of 16 per thread the
   // values stay in registers for pass 2 instead of being loaded again.
+  auto load_x = [&](int m, int g, float (&v)[16]) {
+    load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, v);
+  };
   constexpr int KEEPG = (MM == 1) ? 2 : 1;
   const bool keep = (MM <= 2) && Kw <= KEEPG * NT;
   float vk[KEEPG][MM][16];
@@ -309,7 +265,7 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
 #pragma unroll
         for (int m = 0; m < MM; ++m) {
           if (m < M) {
-            load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, vk[gi][m]);
+            load_x(m, g, vk[gi][m]);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float v = vk[gi][m][i];
@@ -330,7 +286,7 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
       for (int m = 0; m < MM; ++m) {
         if (m < M) {
           float v[16];
-          load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, v);
+          load_x(m, g, v);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float vg = a.gain ? __fmul_rn(v[i], gn[i]) : v[i];
@@ -385,8 +341,8 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
     float s = sc[0];
 #pragma unroll
     for (int mm = 1; mm < MM; ++mm) if (mm == m) s = sc[mm];
-    tok_d0[m] = __fdiv_rn(*a.gamma0, s);
-    if (MODE == kGlu) tok_d1[m] = __fdiv_rn(*a.gamma1, s);
+    tok_d0[m] = __fdiv_rn(gam0, s);
+    if (MODE == kGlu) tok_d1[m] = __fdiv_rn(gam1, s);
     if (MODE == kDown) {
       double s1 = 0.0, s2 = 0.0;
       for (int w = 0; w < kConsumerWarps; ++w) {
@@ -445,7 +401,7 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
       for (int m = 0; m < MM; ++m) {
         if (m < M) {
           float v[16];
-          load_group16<kF32Src>(a.x, (int64_t)m * K + g * 16, v);
+          load_x(m, g, v);
           quant_group(g, m, v, gn);
         }
       }
@@ -459,31 +415,63 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
     }
   }
   consumer_sync();
-  // the epilogue reads the row sums straight from the per-warp partials
-  if (tid < M) {
-    int t = 0;
-    for (int w = 0; w < kConsumerWarps; ++w) t += red_i[w * kMaxTok + tid];
-    tok_rs[tid] = t;
-  }
 
   // ------------------------------------------------------------- main loop
   // A stage holds RS whole rows (of each matrix).  Work items are (block of
-  // RB rows, K-slice) pairs, WK slices per block, dealt to the 16 warps round
-  // robin; each item's per-row totals are added into shared-memory integer
-  // accumulators (exact, order-free), and after a barrier the stage's
-  // outputs are finished from them.
+  // RB rows, K-slice) pairs, WK slices per block, dealt round robin to the
+  // consumer warps and continuing from stage to stage, so the load evens out
+  // over the whole op and no stage waits for all warps.  With one slice per
+  // block (WK == 1) the warp that reduces a block finishes its outputs from
+  // registers.  Otherwise every slice adds its per-row totals into exact
+  // integer accumulators in shared memory (one set per ring stage), and the
+  // warp that completes a block's last slice (per-block counter) finishes
+  // the block's outputs and clears the accumulators.
   const uint32_t x_addr = smem_u32(xperm);
+  const int cnt_words = (int)sm.cnt_words;
+  // dequantise and store one output (row `rr` of the current stage, token m)
+  auto finish = [&](int r0, int rr, int m, int v0, int v1) {
+    const int n = r0 + rr;
+    const int64_t oo = (int64_t)m * N + n;
+    // the token's row sum, from the per-warp partials (stable until the
+    // kernel ends)
+    int rsum = 0;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) rsum += red_i[w * kMaxTok + m];
+    if constexpr (MODE == kGlu) {
+      const int ag = v0 - rsum, au = v1 - rsum;
+      const float g = __fmul_rn(__int2float_rn(ag), tok_d0[m]);
+      const float u = __fmul_rn(__int2float_rn(au), tok_d1[m]);
+      const float rg = fmaxf(g, 0.0f);
+      a.h[oo] = __fmul_rn(__fmul_rn(rg, rg), u);
+      if (a.acc0) a.acc0[oo] = ag;
+      if (a.acc1) a.acc1[oo] = au;
+    } else {
+      const int ac = v0 - rsum;
+      float y32 = __fmul_rn(__int2float_rn(ac), tok_d0[m]);
+      if (MODE == kDown) y32 = __fmul_rn(y32, tok_f[m]);
+      a.y[oo] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+      if (a.y_f32) a.y_f32[oo] = y32;
+      if (a.acc0) a.acc0[oo] = ac;
+    }
+  };
+  int base = 0;   // the warp that takes item 0 of the current stage
   for (int c = 0; c < nchunks; ++c, ++gc) {
     const int s = gc % S;
-    if (ring_ok && !mbar_wait(&sm.full()[s], (gc / S) & 1)) ring_ok = false;
-    const bool ok = ok_in && ring_ok;
     const int r0 = n0 + c * RS;
     const int nr = min(RS, n1 - r0);
-    int* acc = sm.acc_s() + (gc & 1) * acc_words;
-    if (ok) {
+    const int nitems = ((nr + RB - 1) / RB) * WK;
+    int first = warp - base;
+    if (first < 0) first += kConsumerWarps;
+    base = (base + nitems) % kConsumerWarps;
+    // every warp waits for the stage's data before it releases the stage,
+    // also with no item in it: an early release could count towards the
+    // previous use of the stage, which slower warps may still be reading
+    if (ring_ok && !mbar_wait(&sm.full()[s], (gc / S) & 1)) ring_ok = false;
+    if (first < nitems && ring_ok) {
       const uint32_t st_addr = smem_u32(sm.ring() + (size_t)s * sm.stage_bytes);
-      const int nitems = ((nr + RB - 1) / RB) * WK;
-      for (int it = warp; it < nitems; it += kConsumerWarps) {
+      int* acc = sm.acc_s() + s * acc_words;
+      int* cnt = sm.cnt_s() + s * cnt_words;
+      for (int it = first; it < nitems; it += kConsumerWarps) {
         const int b = it >> wk_log2, q = it & (WK - 1);
         const int j0 = (q * Kw) / WK, j1 = ((q + 1) * Kw) / WK;
         uint32_t rowa[NR];             // shared-window byte address of each row
@@ -573,194 +561,69 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
               writer = (lane & 3) == 0;
             }
             const int m = tg + t;
-            if (writer && m < M && RB * b + row < nr)
-              atomicAdd(&acc[(mat * RS + RB * b + row) * kMaxTok + m], tot);
+            const int rr = RB * b + row;
+            if (WK == 1) {
+              // the whole row is in this lane: finish it here (Glu: the up
+              // total sits 4 lanes up)
+              const int up = (NMAT == 2) ? __shfl_down_sync(0xffffffffu, tot, 4) : 0;
+              if (writer && mat == 0 && m < M && rr < nr) finish(r0, rr, m, tot, up);
+            } else if (writer && m < M && rr < nr) {
+              atomicAdd(&acc[(mat * RS + rr) * kMaxTok + m], tot);
+            }
+          }
+        }
+        if (WK > 1) {
+          // the warp that adds a block's last slice finishes the block
+          __syncwarp();
+          int last = 0;
+          if (lane == 0) {
+            __threadfence_block();
+            last = atomicAdd(&cnt[b], 1) == WK - 1;
+          }
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (last) {
+            __threadfence_block();
+            const int rows_b = min(RB, nr - RB * b);
+            for (int o = lane; o < rows_b * M; o += 32) {
+              const int rr = RB * b + o / M, m = o % M;
+              int* p0 = &acc[rr * kMaxTok + m];
+              const int v0 = *p0;
+              *p0 = 0;
+              int v1 = 0;
+              if (NMAT == 2) {
+                int* p1 = &acc[(RS + rr) * kMaxTok + m];
+                v1 = *p1;
+                *p1 = 0;
+              }
+              finish(r0, rr, m, v0, v1);
+            }
+            if (lane == 0) cnt[b] = 0;
           }
         }
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty()[s]);
-    consumer_sync();
-    // finish this stage's outputs; clear the accumulators for stage gc + 2
-    uint16_t* out_y;
-    float* out_y32;
-    int32_t* out_acc0;
-    int32_t* out_acc1;
-    float* out_h;
-    if constexpr (kReload) {
-      const volatile uint64_t* op_out = sm.outp();
-      out_y = reinterpret_cast<uint16_t*>(op_out[0]);
-      out_y32 = reinterpret_cast<float*>(op_out[1]);
-      out_acc0 = reinterpret_cast<int32_t*>(op_out[2]);
-      out_acc1 = reinterpret_cast<int32_t*>(op_out[3]);
-      out_h = reinterpret_cast<float*>(op_out[4]);
-    } else {
-      out_y = a.y;
-      out_y32 = a.y_f32;
-      out_acc0 = a.acc0;
-      out_acc1 = a.acc1;
-      out_h = a.h;
-    }
-    for (int o = tid; o < nr * M; o += NT) {
-      const int row = o / M, m = o - row * M;
-      const int n = r0 + row;
-      const int64_t oo = (int64_t)m * N + n;
-      const int rsum = tok_rs[m];
-      int* p0 = &acc[row * kMaxTok + m];
-      if (MODE == kGlu) {
-        int* p1 = &acc[(RS + row) * kMaxTok + m];
-        const int ag = *p0 - rsum, au = *p1 - rsum;
-        *p0 = 0;
-        *p1 = 0;
-        const float g = __fmul_rn(__int2float_rn(ag), tok_d0[m]);
-        const float u = __fmul_rn(__int2float_rn(au), tok_d1[m]);
-        const float rg = fmaxf(g, 0.0f);
-        if (ok) out_h[oo] = __fmul_rn(__fmul_rn(rg, rg), u);
-        if (ok && out_acc0) out_acc0[oo] = ag;
-        if (ok && out_acc1) out_acc1[oo] = au;
-      } else {
-        const int ac = *p0 - rsum;
-        *p0 = 0;
-        float y32 = __fmul_rn(__int2float_rn(ac), tok_d0[m]);
-        if (MODE == kDown) y32 = __fmul_rn(y32, tok_f[m]);
-        if (ok) {
-          out_y[oo] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
-          if (out_y32) out_y32[oo] = y32;
-          if (out_acc0) out_acc0[oo] = ac;
-        }
-      }
-    }
   }
 }
 
-
-template <int MT, int MM, int CAP, int MODES>
-__global__ void __launch_bounds__(kThreads, 1)
-    decode_kernel(const __grid_constant__ DecodeProgram<CAP> p) {
-  DecodeSmem sm;
-  sm.S = p.stages;
-  sm.stage_bytes = p.stage_bytes;
-  sm.xbytes = p.xbytes;
-  sm.acc_words = p.acc_words;
-  volatile int* fail = sm.fail();
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) {
-    for (int s = 0; s < sm.S; ++s) {
-      mbar_init(&sm.full()[s], 1);
-      mbar_init(&sm.empty()[s], kConsumerWarps);
-    }
-    fence_mbar_init();
-    *fail = 0;
-  }
-  __syncthreads();
-  if (tid == 0) pdl_launch_dependents();
-
-  if (warp == kConsumerWarps) {
-    if (lane == 0) produce(p, sm);
-    return;
-  }
-
-  for (int i = tid; i < 2 * (int)sm.acc_words; i += kConsumerWarps * 32) sm.acc_s()[i] = 0;
-  const int M = p.M;
-  int gc = 0;
-  bool ok = true, ring_ok = true;
-  if constexpr (MODES == (kModeGlu | kModeDown)) {
-    // the FFN block: gate/up, then down (fixed op indices keep the ops'
-    // fields as kernel-parameter operands)
-    pdl_wait();
-    run_op<kGlu, MT, MM, 4, false>(p.op[0], M, sm, gc, ok, ring_ok);
-    consumer_sync();   // every h' value of this CTA is written
-    if (tid == 0) grid_arrive(p.bar);
-    if (tid == 0 && !grid_wait(p.bar, gridDim.x)) *fail = 1;
-    consumer_sync();
-    if (*fail) ok = false;
-    if constexpr (MM == 1) {
-      if (p.op[1].rb == 8) run_op<kDown, MT, MM, 8, false>(p.op[1], M, sm, gc, ok, ring_ok);
-      else run_op<kDown, MT, MM, 4, false>(p.op[1], M, sm, gc, ok, ring_ok);
-    } else {
-      run_op<kDown, MT, MM, 4, false>(p.op[1], M, sm, gc, ok, ring_ok);
-    }
-  } else {
-    static_assert(MODES == kModeLinear, "programs are Linear chains or the FFN block");
-    const int nops = CAP == 1 ? 1 : p.nops;
-    for (int i = 0; i < nops; ++i) {
-      const DecodeOp& o = p.op[CAP == 1 ? 0 : i];
-      if (i == 0) {
-        pdl_wait();
-      } else {
-        if (tid == 0 && ok && !grid_wait(p.bar, (unsigned int)i * gridDim.x)) *fail = 1;
-        consumer_sync();
-        if (*fail) ok = false;
-      }
-      // 8-row blocks only where the op's fields are parameter operands (a
-      // single-op program); chains use 4-row blocks
-      if constexpr (MM == 1 && CAP == 1) {
-        if (o.rb == 8) run_op<kLinear, MT, MM, 8, false>(o, M, sm, gc, ok, ring_ok);
-        else run_op<kLinear, MT, MM, 4, false>(o, M, sm, gc, ok, ring_ok);
-      } else {
-        run_op<kLinear, MT, MM, 4, (CAP > 1)>(o, M, sm, gc, ok, ring_ok);
-      }
-      if (i + 1 < nops) {
-        consumer_sync();   // every output of this CTA for op i is written
-        if (tid == 0) grid_arrive(p.bar);
-      }
-    }
-  }
-}
-
-template <int MT, int MM, int CAP, int MODES>
-static cudaError_t launch_program(const DecodeProgram<CAP>& p, int grid, size_t smem,
-                                  cudaStream_t stream) {
-  static unsigned long long configured = 0;   // one bit per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!(configured & (1ull << (dev & 63)))) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<MT, MM, CAP, MODES>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    if (e != cudaSuccess) return e;
-    configured |= 1ull << (dev & 63);
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  if (p.nops > 1) {
-    // the grid barrier needs every CTA resident: the launch fails instead
-    // of starting if they cannot be
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-  } else {
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-  }
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<MT, MM, CAP, MODES>, p);
-}
-
-template <int CAP, int MODES>
-static cudaError_t launch_by_tokens(const DecodeProgram<CAP>& p, int grid, size_t smem,
-                                    cudaStream_t stream) {
-  if (p.M == 1) return launch_program<1, 1, CAP, MODES>(p, grid, smem, stream);
-  if (p.M == 2) return launch_program<2, 2, CAP, MODES>(p, grid, smem, stream);
-  if (p.M <= 4) return launch_program<4, 4, CAP, MODES>(p, grid, smem, stream);
-  return launch_program<4, 8, CAP, MODES>(p, grid, smem, stream);
-}
-
-// K-slices per row block: balance (blocks x slices) items over the warps
-// against the fixed cost of an item (reduction, shared atomics, set-up).
-static int pick_wk(int nb, int Kw) {
+// K-slices per row block.  Items (block x slice) are dealt round robin over
+// the warps for the whole op, but only the stages in the ring at one time
+// can be worked on together; each item costs its 32-word steps plus a fixed
+// overhead (reduction, and with slices the shared atomics and counter).
+static int pick_wk(int rows_cta, int rs, int rb, int Kw, int stages, int nch) {
+  const int blocks_stage = (rs + rb - 1) / rb;
+  const int blocks_total = (rows_cta + rb - 1) / rb + (nch - 1);
+  const int window = stages < nch ? stages : nch;
   int best = 1;
   double best_cost = 1e30;
   for (int wk = 1; wk <= 32; wk *= 2) {
     if (wk > 1 && Kw / wk < 8) break;
-    const double rounds = (double)((nb * wk + kConsumerWarps - 1) / kConsumerWarps);
+    int par = blocks_stage * wk * window;
+    if (par > kConsumerWarps) par = kConsumerWarps;
+    const double rounds = (double)((blocks_total * wk + par - 1) / par);
     const double iters = (double)((Kw / wk + 31) / 32);
-    const double cost = rounds * (iters + 2.0);   // per-item reduction ~ two 32-word steps
+    const double cost = rounds * (iters + (wk > 1 ? 3.0 : 2.0));
     if (cost < best_cost - 1e-9) { best_cost = cost; best = wk; }
   }
   return best;
@@ -772,96 +635,149 @@ static int gemv_rows_per_block(int M, int K, int nmat) {
   return (nmat == 1 && M == 1 && K >= 8192) ? 8 : 4;
 }
 
-// Host-side planning of a program: per op the rows per stage (stages of at
-// most 56 KB, as few as cover the CTA's rows, equally sized), the work-block
-// height and the K-slicing; for the program the ring stage size (the largest
-// op's) and as many stages as a 200 KB budget holds (2..8).
-template <int CAP>
-static bitnet_status plan_program(DecodeProgram<CAP>& p, int num_sms, int* grid_out,
-                                  size_t* smem_out) {
+
+template <int MODE, int MT, int MM>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ DecodeParams p) {
+  DecodeSmem sm;
+  sm.S = p.stages;
+  sm.stage_bytes = p.stage_bytes;
+  sm.xbytes = p.xbytes;
+  sm.acc_words = p.acc_words;
+  sm.cnt_words = p.cnt_words;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < sm.S; ++s) {
+      mbar_init(&sm.full()[s], 1);
+      mbar_init(&sm.empty()[s], kConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) pdl_launch_dependents();
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0) produce(p.op, sm);
+    return;
+  }
+
+  {   // accumulators and block counters start (and stay, between uses) at zero
+    const int n_acc = sm.S * (int)sm.acc_words, n_cnt = sm.S * (int)sm.cnt_words;
+    for (int i = tid; i < n_acc; i += kConsumerWarps * 32) sm.acc_s()[i] = 0;
+    for (int i = tid; i < n_cnt; i += kConsumerWarps * 32) sm.cnt_s()[i] = 0;
+  }
+  bool ring_ok = true;
+  pdl_wait();
+  // 8-row blocks: one long-row matrix with one token (planned on the host)
+  if constexpr (MM == 1 && MODE != kGlu) {
+    if (p.op.rb == 8) {
+      run_op<MODE, MT, MM, 8>(p.op, p.M, sm, ring_ok);
+      return;
+    }
+  }
+  run_op<MODE, MT, MM, 4>(p.op, p.M, sm, ring_ok);
+}
+
+template <int MODE, int MT, int MM>
+static cudaError_t launch_decode(const DecodeParams& p, int grid, size_t smem,
+                                 cudaStream_t stream) {
+  static unsigned long long configured = 0;   // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(configured & (1ull << (dev & 63)))) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<MODE, MT, MM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    configured |= 1ull << (dev & 63);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<MODE, MT, MM>, p);
+}
+
+template <int MODE>
+static cudaError_t launch_by_tokens(const DecodeParams& p, int grid, size_t smem,
+                                    cudaStream_t stream) {
+  if (p.M == 1) return launch_decode<MODE, 1, 1>(p, grid, smem, stream);
+  if (p.M == 2) return launch_decode<MODE, 2, 2>(p, grid, smem, stream);
+  if (p.M <= 4) return launch_decode<MODE, 4, 4>(p, grid, smem, stream);
+  return launch_decode<MODE, 4, 8>(p, grid, smem, stream);
+}
+
+// Host-side planning of a launch: rows per stage (stages of at most 56 KB,
+// as few as cover the CTA's rows, equally sized), the work-block height, the
+// ring depth (as many stages as the 227 KB of shared memory hold, 2..8) and
+// the K-slicing.
+static bitnet_status plan_decode(DecodeParams& p, int num_sms, int* grid_out, size_t* smem_out) {
+  DecodeOp& o = p.op;
   const int M = p.M;
   const int MT = M == 1 ? 1 : (M == 2 ? 2 : 4);
   const int Mpad = ((M + MT - 1) / MT) * MT;
-  int grid = num_sms;
-  if (p.nops == 1) {
-    const int blocks = (p.op[0].N + 3) / 4;
-    grid = blocks < num_sms ? blocks : num_sms;
-  }
-  size_t stage = 16, xbytes = 128, accw = 1;
-  int total_chunks = 0;
-  for (int i = 0; i < p.nops; ++i) {
-    DecodeOp& o = p.op[i];
-    const int nmat = o.mode == kGlu ? 2 : 1;
-    const size_t row_bytes = (size_t)(o.K / 4) * nmat;
-    // 8-row blocks: single-op programs and the FFN's down step only
-    const int rb = (p.nops > 1 && o.mode == kLinear) ? 4 : gemv_rows_per_block(M, o.K, nmat);
-    const int rows_per_cta = (o.N + grid - 1) / grid;
-    int rs_max = (int)((56 * 1024) / row_bytes) / rb * rb;
-    if (rs_max < rb) rs_max = rb;
-    const int nch = (rows_per_cta + rs_max - 1) / rs_max;
-    int rs = (rows_per_cta + nch - 1) / nch;
-    rs = (rs + rb - 1) / rb * rb;
-    o.rb = rb;
-    o.rows_per_stage = rs;
-    o.wk = pick_wk(rs / rb, o.K / 16);
-    if ((size_t)rs * row_bytes > stage) stage = (size_t)rs * row_bytes;
-    const size_t xb = (((size_t)Mpad * o.K + 127) / 128) * 128;
-    if (xb > xbytes) xbytes = xb;
-    if ((size_t)nmat * rs * kMaxTok > accw) accw = (size_t)nmat * rs * kMaxTok;
-    total_chunks += nch;
-  }
-  const size_t budget = 200 * 1024;
-  const size_t acc_bytes = ((2 * accw * 4 + 127) / 128) * 128;
-  const size_t head = 4096 + xbytes + acc_bytes;
-  int st = budget > head + 2 * stage ? (int)((budget - head) / stage) : 2;
+  const int blocks = (o.N + 3) / 4;
+  const int grid = blocks < num_sms ? blocks : num_sms;
+  const int nmat = o.mode == kGlu ? 2 : 1;
+  const size_t row_bytes = (size_t)(o.K / 4) * nmat;
+  const int rb = gemv_rows_per_block(M, o.K, nmat);
+  const int rows_per_cta = (o.N + grid - 1) / grid;
+  int rs_max = (int)((56 * 1024) / row_bytes) / rb * rb;
+  if (rs_max < rb) rs_max = rb;
+  const int nch = (rows_per_cta + rs_max - 1) / rs_max;
+  int rs = (rows_per_cta + nch - 1) / nch;
+  rs = (rs + rb - 1) / rb * rb;
+  const size_t stage = (size_t)rs * row_bytes;
+  const size_t xbytes = (((size_t)Mpad * o.K + 127) / 128) * 128;
+  const size_t accw = (size_t)nmat * rs * kMaxTok;
+  const size_t cntw = (size_t)(rs / rb);
+  // per ring stage: the stage itself, its accumulators and block counters
+  const size_t budget = 227 * 1024;
+  const size_t head = 4096 + xbytes + 256;
+  const size_t per_stage = stage + 4 * (accw + cntw);
+  int st = budget > head + 2 * per_stage ? (int)((budget - head) / per_stage) : 2;
   if (st > 8) st = 8;
-  if (st > total_chunks) st = total_chunks;
+  if (st > nch) st = nch;
   if (st < 2) st = 2;
+  o.rb = rb;
+  o.rows_per_stage = rs;
+  o.wk = pick_wk(rows_per_cta, rs, rb, o.K / 16, st, nch);
   p.stages = st;
   p.stage_bytes = (uint32_t)stage;
   p.xbytes = (uint32_t)xbytes;
   p.acc_words = (uint32_t)accw;
+  p.cnt_words = (uint32_t)cntw;
   *grid_out = grid;
-  *smem_out = head + (size_t)st * stage;
+  const size_t acc_bytes = ((st * accw + 31) / 32) * 128;
+  const size_t cnt_bytes = ((st * cntw + 31) / 32) * 128;
+  *smem_out = 4096 + xbytes + acc_bytes + cnt_bytes + (size_t)st * stage;
   return *smem_out > 227 * 1024 ? BITNET_ERR_UNSUPPORTED : BITNET_OK;
-}
-
-template <int CAP, int MODES>
-static bitnet_status run_program(const DecodeOp* ops, int nops, int M, unsigned int* bar,
-                                 int num_sms, cudaStream_t stream) {
-  DecodeProgram<CAP> p{};
-  p.nops = nops;
-  p.M = M;
-  p.bar = bar;
-  for (int i = 0; i < nops; ++i) p.op[i] = ops[i];
-  int grid = 0;
-  size_t smem = 0;
-  const bitnet_status st = plan_program(p, num_sms, &grid, &smem);
-  if (st != BITNET_OK) return st;
-  if (nops > 1 && cudaMemsetAsync(bar, 0, sizeof(unsigned int), stream) != cudaSuccess)
-    return BITNET_ERR_CUDA;
-  return launch_by_tokens<CAP, MODES>(p, grid, smem, stream) == cudaSuccess ? BITNET_OK
-                                                                            : BITNET_ERR_CUDA;
 }
 
 }  // namespace bitnet
 
 using namespace bitnet;
 
-// Runs ops[0..nops) as one decode program.  Supported programs: one Linear
-// op; gate/up (Glu) followed by down (Down); up to kMaxProgramOps Linear ops.
-// `bar` (one zeroed word per launch, set here) is needed when nops > 1.
-bitnet_status bitnet_decode_launch(const DecodeOp* ops, int nops, int M, unsigned int* bar,
-                                   int num_sms, cudaStream_t stream) {
-  if (nops < 1 || nops > kMaxProgramOps || M < 1 || M > kMaxTok) return BITNET_ERR_UNSUPPORTED;
-  if (nops > 1 && !bar) return BITNET_ERR_INVALID_ARG;
-  bool all_linear = true;
-  for (int i = 0; i < nops; ++i) all_linear = all_linear && ops[i].mode == kLinear;
-  if (nops == 1 && all_linear)
-    return run_program<1, kModeLinear>(ops, nops, M, bar, num_sms, stream);
-  if (nops == 2 && ops[0].mode == kGlu && ops[1].mode == kDown)
-    return run_program<2, kModeGlu | kModeDown>(ops, nops, M, bar, num_sms, stream);
-  if (all_linear)
-    return run_program<kMaxProgramOps, kModeLinear>(ops, nops, M, bar, num_sms, stream);
-  return BITNET_ERR_UNSUPPORTED;
+// One decode launch: a BitLinear (mode kLinear), or the FFN's gate/up (kGlu)
+// or down (kDown) step.  M <= 8.
+bitnet_status bitnet_decode_launch(const DecodeOp& op, int M, int num_sms, cudaStream_t stream) {
+  if (M < 1 || M > kMaxTok) return BITNET_ERR_UNSUPPORTED;
+  DecodeParams p{};
+  p.op = op;
+  p.M = M;
+  int grid = 0;
+  size_t smem = 0;
+  const bitnet_status st = plan_decode(p, num_sms, &grid, &smem);
+  if (st != BITNET_OK) return st;
+  cudaError_t e = cudaErrorInvalidValue;
+  if (op.mode == kLinear) e = launch_by_tokens<kLinear>(p, grid, smem, stream);
+  else if (op.mode == kGlu) e = launch_by_tokens<kGlu>(p, grid, smem, stream);
+  else if (op.mode == kDown) e = launch_by_tokens<kDown>(p, grid, smem, stream);
+  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }

@@ -49,7 +49,7 @@ def test_workspace_sizes_are_host_only(L):
     assert L.bitnet_linear_workspace_size(4096, 6912, 2560) >= 4096 * 2560
     assert L.bitnet_linear_workspace_size(64, 2560, 6912) >= 64 * 6912 + 64 * 2560 * 4
     assert L.bitnet_linear_workspace_size(8, 400, 68) >= 8 * 68        # ragged K
-    assert L.bitnet_ffn_workspace_size(1, 8192, 28672) == 256 + 28672 * 4   # barrier + h'
+    assert L.bitnet_ffn_workspace_size(1, 8192, 28672) == 28672 * 4     # h' between the launches
     assert L.bitnet_ffn_workspace_size(2048, 8192, 28672) > 2048 * 28672 * 4
 
 
@@ -114,14 +114,15 @@ def _chain_args(Ns, Ks, ys, x=FAKE):
 
 def test_chain_workspace_and_validation(L):
     I64 = ctypes.c_int64 * 2
-    # decode-range chains need only the barrier word
-    assert L.bitnet_linear_chain_workspace_size(2, I64(6912, 2560), I64(2560, 6912), 1) == 256
+    # decode-range layers need no scratch; others reuse the largest layer's
+    assert L.bitnet_linear_chain_workspace_size(2, I64(6912, 2560), I64(2560, 6912), 1) == 0
     big = L.bitnet_linear_chain_workspace_size(2, I64(6912, 2560), I64(2560, 6912), 4096)
-    assert big == 256 + L.bitnet_linear_workspace_size(4096, 2560, 6912)
+    assert big == max(L.bitnet_linear_workspace_size(4096, 6912, 2560),
+                      L.bitnet_linear_workspace_size(4096, 2560, 6912))
     assert L.bitnet_linear_chain_workspace_size(0, I64(1, 1), I64(4, 4), 1) == 0
     y0, y1 = 0x100000, 0x200000
     n, P, G, N, K, x, Y = _chain_args([6912, 2560], [2560, 6912], [y0, y1])
-    ws, nb = FAKE, 256
+    ws, nb = None, 0
 
     def call(**kw):
         a = dict(n=n, P=P, G=G, N=N, K=K, x=x, M=1, Y=Y, ws=ws, nb=nb)
@@ -145,10 +146,10 @@ def test_chain_workspace_and_validation(L):
     _, _, _, _, _, _, Yal2 = _chain_args([6912, 2560], [2560, 6912], [y0, y0 + 16])
     assert call(Y=Yal2) == 1
     # ping-pong (y[2] == y[0]) is allowed by the aliasing rule; here it fails
-    # only on the missing workspace
+    # only on the missing workspace that M = 64 needs
     n3, P3, G3, N3, K3, x3, Y3 = _chain_args([6912, 2560, 6912], [2560, 6912, 2560],
                                              [y0, y1, y0])
-    assert L.bitnet_linear_chain(n3, P3, G3, N3, K3, x3, 1, Y3, None, 0, None) == 4
-    assert call(ws=None) == 4
-    assert call(nb=255) == 4
-    assert call(ws=MIS) == 3
+    assert L.bitnet_linear_chain(n3, P3, G3, N3, K3, x3, 64, Y3, None, 0, None) == 4
+    need = L.bitnet_linear_chain_workspace_size(2, I64(6912, 2560), I64(2560, 6912), 64)
+    assert call(M=64, ws=FAKE, nb=need - 1) == 4
+    assert call(M=64, ws=MIS, nb=need) == 3
