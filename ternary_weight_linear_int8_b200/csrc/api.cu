@@ -105,6 +105,14 @@ int plan_ksplit(int64_t M, int64_t N, int64_t K, int bn, int num_sms) {
   return ks < 1 ? 1 : (int)ks;
 }
 
+// Split-K scratch of the tensor-core path: the integer accumulators [M,N]
+// followed by one counter per (128-feature, token) tile (tiles are at least
+// 32 tokens wide); both are cleared before each launch.
+size_t splitk_acc_bytes(int64_t M, int64_t N) { return al256((size_t)M * N * 4); }
+size_t splitk_cnt_bytes(int64_t M, int64_t N) {
+  return al256((size_t)((N + 127) / 128) * (size_t)((M + 31) / 32) * 4);
+}
+
 struct LinearWs {
   size_t xq, scale, rowsum, acc, total;
 };
@@ -119,7 +127,7 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
   w.acc = w.rowsum + al256((size_t)M * 4);
   w.total = w.acc;
   // split-K accumulators are reserved for every small-M tensor-core shape
-  if (p == kPathGemm && M <= 256) w.total = w.acc + al256((size_t)M * N * 4);
+  if (p == kPathGemm && M <= 256) w.total = w.acc + splitk_acc_bytes(M, N) + splitk_cnt_bytes(M, N);
   return w;
 }
 
@@ -144,7 +152,8 @@ FfnWs ffn_ws_layout(int64_t M, int64_t H, int64_t I) {
     w.rs2 = off; off += al256((size_t)M * 4);
     w.ss2 = off; off += al256((size_t)M * 8);
     if (M <= 256) {   // split-K accumulators: gate (and later down), up
-      w.acc0 = off; off += al256((size_t)M * (H > I ? H : I) * 4);
+      const int64_t HI = H > I ? H : I;
+      w.acc0 = off; off += splitk_acc_bytes(M, HI) + splitk_cnt_bytes(M, HI);
       w.acc1 = off; off += al256((size_t)M * I * 4);
     }
   }
@@ -267,7 +276,10 @@ bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N
   a.y = y; a.y_f32 = y_f32; a.acc0 = acc;
   if (a.ksplit > 1) {
     a.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc);
-    if (cudaMemsetAsync(a.acc_ws0, 0, (size_t)M * N * 4, s) != cudaSuccess) return BITNET_ERR_CUDA;
+    a.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc + splitk_acc_bytes(M, N));
+    if (cudaMemsetAsync(a.acc_ws0, 0, splitk_acc_bytes(M, N) + splitk_cnt_bytes(M, N), s) !=
+        cudaSuccess)
+      return BITNET_ERR_CUDA;
   }
   return bitnet_gemm_launch(0 /*linear*/, xq, packed, nullptr, a, bn, d.num_sms, s);
 }
@@ -343,7 +355,9 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
   if (g.ksplit > 1) {
     g.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
     g.acc_ws1 = reinterpret_cast<int32_t*>(ws + L.acc1);
-    if (cudaMemsetAsync(g.acc_ws0, 0, (size_t)M * I * 4, s) != cudaSuccess ||
+    g.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc0 + splitk_acc_bytes(M, I));
+    if (cudaMemsetAsync(g.acc_ws0, 0, splitk_acc_bytes(M, I) + splitk_cnt_bytes(M, I), s) !=
+            cudaSuccess ||
         cudaMemsetAsync(g.acc_ws1, 0, (size_t)M * I * 4, s) != cudaSuccess)
       return BITNET_ERR_CUDA;
   }
@@ -360,7 +374,10 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
   dn.y = y; dn.y_f32 = dbg.y_f32; dn.acc0 = dbg.acc_down;
   if (dn.ksplit > 1) {
     dn.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
-    if (cudaMemsetAsync(dn.acc_ws0, 0, (size_t)M * H * 4, s) != cudaSuccess) return BITNET_ERR_CUDA;
+    dn.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc0 + splitk_acc_bytes(M, H));
+    if (cudaMemsetAsync(dn.acc_ws0, 0, splitk_acc_bytes(M, H) + splitk_cnt_bytes(M, H), s) !=
+        cudaSuccess)
+      return BITNET_ERR_CUDA;
   }
   return bitnet_gemm_launch(2 /*down*/, xq2, down, nullptr, dn, bn_d, d.num_sms, s);
 }

@@ -48,6 +48,8 @@ struct GemmArgs {
   float* h;                 // Glu [M,N]
   int32_t* acc_ws0;         // split-K accumulators [M,N]
   int32_t* acc_ws1;
+  int32_t* tile_cnt;        // split-K, narrow tiles: K-slices done per tile (the last
+                            // CTA finishes the tile); null: a finaliser kernel does
   int tma_store;            // 1: bf16 y written through the staged TMA store
 };
 
@@ -134,6 +136,62 @@ __device__ __forceinline__ void epi_sync() {
 // with stride gridDim.x.  The stage ring and its barrier phases run on across
 // units; TMEM holds NACC accumulator sets so the epilogue warps drain unit i
 // while the MMA warp already accumulates unit i + 1.
+// Split-K: the CTA that adds a tile's last K-slice finishes the whole tile
+// (features [n0, n0+128) x tokens [t0, t0+bn)) with `nt` threads (`et` =
+// 0..nt-1, which meet at epi_sync): the per-token scalars first (IEEE
+// division and the RMS factors, once per token), then every output from the
+// integer accumulators (added by every K-slice with atomics, read from L2).
+template <int MODE>
+__device__ __forceinline__ void splitk_finish_tile(const GemmArgs& a, int n0, int t0, int bn,
+                                                   int et, int nt, float* tok_d0, int* tok_rs,
+                                                   float* tok_x1) {
+  for (int c = et; c < bn; c += nt) {
+    const int tok = t0 + c;
+    float d0 = 0.f, x1 = 0.f;
+    int rs = 0;
+    if (tok < a.M) {
+      const float s = a.scale[tok];
+      d0 = __fdiv_rn(*a.gamma0, s);
+      if (MODE == gGlu) x1 = __fdiv_rn(*a.gamma1, s);
+      rs = a.rowsum[tok];
+      if (MODE == gDown) {
+        const double eps = (double)a.eps;
+        const double r1 = 1.0 / sqrt(a.sumsq_x[tok] / (double)a.H + eps);
+        const double r1_3 = r1 * r1 * r1;
+        const double r2 = 1.0 / sqrt(r1_3 * r1_3 * (a.sumsq_h[tok] / (double)a.K) + eps);
+        x1 = (float)(r1_3 * r2);
+      }
+    }
+    tok_d0[c] = d0;
+    tok_rs[c] = rs;
+    tok_x1[c] = x1;
+  }
+  epi_sync();
+  for (int idx = et; idx < bn * kBM; idx += nt) {
+    const int c = idx / kBM;
+    const int tok = t0 + c, n = n0 + idx % kBM;
+    if (tok >= a.M || n >= a.N) continue;
+    const int64_t o = (int64_t)tok * a.N + n;
+    const int ac = __ldcg(a.acc_ws0 + o) - tok_rs[c];
+    if (MODE == gGlu) {
+      const int au = __ldcg(a.acc_ws1 + o) - tok_rs[c];
+      const float g = __fmul_rn(__int2float_rn(ac), tok_d0[c]);
+      const float uu = __fmul_rn(__int2float_rn(au), tok_x1[c]);
+      const float rg = fmaxf(g, 0.0f);
+      a.h[o] = __fmul_rn(__fmul_rn(rg, rg), uu);
+      if (a.acc0) a.acc0[o] = ac;
+      if (a.acc1) a.acc1[o] = au;
+    } else {
+      float y32 = __fmul_rn(__int2float_rn(ac), tok_d0[c]);
+      if (MODE == gDown) y32 = __fmul_rn(y32, tok_x1[c]);
+      a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+      if (a.y_f32) a.y_f32[o] = y32;
+      if (a.acc0) a.acc0[o] = ac;
+    }
+  }
+  epi_sync();   // the scalars are free again
+}
+
 template <int MODE, int BN, int NMAT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw0,
@@ -153,6 +211,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_full = mma_done + S;         // [NACC]
   uint64_t* acc_empty = acc_full + NACC;     // [NACC]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + NACC);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(aux + C::kAux - 16);
   float* tok_d0 = reinterpret_cast<float*>(aux + C::kAux);
   int* tok_rs = reinterpret_cast<int*>(tok_d0 + BN);
   float* tok_x1 = reinterpret_cast<float*>(tok_rs + BN);   // Glu: gamma_up / s; Down: r1^3 r2
@@ -441,6 +500,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (a.ksplit > 1 && a.tile_cnt) {
+        // the CTA that adds a tile's last K-slice finishes the tile (a
+        // counter per tile, cleared with the accumulators before the launch)
+        epi_sync();                          // every partial of this unit is added
+        if (et == 0) {
+          __threadfence();
+          *last_flag = atomicAdd(&a.tile_cnt[mt * n_tiles + nt], 1) == a.ksplit - 1;
+        }
+        epi_sync();
+        if (*last_flag) {
+          __threadfence();
+          splitk_finish_tile<MODE>(a, nt * kBM, mt * BN, BN, et, 256, tok_d0, tok_rs, tok_x1);
+        }
+      }
     }
   }
   if (warp >= 6 && lane == 0) bulk_wait0();  // this warp's TMA stores have landed
@@ -590,7 +663,10 @@ int bitnet_gemm_pick_bn(int M, int N, int num_sms) {
   return best;
 }
 
-// Launch the tensor-core kernel (and, with ksplit > 1, its finaliser).
+// Launch the tensor-core kernel.  With ksplit > 1 the caller has cleared
+// acc_ws0 (and acc_ws1) and, for 32-token tiles, tile_cnt: the last CTA of a
+// tile finishes it in the kernel; wider tiles (more outputs than one CTA
+// should finish at the end) go through the finaliser kernel.
 // xq: [M, K] int8 in the permuted K order; w0/w1: packed [N, K/4].
 bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
                                  const uint8_t* w1, GemmArgs a, int bn, int num_sms,
@@ -619,6 +695,7 @@ bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
                     (uint64_t)a.N * 2, 32, 8, false))
       a.tma_store = 1;
   }
+  if (bn > 32) a.tile_cnt = nullptr;
   const int64_t units = (int64_t)((a.N + kBM - 1) / kBM) * ((a.M + bn - 1) / bn) * a.ksplit;
   dim3 grid((unsigned)(units < num_sms ? units : num_sms));
   cudaError_t e = cudaErrorInvalidValue;
@@ -635,7 +712,7 @@ bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
   else { BITNET_GEMM_BN(gDown, 1) }
 #undef BITNET_GEMM_BN
   if (e != cudaSuccess) return BITNET_ERR_CUDA;
-  if (a.ksplit > 1) {
+  if (a.ksplit > 1 && !a.tile_cnt) {
     cudaLaunchConfig_t cfg = {};
     const int64_t total = (int64_t)a.M * a.N;
     int64_t blocks = (total + 255) / 256;

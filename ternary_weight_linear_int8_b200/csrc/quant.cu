@@ -166,6 +166,103 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
   pdl_launch_dependents();
 }
 
+// Few tokens: one 256-thread CTA per token (a warp per token would leave
+// almost the whole GPU idle), block reductions through shared memory.  Same
+// arithmetic as quant_rows_kernel: absmax and the integer row sum do not
+// depend on order; the fp64 sum of squares (the FFN's RMS factor) may differ
+// in rounding order only.
+template <bool kF32, bool kPerm>
+__global__ void __launch_bounds__(256) quant_token_kernel(QuantArgs a) {
+  __shared__ float s_max[8];
+  __shared__ double s_ss[8];
+  __shared__ int s_rs[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t m = blockIdx.x;
+  const int64_t K = a.K;
+  const int64_t base = m * K;
+  pdl_wait();
+  // pass 1: absmax of src * gain, sum of squares of src; groups of 4
+  float amax = 0.f;
+  double ss = 0.0;
+  for (int64_t k = (int64_t)threadIdx.x * 4; k < K; k += 1024) {
+    float v[4];
+    load4<kF32>(a.src, base + k, v);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (a.sumsq) ss += (double)v[c] * (double)v[c];
+      const float g = a.gain ? __fmul_rn(v[c], a.gain[k + c]) : v[c];
+      amax = fmaxf(amax, fabsf(g));
+    }
+  }
+  amax = warp_max(amax);
+  if (a.sumsq) ss = warp_sum_d(ss);
+  if (lane == 0) {
+    s_max[warp] = amax;
+    s_ss[warp] = ss;
+  }
+  __syncthreads();
+  float am = s_max[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) am = fmaxf(am, s_max[w]);
+  const float s = qscale(am);
+  // pass 2: quantise (groups of 16 for the permuted layout, else 4)
+  int rs = 0;
+  if (kPerm) {
+    for (int64_t k = (int64_t)threadIdx.x * 16; k < K; k += 4096) {
+      float v0[8], v1[8];
+      load8<kF32>(a.src, base + k, v0);
+      load8<kF32>(a.src, base + k + 8, v1);
+      int q[16];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float g0 = a.gain ? __fmul_rn(v0[c], a.gain[k + c]) : v0[c];
+        const float g1 = a.gain ? __fmul_rn(v1[c], a.gain[k + 8 + c]) : v1[c];
+        q[c] = quant_code(g0, s);
+        q[8 + c] = quant_code(g1, s);
+      }
+#pragma unroll
+      for (int c = 0; c < 16; ++c) rs += q[c];
+      // slot 4*t + b holds natural index 4*b + t
+      *reinterpret_cast<uint4*>(a.xq + m * a.ld_q + k) =
+          make_uint4(pack4(q[0], q[4], q[8], q[12]), pack4(q[1], q[5], q[9], q[13]),
+                     pack4(q[2], q[6], q[10], q[14]), pack4(q[3], q[7], q[11], q[15]));
+      if (a.xq_natural)
+        *reinterpret_cast<uint4*>(a.xq_natural + m * K + k) =
+            make_uint4(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]),
+                       pack4(q[8], q[9], q[10], q[11]), pack4(q[12], q[13], q[14], q[15]));
+    }
+  } else {
+    for (int64_t k = (int64_t)threadIdx.x * 4; k < K; k += 1024) {
+      float v[4];
+      load4<kF32>(a.src, base + k, v);
+      int q[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float g = a.gain ? __fmul_rn(v[c], a.gain[k + c]) : v[c];
+        q[c] = quant_code(g, s);
+        rs += q[c];
+      }
+      *reinterpret_cast<uint32_t*>(a.xq + m * a.ld_q + k) = pack4(q[0], q[1], q[2], q[3]);
+    }
+  }
+  rs = warp_sum_i(rs);
+  if (lane == 0) s_rs[warp] = rs;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    double d = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      t += s_rs[w];
+      d += s_ss[w];
+    }
+    a.scale[m] = s;
+    if (a.rowsum) a.rowsum[m] = t;
+    if (a.sumsq) a.sumsq[m] = d;
+  }
+  pdl_launch_dependents();
+}
+
 }  // namespace bitnet
 
 using namespace bitnet;
@@ -177,7 +274,9 @@ bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* ga
                                   cudaStream_t stream) {
   QuantArgs a{src, gain, M, K, xq, ld_q, scale, rowsum, sumsq, xq_natural};
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((M + 7) / 8));
+  // up to 256 tokens: a CTA per token; more: a warp per token
+  const bool per_token = M <= 256;
+  cfg.gridDim = dim3((unsigned)(per_token ? M : (M + 7) / 8));
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -187,7 +286,15 @@ bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* ga
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (src_f32) {
+  if (per_token) {
+    if (src_f32) {
+      e = perm ? cudaLaunchKernelEx(&cfg, quant_token_kernel<true, true>, a)
+               : cudaLaunchKernelEx(&cfg, quant_token_kernel<true, false>, a);
+    } else {
+      e = perm ? cudaLaunchKernelEx(&cfg, quant_token_kernel<false, true>, a)
+               : cudaLaunchKernelEx(&cfg, quant_token_kernel<false, false>, a);
+    }
+  } else if (src_f32) {
     e = perm ? cudaLaunchKernelEx(&cfg, quant_rows_kernel<true, true>, a)
              : cudaLaunchKernelEx(&cfg, quant_rows_kernel<true, false>, a);
   } else {
