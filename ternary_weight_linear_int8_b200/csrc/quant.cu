@@ -166,8 +166,9 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
   pdl_launch_dependents();
 }
 
-// Few tokens: one 256-thread CTA per token (a warp per token would leave
-// almost the whole GPU idle), block reductions through shared memory.  Same
+// One 256-thread CTA per token, block reductions through shared memory: for
+// few tokens (a warp per token would leave almost the whole GPU idle) and
+// for long rows (a warp per token is a long chain of dependent loads).  Same
 // arithmetic as quant_rows_kernel: absmax and the integer row sum do not
 // depend on order; the fp64 sum of squares (the FFN's RMS factor) may differ
 // in rounding order only.
@@ -181,10 +182,23 @@ __global__ void __launch_bounds__(256) quant_token_kernel(QuantArgs a) {
   const int64_t K = a.K;
   const int64_t base = m * K;
   pdl_wait();
-  // pass 1: absmax of src * gain, sum of squares of src; groups of 4
+  // pass 1: absmax of src * gain, sum of squares of src; groups of 8
+  // (16-byte bf16 loads) when rows start 16-byte aligned, else of 4
   float amax = 0.f;
   double ss = 0.0;
-  for (int64_t k = (int64_t)threadIdx.x * 4; k < K; k += 1024) {
+  const int64_t K8 = (K & 7) == 0 ? K : 0;
+#pragma unroll 2
+  for (int64_t k = (int64_t)threadIdx.x * 8; k < K8; k += 2048) {
+    float v[8];
+    load8<kF32>(a.src, base + k, v);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (a.sumsq) ss += (double)v[c] * (double)v[c];
+      const float g = a.gain ? __fmul_rn(v[c], a.gain[k + c]) : v[c];
+      amax = fmaxf(amax, fabsf(g));
+    }
+  }
+  for (int64_t k = K8 + (int64_t)threadIdx.x * 4; k < K; k += 1024) {
     float v[4];
     load4<kF32>(a.src, base + k, v);
 #pragma unroll
@@ -274,8 +288,9 @@ bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* ga
                                   cudaStream_t stream) {
   QuantArgs a{src, gain, M, K, xq, ld_q, scale, rowsum, sumsq, xq_natural};
   cudaLaunchConfig_t cfg = {};
-  // up to 256 tokens: a CTA per token; more: a warp per token
-  const bool per_token = M <= 256;
+  // a CTA per token for up to 256 tokens or rows longer than 4096 values;
+  // else a warp per token (measured faster for many short rows)
+  const bool per_token = M <= 256 || K > 4096;
   cfg.gridDim = dim3((unsigned)(per_token ? M : (M + 7) / 8));
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;

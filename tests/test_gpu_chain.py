@@ -1,6 +1,7 @@
-"""GPU parity of bitnet_linear_chain: a chain of BitLinear layers run as one
-decode program (one cooperative launch with a grid barrier between layers)
-must give, layer for layer, exactly the oracle's bf16 outputs."""
+"""GPU parity of bitnet_linear_chain: a chain of BitLinear layers, each fed
+the previous one's output (one launch per layer, programmatic dependent
+launch between them), must give, layer for layer, exactly the oracle's bf16
+outputs."""
 from __future__ import annotations
 
 import numpy as np
@@ -44,7 +45,7 @@ def _run_chain(Ws, x, ys=None):
 
 @pytest.mark.parametrize("M", [1, 2, 3, 8])
 def test_chain_small_layers_match_oracle(M):
-    """Nine decode-range layers of mixed widths (one program)."""
+    """Nine decode-range layers of mixed widths."""
     dims = [512, 1024, 256, 768, 64, 320, 2048, 128, 640, 512]
     x, Ws = _chain_case(dims, M, seed=11 + M)
     ys = _run_chain(Ws, x)
@@ -52,8 +53,8 @@ def test_chain_small_layers_match_oracle(M):
         assert np.array_equal(host_bits(ys[l]), want), f"layer {l}"
 
 
-def test_chain_longer_than_one_program():
-    """70 layers: two programs of 64 and 6 layers back to back."""
+def test_chain_of_70_layers():
+    """70 layers of mixed widths back to back."""
     rng = np.random.default_rng(3)
     dims = [256] + [int(v) for v in rng.choice([128, 192, 256, 384], size=70)]
     x, Ws = _chain_case(dims, 1, seed=5)
@@ -64,7 +65,7 @@ def test_chain_longer_than_one_program():
 
 
 def test_chain_with_layers_outside_the_decode_range():
-    """K % 64 != 0 (400) runs as its own bitnet_linear call between programs."""
+    """K % 64 != 0 (400) takes the scalar path between decode-kernel layers."""
     dims = [512, 400, 256, 320, 128, 400, 64]
     x, Ws = _chain_case(dims, 4, seed=21)
     ys = _run_chain(Ws, x)
