@@ -72,6 +72,19 @@ __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
+// Warp-level integer MMA, D = A(16x32, u8, row) * B(32x8, s8, col) + C.
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t u4_at(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
 // Halving step of the butterfly: n values -> n/2, exchanging with lane ^ off.
 template <int N>
 __device__ __forceinline__ void halve(const int (&v)[N], int (&o)[N / 2], int off, int lane) {
@@ -208,7 +221,9 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
   constexpr int NMAT = (MODE == kGlu) ? 2 : 1;
   // RB: rows per work block (per matrix); NR values per lane per block
   constexpr int NR = RB * NMAT;
-  static_assert(NR == 4 || NR == 8, "4 or 8 values per block");
+  // RB 16: tensor-core items (16-row tiles, all tokens in one MMA column set)
+  constexpr bool kMma = RB == 16;
+  static_assert(kMma || NR == 4 || NR == 8, "4 or 8 values per block");
   constexpr bool kF32Src = (MODE == kDown);
   constexpr int NT = kConsumerWarps * 32;
   float* tok_d0 = sm.tok_d0();
@@ -471,6 +486,111 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
       const uint32_t st_addr = smem_u32(sm.ring() + (size_t)s * sm.stage_bytes);
       int* acc = sm.acc_s() + s * acc_words;
       int* cnt = sm.cnt_s() + s * cnt_words;
+      if constexpr (kMma) {
+      // Tensor-core items: a 16-row tile (per matrix) x a K-slice of 16-word
+      // windows.  MMA row = tile row, MMA k = activation position, MMA
+      // column = token.  Lane (g = lane/4, q = lane%4) loads words 4q..4q+3
+      // of rows g and g+8 of each window (16 bytes each) and the four
+      // 16-activation groups of those words for token g.  Word 4q+2p gives
+      // k = 4q..4q+3 and word 4q+2p+1 gives k = 16+4q..16+4q+3 of the MMA
+      // for pair p and code plane t (masked in place, so its codes are
+      // scaled by 4^t; one accumulator set per plane, shifted back at the
+      // end, exactly).
+      const int g = lane >> 2, qd = lane & 3;
+      const int nwin = (Kw + 15) >> 4;
+      const uint32_t xa = x_addr + (uint32_t)(g * K + 64 * qd);
+      const bool tok_ok = g < M;
+      for (int it = first; it < nitems; it += kConsumerWarps) {
+        const int b = it >> wk_log2, q = it & (WK - 1);
+        const int w0 = (q * nwin) / WK, w1 = ((q + 1) * nwin) / WK;
+        uint32_t rowa[NMAT][2];
+#pragma unroll
+        for (int mat = 0; mat < NMAT; ++mat)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            rowa[mat][h] = st_addr + (uint32_t)((mat * RS + 16 * b + g + 8 * h) * Kb + 16 * qd);
+        int C[NMAT][4][4];
+#pragma unroll
+        for (int mat = 0; mat < NMAT; ++mat)
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) C[mat][t][e] = 0;
+        for (int w = w0; w < w1; ++w) {
+          // the row's last window may be partial: lanes past the end add 0
+          const bool valid = 16 * w + 4 * qd < Kw;
+          uint4 wr[NMAT][2];
+#pragma unroll
+          for (int mat = 0; mat < NMAT; ++mat)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              wr[mat][h] = valid ? lds_v4(rowa[mat][h] + 64u * w) : make_uint4(0, 0, 0, 0);
+          uint4 xg[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            xg[i] = (valid && tok_ok) ? lds_v4(xa + 256u * w + 16u * i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int pp = 0; pp < 2; ++pp) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const uint32_t mask = 0x03030303u << (2 * t);
+              const uint32_t b0 = u4_at(xg[2 * pp], t), b1 = u4_at(xg[2 * pp + 1], t);
+#pragma unroll
+              for (int mat = 0; mat < NMAT; ++mat)
+                mma_u8s8(C[mat][t], u4_at(wr[mat][0], 2 * pp) & mask,
+                         u4_at(wr[mat][1], 2 * pp) & mask, u4_at(wr[mat][0], 2 * pp + 1) & mask,
+                         u4_at(wr[mat][1], 2 * pp + 1) & mask, b0, b1);
+            }
+          }
+        }
+        // C element e: row g + 8*(e/2) of the tile, token 2q + e%2
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          int v[NMAT];
+#pragma unroll
+          for (int mat = 0; mat < NMAT; ++mat)
+            v[mat] = C[mat][0][e] + (C[mat][1][e] >> 2) + (C[mat][2][e] >> 4) + (C[mat][3][e] >> 6);
+          const int rr = 16 * b + g + 8 * (e >> 1), m = 2 * qd + (e & 1);
+          if (m < M && rr < nr) {
+            if (WK == 1) {
+              finish(r0, rr, m, v[0], v[NMAT - 1]);
+            } else {
+#pragma unroll
+              for (int mat = 0; mat < NMAT; ++mat)
+                atomicAdd(&acc[(mat * RS + rr) * kMaxTok + m], v[mat]);
+            }
+          }
+        }
+        if (WK > 1) {
+          // the warp that adds a block's last slice finishes the block
+          __syncwarp();
+          int last = 0;
+          if (lane == 0) {
+            __threadfence_block();
+            last = atomicAdd(&cnt[b], 1) == WK - 1;
+          }
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (last) {
+            __threadfence_block();
+            const int rows_b = min(RB, nr - RB * b);
+            for (int o = lane; o < rows_b * M; o += 32) {
+              const int rr = RB * b + o / M, m = o % M;
+              int* p0 = &acc[rr * kMaxTok + m];
+              const int v0 = *p0;
+              *p0 = 0;
+              int v1 = 0;
+              if (NMAT == 2) {
+                int* p1 = &acc[(RS + rr) * kMaxTok + m];
+                v1 = *p1;
+                *p1 = 0;
+              }
+              finish(r0, rr, m, v0, v1);
+            }
+            if (lane == 0) cnt[b] = 0;
+          }
+        }
+      }
+      } else {
       for (int it = first; it < nitems; it += kConsumerWarps) {
         const int b = it >> wk_log2, q = it & (WK - 1);
         const int j0 = (q * Kw) / WK, j1 = ((q + 1) * Kw) / WK;
@@ -601,6 +721,7 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
           }
         }
       }
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty()[s]);
@@ -629,9 +750,13 @@ static int pick_wk(int rows_cta, int rs, int rb, int Kw, int stages, int nch) {
   return best;
 }
 
-// Rows per work block: 8 for a single matrix with long rows and one token
-// (the activation loads and the reduction are shared by more rows), else 4.
+// Rows per work block: 16 (tensor-core items) for 4 or more tokens where 16
+// rows of every matrix fit a 64 KB stage (measured: 7 % faster at M = 4 and
+// 8, slower at M = 1, where dp4a does one token's work only); else dp4a
+// items of 8 rows for a single matrix with long rows and one token (the
+// activation loads and the reduction are shared by more rows), or 4.
 static int gemv_rows_per_block(int M, int K, int nmat) {
+  if (M >= 4 && (size_t)16 * (K / 4) * nmat <= 64 * 1024) return 16;
   return (nmat == 1 && M == 1 && K >= 8192) ? 8 : 4;
 }
 
@@ -669,6 +794,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   bool ring_ok = true;
   pdl_wait();
+  // 16-row tiles: the tensor-core items (planned on the host)
+  if (p.op.rb == 16) {
+    run_op<MODE, MT, MM, 16>(p.op, p.M, sm, ring_ok);
+    return;
+  }
   // 8-row blocks: one long-row matrix with one token (planned on the host)
   if constexpr (MM == 1 && MODE != kGlu) {
     if (p.op.rb == 8) {
@@ -728,6 +858,7 @@ static bitnet_status plan_decode(DecodeParams& p, int num_sms, int* grid_out, si
   const size_t row_bytes = (size_t)(o.K / 4) * nmat;
   const int rb = gemv_rows_per_block(M, o.K, nmat);
   const int rows_per_cta = (o.N + grid - 1) / grid;
+  // stages of at most 56 KB (64 KB where one 16-row tile needs it)
   int rs_max = (int)((56 * 1024) / row_bytes) / rb * rb;
   if (rs_max < rb) rs_max = rb;
   const int nch = (rows_per_cta + rs_max - 1) / rs_max;
@@ -747,7 +878,10 @@ static bitnet_status plan_decode(DecodeParams& p, int num_sms, int* grid_out, si
   if (st < 2) st = 2;
   o.rb = rb;
   o.rows_per_stage = rs;
-  o.wk = pick_wk(rows_per_cta, rs, rb, o.K / 16, st, nch);
+  // an MMA item step is a 16-word window of 16 rows (about twice a dp4a
+  // item's 32-word step of 4 rows in time): planned as 2 steps of Kw/16
+  o.wk = rb == 16 ? pick_wk(rows_per_cta, rs, rb, o.K / 8, st, nch)
+                  : pick_wk(rows_per_cta, rs, rb, o.K / 16, st, nch);
   p.stages = st;
   p.stage_bytes = (uint32_t)stage;
   p.xbytes = (uint32_t)xbytes;
