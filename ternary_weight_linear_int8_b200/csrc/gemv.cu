@@ -794,10 +794,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   bool ring_ok = true;
   pdl_wait();
-  // 16-row tiles: the tensor-core items (planned on the host)
-  if (p.op.rb == 16) {
-    run_op<MODE, MT, MM, 16>(p.op, p.M, sm, ring_ok);
-    return;
+  // 16-row tiles: the tensor-core items (planned on the host for 4 or more
+  // tokens; not compiled into the 1- and 2-token kernels)
+  if constexpr (MM >= 4) {
+    if (p.op.rb == 16) {
+      run_op<MODE, MT, MM, 16>(p.op, p.M, sm, ring_ok);
+      return;
+    }
   }
   // 8-row blocks: one long-row matrix with one token (planned on the host)
   if constexpr (MM == 1 && MODE != kGlu) {
