@@ -441,8 +441,8 @@ def profile_case(case):
         p, g = B.bitnet_pack_weights(torch.from_numpy(inputs.weights(N, K, seed=2000)).to(dev))
         for _ in range(4):
             B.bitnet_linear(p, g, x)
-    elif case == "batched16":
-        M = 16
+    elif case in ("batched8", "batched16"):
+        M = int(case[len("batched"):])
         packs = build_decode_chain(B, inputs, torch, dev, n_layers=6)
         x = torch.from_numpy(inputs.activations((M, HIDDEN), seed=0, outliers=True).view(np.int16)).to(dev)
         bufs = [torch.empty((M, INTER), dtype=torch.bfloat16, device=dev),
@@ -607,7 +607,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--profile-case", choices=["prefill", "ffn2048", "gemv_big", "batched16"],
+    ap.add_argument("--profile-case", choices=["prefill", "ffn2048", "gemv_big", "batched8", "batched16"],
                     default=None,
                     help="run a few calls of one workload for an ncu capture, print nothing")
     args = ap.parse_args()

@@ -181,8 +181,8 @@ def test_linear_under_cuda_graph_replay():
 
 
 # ------------------------------------------------------------------- FFN
-FFN_SHAPES = [(1, 256, 512), (2, 512, 1024), (1, 2560, 6912), (9, 256, 512), (64, 512, 1024),
-              (130, 256, 768), (300, 128, 320)]
+FFN_SHAPES = [(1, 256, 512), (2, 512, 1024), (1, 2560, 6912), (5, 256, 512), (8, 512, 1024),
+              (9, 256, 512), (64, 512, 1024), (130, 256, 768), (300, 128, 320)]
 
 
 def _ffn_case(M, H, I, seed=0, gains=True):
