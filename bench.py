@@ -450,8 +450,8 @@ def profile_case(case):
         call = ChainCall(B, torch, packs, bufs, dev)
         for _ in range(3):
             call(x)
-    elif case == "prefill":
-        M, N, K = 4096, INTER, HIDDEN
+    elif case in ("prefill", "prefill_down"):
+        M, N, K = (4096, INTER, HIDDEN) if case == "prefill" else (4096, HIDDEN, INTER)
         x = torch.from_numpy(inputs.activations((M, K), seed=0).view(np.int16)).to(dev)
         W = torch.from_numpy(inputs.weights(N, K, seed=1000)).to(dev)
         p, g = B.bitnet_pack_weights(W)
@@ -607,7 +607,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--profile-case", choices=["prefill", "ffn2048", "gemv_big", "batched8", "batched16"],
+    ap.add_argument("--profile-case", choices=["prefill", "prefill_down", "ffn2048", "gemv_big", "batched8", "batched16"],
                     default=None,
                     help="run a few calls of one workload for an ncu capture, print nothing")
     args = ap.parse_args()
