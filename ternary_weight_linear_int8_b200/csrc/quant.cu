@@ -1,4 +1,5 @@
-// Per-token absmax int8 activation quantisation (one warp per token).
+// Per-token absmax int8 activation quantisation: one warp per token for many
+// short rows, one 256-thread CTA per token for few tokens or long rows.
 //
 // youngju.dev "BitNet論文分析：1-Bit LLMの時代", section "Absmean量子化関数",
 // BitLinear_b158.activation_quant: per-token absmax scale, round, clamp.
