@@ -135,13 +135,16 @@ def bitnet_pack_weights(W: torch.Tensor, packed=None, gamma=None, workspace=None
     return packed, gamma
 
 
-def bitnet_quant_act(x: torch.Tensor, with_rowsum: bool = True):
-    """x bf16 [M,K] -> (x_q int8 [M,K], scale fp32 [M], rowsum int32 [M] or None)."""
+def bitnet_quant_act(x: torch.Tensor, with_rowsum: bool = True, xq=None, scale=None,
+                     rowsum=None):
+    """x bf16 [M,K] -> (x_q int8 [M,K], scale fp32 [M], rowsum int32 [M] or None).
+    The outputs may be given as preallocated tensors."""
     _bits16(x, "x")
     M, K = x.shape
-    xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
-    s = torch.empty(M, dtype=torch.float32, device=x.device)
-    rs = torch.empty(M, dtype=torch.int32, device=x.device) if with_rowsum else None
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device) if xq is None else _dev(xq, "xq")
+    s = torch.empty(M, dtype=torch.float32, device=x.device) if scale is None else _dev(scale, "scale")
+    rs = rowsum if rowsum is not None else (
+        torch.empty(M, dtype=torch.int32, device=x.device) if with_rowsum else None)
     st = lib().bitnet_quant_act(_ptr(x), M, K, _ptr(xq), _ptr(s), _ptr(rs), _stream())
     _check("bitnet_quant_act", st)
     return xq, s, rs
@@ -152,8 +155,10 @@ def bitnet_linear_workspace_size(M: int, N: int, K: int) -> int:
 
 
 def bitnet_linear(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, y=None,
-                  want_f32: bool = False, want_acc: bool = False, workspace=None):
-    """y = BitLinear(x) on packed weights.  Returns (y bf16 [M,N], y_f32, acc)."""
+                  want_f32: bool = False, want_acc: bool = False, workspace=None,
+                  y_f32=None, acc=None):
+    """y = BitLinear(x) on packed weights.  Returns (y bf16 [M,N], y_f32, acc).
+    `y`, `y_f32` and `acc` may be given as preallocated [M,N] tensors."""
     _dev(packed, "packed")
     _dev(gamma, "gamma")
     _bits16(x, "x")
@@ -162,8 +167,15 @@ def bitnet_linear(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, y=
     if K != 4 * Kb:
         raise ValueError("x and packed disagree on K")
     y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
-    y32 = torch.empty((M, N), dtype=torch.float32, device=x.device) if want_f32 else None
-    acc = torch.empty((M, N), dtype=torch.int32, device=x.device) if want_acc else None
+    y32 = y_f32 if y_f32 is not None else (
+        torch.empty((M, N), dtype=torch.float32, device=x.device) if want_f32 else None)
+    acc = acc if acc is not None else (
+        torch.empty((M, N), dtype=torch.int32, device=x.device) if want_acc else None)
+    for t, name in ((y, "y"), (y32, "y_f32"), (acc, "acc")):
+        if t is not None:
+            _dev(t, name)
+            if tuple(t.shape) != (M, N):
+                raise ValueError(f"{name} must have shape [M, N]")
     nb = lib().bitnet_linear_workspace_size(M, N, K)
     ws = _workspace(nb, x.device, workspace)
     st = lib().bitnet_linear(_ptr(packed), _ptr(gamma), N, K, _ptr(x), M, _ptr(y), _ptr(y32),
@@ -188,9 +200,11 @@ class FfnWeights:
     norm2_w: torch.Tensor | None = None
 
 
-def bitnet_ffn(x: torch.Tensor, w: FfnWeights, eps: float = 1e-5, y=None, debug: bool = False,
+def bitnet_ffn(x: torch.Tensor, w: FfnWeights, eps: float = 1e-5, y=None, debug=False,
                workspace=None):
-    """Fused FFN block.  Returns (y bf16 [M,H], dict of debug outputs or None)."""
+    """Fused FFN block.  Returns (y bf16 [M,H], dict of debug outputs or None).
+    `debug` is False, True (the binding allocates the debug outputs) or a dict
+    of preallocated tensors with the keys below."""
     _bits16(x, "x")
     M, H = x.shape
     I = w.gate.shape[0]
@@ -198,7 +212,9 @@ def bitnet_ffn(x: torch.Tensor, w: FfnWeights, eps: float = 1e-5, y=None, debug:
     y = torch.empty((M, H), dtype=torch.bfloat16, device=dev) if y is None else y
     dbg = None
     dstruct = None
-    if debug:
+    if isinstance(debug, dict):
+        dbg = debug
+    elif debug:
         dbg = {
             "xq1": torch.empty((M, H), dtype=torch.int8, device=dev),
             "acc_gate": torch.empty((M, I), dtype=torch.int32, device=dev),
@@ -208,6 +224,7 @@ def bitnet_ffn(x: torch.Tensor, w: FfnWeights, eps: float = 1e-5, y=None, debug:
             "acc_down": torch.empty((M, H), dtype=torch.int32, device=dev),
             "y_f32": torch.empty((M, H), dtype=torch.float32, device=dev),
         }
+    if dbg is not None:
         dstruct = FfnDebug(*[_ptr(dbg[k]) for k in
                              ("xq1", "acc_gate", "acc_up", "h", "xq2", "acc_down", "y_f32")])
     nb = lib().bitnet_ffn_workspace_size(M, H, I)

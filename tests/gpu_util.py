@@ -51,3 +51,34 @@ def assert_bf16_close(got_bits: np.ndarray, want_bits: np.ndarray, got32, want32
 
 def oracle_pack(W: np.ndarray):
     return O.pack_weights(W)
+
+
+class Guarded:
+    """A device output with guard bands: the tensor `t` sits inside a larger
+    allocation whose 256 bytes before it and 4 KB after it hold a sentinel
+    byte pattern.  check() asserts that no kernel wrote outside `t` (the
+    bounds check that stands in for a memory checker)."""
+
+    HEAD = 256
+    TAIL = 4096
+    SENTINEL = 0xA5
+
+    def __init__(self, shape, dtype):
+        es = torch.empty((), dtype=dtype).element_size()
+        self.n = int(np.prod(shape))
+        self.head = self.HEAD // es
+        self.full = torch.empty(self.head + self.n + self.TAIL // es, dtype=dtype, device="cuda")
+        self.full.view(torch.uint8).fill_(self.SENTINEL)
+        self.t = self.full[self.head:self.head + self.n].view(shape)
+        self.es = es
+
+    def check(self):
+        raw = self.full.view(torch.uint8)
+        lo = self.head * self.es
+        hi = lo + self.n * self.es
+        assert bool((raw[:lo] == self.SENTINEL).all()), "write before the start of an output"
+        assert bool((raw[hi:] == self.SENTINEL).all()), "write past the end of an output"
+
+
+def guarded(shape, dtype):
+    return Guarded(shape, dtype)

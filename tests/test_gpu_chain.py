@@ -11,7 +11,7 @@ import torch
 from oracle import bitlinear as O
 from ternary_weight_linear_int8_b200 import bitnet as B
 from ternary_weight_linear_int8_b200 import inputs
-from tests.gpu_util import dev_bits, dev_f32, host_bits
+from tests.gpu_util import dev_bits, dev_f32, guarded, host_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -51,6 +51,26 @@ def test_chain_small_layers_match_oracle(M):
     ys = _run_chain(Ws, x)
     for l, want in enumerate(_oracle_chain(Ws, x)):
         assert np.array_equal(host_bits(ys[l]), want), f"layer {l}"
+
+
+@pytest.mark.parametrize("M", [2, 4, 8])
+def test_chain_2b_shapes_batched(M):
+    """2B-class layers, up [6912,2560] then down [2560,6912], twice, with M
+    tokens carrying outlier channels: every layer's output equals the
+    oracle's, and no layer writes outside its output."""
+    L = 4
+    x = inputs.activations((M, 2560), seed=M, outliers=True)
+    Ws = [inputs.weights(*((6912, 2560) if l % 2 == 0 else (2560, 6912)),
+                         seed=inputs.layer_seed(l)) for l in range(L)]
+    want = _oracle_chain(Ws, x)
+    packs = [B.bitnet_pack_weights(dev_f32(W)) for W in Ws]
+    outs = [guarded((M, W.shape[0]), torch.bfloat16) for W in Ws]
+    B.bitnet_linear_chain([p for p, _ in packs], [g for _, g in packs], dev_bits(x),
+                          ys=[o.t for o in outs])
+    torch.cuda.synchronize()
+    for l in range(L):
+        assert np.array_equal(host_bits(outs[l].t), want[l]), f"layer {l}"
+        outs[l].check()
 
 
 def test_chain_of_70_layers():

@@ -13,7 +13,7 @@ from oracle import bitlinear as O
 from ternary_weight_linear_int8_b200 import bitnet as B
 from ternary_weight_linear_int8_b200 import inputs
 from tests.gpu_util import (assert_bf16_close, assert_f32_rel, dev_bits, dev_f32, dev_u8,
-                            f32_bits, host_bits)
+                            f32_bits, guarded, host_bits)
 
 pytestmark = pytest.mark.gpu
 
@@ -33,6 +33,54 @@ PACK_SHAPES = [(400, 512, 1000), (7, 68, 1), (1, 4, 2), (33, 1024, 3), (6912, 25
 def test_pack_matches_oracle(N, K, seed):
     W = inputs.weights(N, K, seed=seed)
     p_ref, g_ref = O.pack_weights(W)
+    pg, gg = guarded((N, K // 4), torch.uint8), guarded((1,), torch.float32)
+    p, g = B.bitnet_pack_weights(dev_f32(W), packed=pg.t, gamma=gg.t)
+    assert f32_bits(g.cpu().numpy())[0] == f32_bits(g_ref)
+    assert np.array_equal(p.cpu().numpy(), p_ref)
+    pg.check()
+    gg.check()
+
+
+def _threshold_weights(N, K, seed):
+    """Gaussian weights with 48 entries placed exactly on the ternary
+    rounding thresholds of their own matrix: +-0.5*(gamma+1e-5), the fp32
+    neighbours of those, and +-1.5*(gamma+1e-5).  gamma depends on the
+    placed values, so the placement is repeated until gamma stops moving."""
+    rng = np.random.default_rng(seed)
+    W = inputs.weights(N, K, rng=rng)
+    pos = rng.choice(N * K, 48, replace=False)
+    for _ in range(20):
+        den = np.float32(O.absmean_gamma(W)) + O.EPS_F32
+        half = np.float32(den * np.float32(0.5))
+        up, dn = np.nextafter(half, np.float32(1)), np.nextafter(half, np.float32(0))
+        th = np.float32(den * np.float32(1.5))
+        vals = np.array([half, -half, up, -up, dn, -dn, th, -th], np.float32)
+        W2 = W.copy()
+        W2.ravel()[pos] = vals[np.arange(48) % 8]
+        if np.array_equal(W2, W):
+            break
+        W = W2
+    else:
+        raise AssertionError("threshold placement did not settle")
+    return W, pos
+
+
+@pytest.mark.parametrize("N,K", [(64, 256), (6912, 2560)])
+def test_pack_threshold_weights(N, K):
+    """Weights exactly on +-0.5 (gamma + 1e-5) round half to even (to 0),
+    their fp32 neighbours go wherever the fp32 quotient lands, and
+    +-1.5 (gamma + 1e-5) clamps to +-1: GPU codes and gamma equal the
+    oracle's, and the oracle confirms the placed values sit on the
+    thresholds of the final gamma."""
+    W, pos = _threshold_weights(N, K, seed=N + K)
+    g_ref = O.absmean_gamma(W)
+    den = np.float32(g_ref) + O.EPS_F32
+    q = (W.ravel()[pos] / den).astype(np.float32)
+    assert np.all(np.abs(q[0::8]) == 0.5) and np.all(np.abs(q[1::8]) == 0.5)
+    w_ref = O.ternarize(W, g_ref).ravel()[pos]
+    assert np.all(w_ref[0::8] == 0) and np.all(w_ref[1::8] == 0)
+    assert np.all(w_ref[6::8] == 1) and np.all(w_ref[7::8] == -1)
+    p_ref, _ = O.pack_weights(W)
     p, g = B.bitnet_pack_weights(dev_f32(W))
     assert f32_bits(g.cpu().numpy())[0] == f32_bits(g_ref)
     assert np.array_equal(p.cpu().numpy(), p_ref)
@@ -81,10 +129,13 @@ def test_quant_act_matches_oracle(M, K, outl):
     if M > 2:
         x[2, :] = 0                # an all-zero token
     q_ref, s_ref, r_ref = O.act_quant(x)
-    q, s, r = B.bitnet_quant_act(dev_bits(x))
+    outs = [guarded((M, K), torch.int8), guarded((M,), torch.float32), guarded((M,), torch.int32)]
+    q, s, r = B.bitnet_quant_act(dev_bits(x), xq=outs[0].t, scale=outs[1].t, rowsum=outs[2].t)
     assert np.array_equal(q.cpu().numpy(), q_ref)
     assert np.array_equal(f32_bits(s.cpu().numpy()), f32_bits(s_ref))
     assert np.array_equal(r.cpu().numpy(), r_ref)
+    for o in outs:
+        o.check()
 
 
 # ------------------------------------------------------------- BitLinear
@@ -92,7 +143,8 @@ def test_quant_act_matches_oracle(M, K, outl):
 # without split-K), and the ragged-K kernel.
 LINEAR_SHAPES = [
     (1, 6912, 2560), (1, 2560, 6912), (8, 400, 512), (2, 7, 64), (3, 1, 128), (5, 33, 1024),
-    (4, 6912, 2560), (1, 257, 8192),
+    (4, 6912, 2560), (1, 257, 8192), (4, 2560, 6912), (8, 2560, 6912), (8, 6912, 2560),
+    (2, 2560, 6912), (3, 6912, 2560),
     (9, 400, 512), (16, 6912, 2560), (64, 2560, 6912), (65, 257, 640), (17, 1, 256),
     (300, 1000, 1024), (129, 128, 128), (256, 300, 2560),
     (8, 400, 68), (3, 5, 4), (1, 9, 20), (70, 13, 36),
@@ -109,6 +161,63 @@ def _linear_case(M, N, K, seed=0, outliers=True):
 @pytest.mark.parametrize("M,N,K", LINEAR_SHAPES)
 def test_linear_matches_oracle(M, N, K):
     x, W = _linear_case(M, N, K)
+    ref = O.linear_from_float(W, x)
+    p, g = B.bitnet_pack_weights(dev_f32(W))
+    outs = [guarded((M, N), torch.bfloat16), guarded((M, N), torch.float32),
+            guarded((M, N), torch.int32)]
+    y, y32, acc = B.bitnet_linear(p, g, dev_bits(x), y=outs[0].t, y_f32=outs[1].t, acc=outs[2].t)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"].astype(np.int32))
+    assert np.array_equal(f32_bits(y32.cpu().numpy()), f32_bits(ref["y32"]))
+    assert np.array_equal(host_bits(y), ref["y"])
+    for o in outs:
+        o.check()
+
+
+def _edge_tokens(M, K, seed):
+    """Tokens that pin the quantiser's definition on the GPU:
+    0: max |x| = 2 (s = 63.5 exactly) with +-1.0 entries, x*s = +-63.5, a tie
+       that rounds to the even +-64;
+    1: max |x| = 63.5 (s = 2) with +-0.25, 0.75, 1.25: ties at 0.5, 1.5,
+       2.5 -> 0, 2, 2;
+    2: a non-zero token whose max |x| is below the 1e-5 floor (s = 127/1e-5,
+       not 127/(a + 1e-5));
+    3: all zeros; the rest ~N(0,1)."""
+    rng = np.random.default_rng(seed)
+    xf = rng.standard_normal((M, K)).astype(np.float32)
+    rows = []
+    r0 = (rng.standard_normal(K) * 0.4).clip(-1.9, 1.9).astype(np.float32)
+    r0[: K // 8] = np.where(np.arange(K // 8) % 2 == 0, 1.0, -1.0)
+    r0[K // 8] = 2.0
+    rows.append(r0)
+    r1 = (rng.standard_normal(K) * 3).clip(-60, 60).astype(np.float32)
+    r1[: 3 * (K // 16)] = np.tile(np.array([0.25, 0.75, 1.25], np.float32), K // 16)
+    r1[K // 2] = -63.5
+    rows.append(r1)
+    rows.append((rng.standard_normal(K) * 2e-6).clip(-9e-6, 9e-6).astype(np.float32))
+    rows.append(np.zeros(K, np.float32))
+    for i, r in enumerate(rows[:M]):
+        xf[i] = r
+    return inputs.to_bf16_bits(xf)
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 9, 64])
+@pytest.mark.parametrize("K", [512, 2560])
+def test_linear_edge_activations(M, K):
+    """Rounding ties, a sub-floor absmax and a zero token, through the
+    standalone quantiser and every BitLinear path (decode, tensor-core)."""
+    N = 300
+    x = _edge_tokens(M, K, seed=M * 131 + K)
+    ref_q, ref_s, _ = O.act_quant(x)
+    if M >= 2:
+        assert ref_q[0][np.flatnonzero(O.bf16_bits_to_f32(x[0]) == 1.0)].min() == 64
+        assert ref_q[1][np.flatnonzero(O.bf16_bits_to_f32(x[1]) == 0.75)].min() == 2
+    if M >= 3:
+        xs = O.bf16_bits_to_f32(x[2])
+        assert 0 < np.abs(xs).max() < 1e-5 and ref_s[2] == np.float32(127.0) / np.float32(1e-5)
+    q, s, _ = B.bitnet_quant_act(dev_bits(x))
+    assert np.array_equal(q.cpu().numpy(), ref_q)
+    assert np.array_equal(f32_bits(s.cpu().numpy()), f32_bits(ref_s))
+    W = inputs.weights(N, K, seed=K + 5)
     ref = O.linear_from_float(W, x)
     p, g = B.bitnet_pack_weights(dev_f32(W))
     y, y32, acc = B.bitnet_linear(p, g, dev_bits(x), want_f32=True, want_acc=True)
@@ -196,12 +305,26 @@ def _ffn_case(M, H, I, seed=0, gains=True):
 
 
 def _run_ffn(x, Wg, Wu, Wd, n1, n2, eps=1e-5):
+    """The FFN with every output (y and the debug intermediates) allocated
+    inside guard bands, which are checked after the call."""
     pg, gg = B.bitnet_pack_weights(dev_f32(Wg))
     pu, gu = B.bitnet_pack_weights(dev_f32(Wu))
     pd, gd = B.bitnet_pack_weights(dev_f32(Wd))
     w = B.FfnWeights(pg, gg, pu, gu, pd, gd,
                      None if n1 is None else dev_f32(n1), None if n2 is None else dev_f32(n2))
-    return B.bitnet_ffn(dev_bits(x), w, eps=eps, debug=True)
+    M, H = x.shape
+    I = Wg.shape[0]
+    specs = {"xq1": ((M, H), torch.int8), "acc_gate": ((M, I), torch.int32),
+             "acc_up": ((M, I), torch.int32), "h": ((M, I), torch.float32),
+             "xq2": ((M, I), torch.int8), "acc_down": ((M, H), torch.int32),
+             "y_f32": ((M, H), torch.float32)}
+    g = {k: guarded(*v) for k, v in specs.items()}
+    gy = guarded((M, H), torch.bfloat16)
+    y, dbg = B.bitnet_ffn(dev_bits(x), w, eps=eps, y=gy.t, debug={k: v.t for k, v in g.items()})
+    torch.cuda.synchronize()
+    for v in list(g.values()) + [gy]:
+        v.check()
+    return y, dbg
 
 
 def _check_ffn(ref, y, dbg, rows=None):
@@ -258,23 +381,25 @@ def test_fullsize_decode_chain_2b():
 
 
 @pytest.mark.parametrize("N,K", [(6912, 2560), (2560, 6912)])
-def test_fullsize_prefill_sampled_rows(N, K):
-    """Prefill M=4096 on the tensor-core kernel; the oracle checks 48
-    seed-chosen tokens (tokens are independent)."""
+def test_fullsize_prefill_all_rows(N, K):
+    """Prefill M=4096 on the tensor-core kernel, every token checked against
+    the oracle, outputs inside guard bands."""
     M = 4096
     x = inputs.activations((M, K), seed=0)
     W = inputs.weights(N, K, seed=1000)
-    rows = np.sort(np.random.default_rng(123).choice(M, 48, replace=False))
-    rows[-1] = M - 1
-    ref = O.linear_from_float(W, x[rows])
+    ref = O.linear_from_float(W, x)
     p, g = B.bitnet_pack_weights(dev_f32(W))
-    y, y32, acc = B.bitnet_linear(p, g, dev_bits(x), want_f32=True, want_acc=True)
-    assert np.array_equal(acc.cpu().numpy()[rows], ref["acc"].astype(np.int32))
-    assert np.array_equal(f32_bits(y32.cpu().numpy()[rows]), f32_bits(ref["y32"]))
-    assert np.array_equal(host_bits(y)[rows], ref["y"])
+    outs = [guarded((M, N), torch.bfloat16), guarded((M, N), torch.float32),
+            guarded((M, N), torch.int32)]
+    y, y32, acc = B.bitnet_linear(p, g, dev_bits(x), y=outs[0].t, y_f32=outs[1].t, acc=outs[2].t)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"].astype(np.int32))
+    assert np.array_equal(f32_bits(y32.cpu().numpy()), f32_bits(ref["y32"]))
+    assert np.array_equal(host_bits(y), ref["y"])
+    for o in outs:
+        o.check()
 
 
-@pytest.mark.parametrize("M", [16, 64])
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16, 64])
 def test_fullsize_batched_decode(M):
     for N, K in [(6912, 2560), (2560, 6912)]:
         x = inputs.activations((M, K), seed=0, outliers=True)
@@ -298,11 +423,18 @@ def ffn_100b():
 @pytest.mark.parametrize("M", [1, 2048])
 def test_fullsize_ffn_100b(M, ffn_100b):
     """100B-class FFN block, hidden 8192, intermediate 28672.  M=1 is checked
-    whole; M=2048 on 8 seed-chosen tokens."""
+    whole; M=2048 on the first and last token of every 64-token block (so
+    every token tile of the tensor-core kernel, 64, 128, 192 or 256 wide,
+    has its edges checked) plus 16 seed-chosen tokens."""
     H = 8192
     Wg, Wu, Wd, packed = ffn_100b
     x = inputs.activations((M, H), seed=0)
-    rows = np.arange(M) if M == 1 else np.sort(np.random.default_rng(7).choice(M, 8, replace=False))
+    if M == 1:
+        rows = np.arange(1)
+    else:
+        edges = np.concatenate([np.arange(0, M, 64), np.arange(63, M, 64)])
+        extra = np.random.default_rng(7).choice(M, 16, replace=False)
+        rows = np.unique(np.concatenate([edges, extra]))
     ref = O.ffn(x[rows], *packed, None, None, 1e-5)
     y, dbg = _run_ffn(x, Wg, Wu, Wd, None, None)
     _check_ffn(ref, y, dbg, rows=rows)

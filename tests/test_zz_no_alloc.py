@@ -15,6 +15,7 @@ import torch
 
 from ternary_weight_linear_int8_b200 import bitnet as B
 from ternary_weight_linear_int8_b200 import inputs
+from tests.gpu_util import guarded
 
 SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -44,9 +45,11 @@ def test_noalloc_matches_linear_two_calls_in_a_row(M, N, K):
     refs = [_bits(B.bitnet_linear(p, g, x)[0]) for x in xs]
     assert not np.array_equal(refs[0], refs[1])
     for x, ref in zip(xs, refs):            # two calls in a row, different inputs
-        y = B.bitnet_linear_noalloc(p, g, x)
+        out = guarded((M, N), torch.bfloat16)
+        y = B.bitnet_linear_noalloc(p, g, x, y=out.t)
         torch.cuda.synchronize()
         assert np.array_equal(_bits(y), ref)
+        out.check()
     assert B.bitnet_last_device_status() == 0
 
 
