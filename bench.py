@@ -441,6 +441,14 @@ def profile_case(case):
         p, g = B.bitnet_pack_weights(torch.from_numpy(inputs.weights(N, K, seed=2000)).to(dev))
         for _ in range(4):
             B.bitnet_linear(p, g, x)
+    elif case == "chain2b":
+        packs = build_decode_chain(B, inputs, torch, dev, n_layers=4)
+        x = torch.from_numpy(inputs.activations((1, HIDDEN), seed=0).view(np.int16)).to(dev)
+        bufs = [torch.empty((1, INTER), dtype=torch.bfloat16, device=dev),
+                torch.empty((1, HIDDEN), dtype=torch.bfloat16, device=dev)]
+        call = ChainCall(B, torch, packs, bufs, dev)
+        for _ in range(3):
+            call(x)
     elif case in ("batched8", "batched16"):
         M = int(case[len("batched"):])
         packs = build_decode_chain(B, inputs, torch, dev, n_layers=6)
@@ -607,7 +615,8 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--profile-case", choices=["prefill", "prefill_down", "ffn2048", "gemv_big", "batched8", "batched16"],
+    ap.add_argument("--profile-case", choices=["prefill", "prefill_down", "ffn2048", "gemv_big", "batched8", "batched16",
+                             "chain2b"],
                     default=None,
                     help="run a few calls of one workload for an ncu capture, print nothing")
     args = ap.parse_args()

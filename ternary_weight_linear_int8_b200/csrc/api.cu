@@ -16,6 +16,10 @@ bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* ga
                                   int32_t* rowsum, double* sumsq, int8_t* xq_natural,
                                   cudaStream_t stream);
 bitnet_status bitnet_decode_launch(const DecodeOp& op, int M, int num_sms, cudaStream_t stream);
+bool bitnet_resident_fits(int64_t M, int64_t N, int64_t K, int num_sms);
+bitnet_status bitnet_resident_launch(const uint8_t* w, const float* gamma, int N, int K,
+                                     const uint16_t* x, int M, uint16_t* y, float* y_f32,
+                                     int32_t* acc, int num_sms, cudaStream_t stream);
 bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
                                  const uint8_t* w1, GemmArgs a, int bn, int num_sms,
                                  cudaStream_t stream);
@@ -55,19 +59,25 @@ struct DevInfo {
   int major = 0;
 };
 
+// Per-device attributes, cached; an entry packs (major << 16) | SM count into
+// one atomic word, so concurrent host threads read either 0 (not yet known,
+// each queries it) or a complete entry.
 bitnet_status device_info(DevInfo* out) {
-  static DevInfo cache[64];
+  static std::atomic<uint32_t> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BITNET_ERR_CUDA;
   if (dev < 0 || dev >= 64) return BITNET_ERR_UNSUPPORTED;
-  if (cache[dev].num_sms == 0) {
-    DevInfo d;
-    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+  uint32_t v = cache[dev].load(std::memory_order_acquire);
+  if (v == 0) {
+    int sms = 0, major = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
       return BITNET_ERR_CUDA;
-    cache[dev] = d;
+    v = ((uint32_t)major << 16) | ((uint32_t)sms & 0xffffu);
+    cache[dev].store(v, std::memory_order_release);
   }
-  *out = cache[dev];
+  out->num_sms = (int)(v & 0xffffu);
+  out->major = (int)(v >> 16);
   if (out->major != 10) return BITNET_ERR_UNSUPPORTED;
   return BITNET_OK;
 }
@@ -245,6 +255,9 @@ bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N
   cudaStream_t s = as_stream(stream);
   const LinearPath p = linear_path(M, K);
   if (p == kPathGemv) {
+    if (bitnet_resident_fits(M, N, K, d.num_sms))
+      return bitnet_resident_launch(packed, gamma, (int)N, (int)K, x, (int)M, y, y_f32, acc,
+                                    d.num_sms, s);
     DecodeOp a{};
     a.mode = kLinear;
     a.w0 = packed; a.gamma0 = gamma;

@@ -4,6 +4,7 @@
 #include "pack.cu"
 #include "quant.cu"
 #include "gemv.cu"
+#include "resident.cu"
 #include "gemm.cu"
 #include "api.cu"
 #include "noalloc.cu"

@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "bitnet.h"
 
 namespace bitnet {
@@ -178,6 +180,13 @@ __device__ __forceinline__ int quant_code(float v, float s) {
   q = q > 127 ? 127 : q;
   return q;
 }
+// The same code in one conversion: round to nearest even and saturate to
+// [-128, 127] (identical to quant_code for finite v * s).
+__device__ __forceinline__ int quant_code_sat(float v, float s) {
+  int q;
+  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(q) : "f"(__fmul_rn(v, s)));
+  return q;
+}
 // fp32 -> bf16 bits, round to nearest even, on the integer pipe (finite x).
 __device__ __forceinline__ uint32_t f32_to_bf16_rne_bits(float x) {
   const uint32_t u = __float_as_uint(x);
@@ -209,6 +218,9 @@ __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
                "r"(v.z), "r"(v.w)
                : "memory");
+}
+__device__ __forceinline__ void sts_u16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 __device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
@@ -266,6 +278,25 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 __host__ __device__ __forceinline__ int64_t perm_k(int64_t k) {
   const int64_t i = k & 15;
   return (k & ~int64_t(15)) | ((i & 3) << 2) | (i >> 2);
+}
+
+// Host: set a kernel's dynamic shared-memory limit (and, if given, its
+// shared-memory carveout) once per device; `mask` holds one bit per device
+// (ordinals 0..63) and may be shared by concurrent host threads.
+template <typename Kernel>
+inline cudaError_t set_smem_attr_once(std::atomic<uint64_t>& mask, Kernel* kernel, int bytes,
+                                      int carveout = -1) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const uint64_t bit = 1ull << dev;
+  if (mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && carveout >= 0)
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carveout);
+  if (e == cudaSuccess) mask.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
 }
 
 }  // namespace bitnet

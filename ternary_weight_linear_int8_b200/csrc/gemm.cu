@@ -615,16 +615,9 @@ static cudaError_t launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw0,
                                  const CUtensorMap& tw1, const CUtensorMap& ty, const GemmArgs& a,
                                  dim3 grid, cudaStream_t stream) {
   using C = GemmCfg<BN, NMAT>;
-  static int configured_dev_mask = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!(configured_dev_mask & (1 << (dev & 31)))) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<MODE, BN, NMAT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmem);
-    if (e != cudaSuccess) return e;
-    configured_dev_mask |= 1 << (dev & 31);
-  }
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = set_smem_attr_once(configured, gemm_kernel<MODE, BN, NMAT>, (int)C::kSmem);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kGemmThreads);

@@ -815,15 +815,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int MODE, int MT, int MM>
 static cudaError_t launch_decode(const DecodeParams& p, int grid, size_t smem,
                                  cudaStream_t stream) {
-  static unsigned long long configured = 0;   // one bit per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!(configured & (1ull << (dev & 63)))) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<MODE, MT, MM>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    if (e != cudaSuccess) return e;
-    configured |= 1ull << (dev & 63);
-  }
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = set_smem_attr_once(configured, decode_kernel<MODE, MT, MM>, 227 * 1024);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(kThreads);

@@ -1,0 +1,430 @@
+// Resident decode kernel: BitLinear for a few tokens on layers whose
+// per-CTA slice of packed weights fits in shared memory next to the
+// quantised activations (2B-class decode: about 30 KB of weights per SM).
+//
+// dashen-tech.com "BitNet.cpp 深度解析", section "3.1 計算コア：整数行列乗算":
+// the product with ternary weights is sum_pos - sum_neg, taken here in the
+// offset form sum_k x_q * code - sum_k x_q (code = w + 1) with dp4a on the
+// masked code planes of each packed word, exactly as the streaming decode
+// kernel does.
+//
+// What differs from the streaming decode kernel is the schedule.  Two CTAs
+// fit on each SM (at most 112 KB of shared memory and 64 registers per
+// thread), so with programmatic dependent launch the CTA of the next layer
+// becomes resident while this layer computes.  Its first act is to request
+// its whole weight slice with bulk async copies (before griddepcontrol.wait:
+// weights never depend on the previous kernel), so in a chain of layers the
+// weights land while the layers before finish, and after the wait only the
+// dependent sequence remains: activation loads, per-token absmax and
+// quantisation into shared memory, the products from shared memory and the
+// dequantised stores.
+#include "common.cuh"
+
+namespace bitnet {
+
+struct ResidentParams {
+  const uint8_t* w;        // packed [N, K/4]
+  const float* gamma;
+  const uint16_t* x;       // bf16 [M, K]
+  uint16_t* y;             // bf16 [M, N]
+  float* y_f32;            // optional [M, N]
+  int32_t* acc;            // optional [M, N]
+  int N, K, M;
+  int wk;                  // K-slices per 4-row block (1, 2, 4 or 8)
+  int pieces;              // weight copy groups (1..4), one mbarrier each
+  uint32_t x_off;          // shared-memory offsets (bytes, multiples of 128)
+  uint32_t acc_off;
+  uint32_t w_off;
+};
+
+constexpr int kResWarps = 16;
+constexpr int kResThreads = kResWarps * 32;
+constexpr int kResMaxTok = 8;
+// two CTAs per SM: 228 KB of shared memory per SM, 1 KB reserved per CTA
+constexpr uint32_t kResSmemMax = 112 * 1024;
+constexpr uint32_t kResHead = 1152;     // barriers, token scalars, warp partials
+
+extern __shared__ __align__(128) uint8_t g_res_smem[];
+
+template <int MT, int MM>
+__global__ void __launch_bounds__(kResThreads, 2)
+    resident_kernel(const __grid_constant__ ResidentParams p) {
+  uint64_t* bars = reinterpret_cast<uint64_t*>(g_res_smem);          // [4]
+  float* tok_d = reinterpret_cast<float*>(g_res_smem + 64);          // [8]
+  float* red_f = reinterpret_cast<float*>(g_res_smem + 128);         // [16 warps][8]
+  int* red_i = reinterpret_cast<int*>(g_res_smem + 640);             // [16 warps][8]
+  uint8_t* xq = g_res_smem + p.x_off;                                // [Mpad][K], kernel order
+  int* accs = reinterpret_cast<int*>(g_res_smem + p.acc_off);        // [rows][8] (wk > 1)
+  uint8_t* wsm = g_res_smem + p.w_off;                               // [rows][K/4]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int K = p.K, N = p.N, M = p.M;
+  const int Kb = K >> 2, Kw = K >> 4;
+  const int n0 = (int)(((int64_t)blockIdx.x * N) / gridDim.x);
+  const int n1 = (int)(((int64_t)(blockIdx.x + 1) * N) / gridDim.x);
+  const int R = n1 - n0;
+  const int nblk = (R + 3) >> 2;
+  const int P = p.pieces;
+  const int cs = (nblk + P - 1) / P;   // 4-row blocks per piece
+
+  // ---- weights: the whole slice, in P pieces of cs whole 4-row blocks
+  if (tid == 0) {
+    for (int i = 0; i < P; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+    pdl_launch_dependents();
+    const uint64_t pol = policy_evict_first();
+    for (int i = 0; i < P; ++i) {
+      const int r0 = min(R, 4 * i * cs);
+      const int r1 = min(R, 4 * (i + 1) * cs);
+      if (r1 <= r0) {            // empty piece: complete its phase at once
+        mbar_arrive(&bars[i]);
+        continue;
+      }
+      const uint32_t bytes = (uint32_t)(r1 - r0) * (uint32_t)Kb;
+      mbar_arrive_expect_tx(&bars[i], bytes);
+      const uint8_t* src = p.w + (int64_t)(n0 + r0) * Kb;
+      uint8_t* dst = wsm + (size_t)r0 * Kb;
+      for (uint32_t off = 0; off < bytes; off += 4096u) {
+        const uint32_t nb = bytes - off < 4096u ? bytes - off : 4096u;
+        bulk_g2s(dst + off, src + off, nb, &bars[i], pol);
+      }
+    }
+  }
+  const int Mpad = ((M + MT - 1) / MT) * MT;
+  for (int i = M * K + tid * 16; i < Mpad * K; i += kResThreads * 16)
+    sts_v4(smem_u32(xq + i), make_uint4(0, 0, 0, 0));
+  const int WK = p.wk;
+  if (WK > 1)
+    for (int i = tid; i < nblk * 4 * kResMaxTok; i += kResThreads) accs[i] = 0;
+
+  pdl_wait();
+
+  // ---- per-token absmax (pass 1) and quantisation (pass 2).  A thread owns
+  // (token, 8 consecutive values) pairs; up to two pairs per thread stay in
+  // registers between the passes, otherwise pass 2 loads them again.
+  float gam = 0.f;
+  if (tid < M) gam = *p.gamma;
+  const int Kh = Kw * 2;                 // 8-value pieces per token
+  const int npair = M * Kh;
+  const bool keep = npair <= 2 * kResThreads;
+  uint4 kv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+  float am[MM];
+#pragma unroll
+  for (int m = 0; m < MM; ++m) am[m] = 0.f;
+  auto absmax8 = [](const uint4& v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      mx = fmaxf(mx, fabsf(__uint_as_float(w[i] << 16)));
+      mx = fmaxf(mx, fabsf(__uint_as_float(w[i] & 0xffff0000u)));
+    }
+    return mx;
+  };
+  auto tok_of = [&](int pi) { return MM == 1 ? 0 : pi / Kh; };
+  if (keep) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int pi = tid + i * kResThreads;
+      if (pi < npair) {
+        const int m = tok_of(pi);
+        kv[i] = *reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (pi - m * Kh) * 8);
+        const float mx = absmax8(kv[i]);
+#pragma unroll
+        for (int mm = 0; mm < MM; ++mm)
+          if (mm == m) am[mm] = fmaxf(am[mm], mx);
+      }
+    }
+  } else {
+    for (int pi = tid; pi < npair; pi += kResThreads) {
+      const int m = tok_of(pi);
+      const float mx =
+          absmax8(*reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (pi - m * Kh) * 8));
+#pragma unroll
+      for (int mm = 0; mm < MM; ++mm)
+        if (mm == m) am[mm] = fmaxf(am[mm], mx);
+    }
+  }
+  // warp maxima with one redux each (|x| >= 0, so the bit patterns order
+  // like the values)
+#pragma unroll
+  for (int m = 0; m < MM; ++m) {
+    const uint32_t w = __reduce_max_sync(0xffffffffu, __float_as_uint(am[m]));
+    if (lane == 0 && m < M) red_f[warp * kResMaxTok + m] = __uint_as_float(w);
+  }
+  __syncthreads();
+  float sc[MM];
+#pragma unroll
+  for (int m = 0; m < MM; ++m) {
+    float a = 0.f;
+    if (m < M) {
+      float v[kResWarps];
+#pragma unroll
+      for (int w = 0; w < kResWarps; ++w) v[w] = red_f[w * kResMaxTok + m];
+#pragma unroll
+      for (int h = kResWarps / 2; h > 0; h >>= 1)
+#pragma unroll
+        for (int w = 0; w < h; ++w) v[w] = fmaxf(v[w], v[w + h]);
+      a = v[0];
+    }
+    sc[m] = qscale(a);
+  }
+  if (tid < M) {
+    float s = sc[0];
+#pragma unroll
+    for (int mm = 1; mm < MM; ++mm)
+      if (mm == tid) s = sc[mm];
+    tok_d[tid] = __fdiv_rn(gam, s);
+  }
+  int rs[MM];
+#pragma unroll
+  for (int m = 0; m < MM; ++m) rs[m] = 0;
+  // 8 values k = 16g + 8h + i (i = 0..7) land at slots 4(i%4) + 2h + i/4 of
+  // group g: per code plane t one 16-bit half (values t and t + 4)
+  auto quant8 = [&](int pi, const uint4& v) {
+    const int m = tok_of(pi), hg = pi - m * Kh;
+    float s = sc[0];
+#pragma unroll
+    for (int mm = 1; mm < MM; ++mm)
+      if (mm == m) s = sc[mm];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    int q[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      q[2 * i] = quant_code_sat(__uint_as_float(w[i] << 16), s);
+      q[2 * i + 1] = quant_code_sat(__uint_as_float(w[i] & 0xffff0000u), s);
+    }
+    const uint32_t base =
+        smem_u32(xq) + (uint32_t)(m * K + (hg >> 1) * 16 + 2 * (hg & 1));
+    int sum = 0;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      sts_u16(base + 4 * t, (uint16_t)__byte_perm((uint32_t)q[t], (uint32_t)q[4 + t], 0x0040));
+      sum += q[t] + q[4 + t];
+    }
+#pragma unroll
+    for (int mm = 0; mm < MM; ++mm)
+      if (mm == m) rs[mm] += sum;
+  };
+  if (keep) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int pi = tid + i * kResThreads;
+      if (pi < npair) quant8(pi, kv[i]);
+    }
+  } else {
+    for (int pi = tid; pi < npair; pi += kResThreads) {
+      const int m = tok_of(pi);
+      quant8(pi, *reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (pi - m * Kh) * 8));
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MM; ++m) {
+    const int t = __reduce_add_sync(0xffffffffu, rs[m]);
+    if (lane == 0 && m < M) red_i[warp * kResMaxTok + m] = t;
+  }
+  __syncthreads();
+  // each token's row sum (identical in every thread)
+  int rtot[MM];
+#pragma unroll
+  for (int m = 0; m < MM; ++m) {
+    int t = 0;
+    if (m < M) {
+#pragma unroll
+      for (int w = 0; w < kResWarps; ++w) t += red_i[w * kResMaxTok + m];
+    }
+    rtot[m] = t;
+  }
+
+  // ---- products: items (4-row block b, K-slice q), dealt round robin to the
+  // warps; lane l reads words l, l+32, ... of the slice of each row.
+  auto finish = [&](int r, int m, int v) {
+    int rsum = rtot[0];
+#pragma unroll
+    for (int mm = 1; mm < MM; ++mm)
+      if (mm == m) rsum = rtot[mm];
+    const int ac = v - rsum;
+    const float y32 = __fmul_rn(__int2float_rn(ac), tok_d[m]);
+    const int64_t o = (int64_t)m * N + n0 + r;
+    p.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+    if (p.y_f32) p.y_f32[o] = y32;
+    if (p.acc) p.acc[o] = ac;
+  };
+  constexpr int kUnroll = MT == 1 ? 4 : 2;
+  const int wkl = __ffs(WK) - 1;
+  const int nitems = nblk * WK;
+  const uint32_t x_addr = smem_u32(xq), w_addr = smem_u32(wsm);
+  bool ok = true;
+  int pc = 0;            // weight piece of the current block (blocks only grow)
+  for (int it = warp; it < nitems; it += kResWarps) {
+    const int b = it >> wkl, qs = it & (WK - 1);
+    while ((pc + 1) * cs <= b) ++pc;
+    if (!mbar_wait(&bars[pc], 0)) { ok = false; break; }
+    const int j0 = (qs * Kw) >> wkl, j1 = ((qs + 1) * Kw) >> wkl;
+    uint32_t rowa[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) rowa[r] = w_addr + (uint32_t)(min(4 * b + r, R - 1) * Kb);
+    for (int tg = 0; tg < M; tg += MT) {
+      int acc_r[4][MT];
+      int acc4[4][4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+#pragma unroll
+        for (int t = 0; t < MT; ++t) acc_r[r][t] = 0;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) acc4[r][t] = 0;
+      }
+      const uint32_t xt = x_addr + (uint32_t)(tg * K);
+#pragma unroll kUnroll
+      for (int j = j0 + lane; j < j1; j += 32) {
+        uint32_t w[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) w[r] = lds_u32(rowa[r] + 4u * j);
+        uint4 xv[MT];
+#pragma unroll
+        for (int t = 0; t < MT; ++t) xv[t] = lds_v4(xt + (uint32_t)(t * K) + 16u * j);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          if constexpr (MT == 1) {
+            acc4[r][0] = dp4a_su((int)xv[0].x, w[r] & 0x03030303u, acc4[r][0]);
+            acc4[r][1] = dp4a_su((int)xv[0].y, w[r] & 0x0c0c0c0cu, acc4[r][1]);
+            acc4[r][2] = dp4a_su((int)xv[0].z, w[r] & 0x30303030u, acc4[r][2]);
+            acc4[r][3] = dp4a_su((int)xv[0].w, w[r] & 0xc0c0c0c0u, acc4[r][3]);
+          } else {
+            const uint32_t c0 = w[r] & 0x03030303u;
+            const uint32_t c1 = (w[r] >> 2) & 0x03030303u;
+            const uint32_t c2 = (w[r] >> 4) & 0x03030303u;
+            const uint32_t c3 = (w[r] >> 6) & 0x03030303u;
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+              int v = acc_r[r][t];
+              v = dp4a_su((int)xv[t].x, c0, v);
+              v = dp4a_su((int)xv[t].y, c1, v);
+              v = dp4a_su((int)xv[t].z, c2, v);
+              v = dp4a_su((int)xv[t].w, c3, v);
+              acc_r[r][t] = v;
+            }
+          }
+        }
+      }
+      if constexpr (MT == 1) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          acc_r[r][0] = acc4[r][0] + (acc4[r][1] >> 2) + (acc4[r][2] >> 4) + (acc4[r][3] >> 6);
+      }
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        const int v[4] = {acc_r[0][t], acc_r[1][t], acc_r[2][t], acc_r[3][t]};
+        // butterfly over the 4 rows: lane l ends with row l >> 3
+        int h2[2], h1[1];
+        halve<4>(v, h2, 16, lane);
+        halve<2>(h2, h1, 8, lane);
+        int tot = h1[0];
+        tot += __shfl_xor_sync(0xffffffffu, tot, 4);
+        tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+        tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+        const int r = 4 * b + (lane >> 3), m = tg + t;
+        if ((lane & 7) == 0 && m < M && r < R) {
+          if (WK == 1) finish(r, m, tot);
+          else atomicAdd(&accs[r * kResMaxTok + m], tot);
+        }
+      }
+    }
+  }
+  if (WK > 1) {
+    __syncthreads();
+    for (int o = tid; o < R * M; o += kResThreads) {
+      const int r = MM == 1 ? o : o / M, m = o - r * M;
+      finish(r, m, accs[r * kResMaxTok + m]);
+    }
+  }
+  if (!ok) {
+    // a wait gave up (recorded in the status word): let this CTA's copies
+    // finish, within the same limit, before its shared memory is released
+    for (int i = 0; i < P; ++i) mbar_wait(&bars[i], 0);
+  }
+}
+
+// Host-side plan: does the layer fit, and with how many K-slices and pieces.
+struct ResidentPlan {
+  ResidentParams p;
+  int grid;
+  uint32_t smem;
+};
+
+static uint32_t al128(uint64_t v) { return (uint32_t)((v + 127) & ~uint64_t(127)); }
+
+static bool plan_resident(int M, int N, int K, int num_sms, ResidentPlan* out) {
+  if (M < 1 || M > 3 || K % 64 != 0) return false;
+  const int MT = M == 1 ? 1 : 2;
+  const int Mpad = ((M + MT - 1) / MT) * MT;
+  const int grid = (N + 3) / 4 < num_sms ? (N + 3) / 4 : num_sms;
+  const int rows_max = (N + grid - 1) / grid;
+  const int nblk = (rows_max + 3) / 4;
+  const int Kw = K / 16;
+  // K-slices: rounds of items over the warps x (32-word steps + a fixed
+  // per-item cost of about two steps)
+  int wk = 1;
+  double best = 1e30;
+  for (int c = 1; c <= 8; c *= 2) {
+    if (c > 1 && Kw / c < 32) break;
+    const double rounds = (double)((nblk * c + kResWarps - 1) / kResWarps);
+    const double cost = rounds * ((double)((Kw / c + 31) / 32) + 2.0);
+    if (cost < best - 1e-9) { best = cost; wk = c; }
+  }
+  ResidentParams& p = out->p;
+  p = ResidentParams{};
+  p.N = N; p.K = K; p.M = M; p.wk = wk;
+  p.pieces = nblk < 4 ? nblk : 4;
+  p.x_off = kResHead;
+  p.acc_off = p.x_off + al128((uint64_t)Mpad * K);
+  p.w_off = p.acc_off + (wk > 1 ? al128((uint64_t)nblk * 4 * kResMaxTok * 4) : 0u);
+  const uint64_t total = (uint64_t)p.w_off + al128((uint64_t)nblk * 4 * (K / 4));
+  if (total > kResSmemMax) return false;
+  out->grid = grid;
+  out->smem = (uint32_t)total;
+  return true;
+}
+
+template <int MT, int MM>
+static cudaError_t launch_resident_t(const ResidentPlan& pl, cudaStream_t stream) {
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = set_smem_attr_once(configured, resident_kernel<MT, MM>, (int)kResSmemMax,
+                                     cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)pl.grid);
+  cfg.blockDim = dim3(kResThreads);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, resident_kernel<MT, MM>, pl.p);
+}
+
+}  // namespace bitnet
+
+using namespace bitnet;
+
+// Whether the resident kernel serves this BitLinear shape.
+bool bitnet_resident_fits(int64_t M, int64_t N, int64_t K, int num_sms) {
+  if (M > 8 || N > 0x7fffffff || K > 0x7fffffff) return false;
+  ResidentPlan pl;
+  return plan_resident((int)M, (int)N, (int)K, num_sms, &pl);
+}
+
+bitnet_status bitnet_resident_launch(const uint8_t* w, const float* gamma, int N, int K,
+                                     const uint16_t* x, int M, uint16_t* y, float* y_f32,
+                                     int32_t* acc, int num_sms, cudaStream_t stream) {
+  ResidentPlan pl;
+  if (!plan_resident(M, N, K, num_sms, &pl)) return BITNET_ERR_UNSUPPORTED;
+  pl.p.w = w; pl.p.gamma = gamma; pl.p.x = x; pl.p.y = y; pl.p.y_f32 = y_f32; pl.p.acc = acc;
+  cudaError_t e;
+  if (M == 1) e = launch_resident_t<1, 1>(pl, stream);
+  else if (M == 2) e = launch_resident_t<2, 2>(pl, stream);
+  else e = launch_resident_t<2, 4>(pl, stream);
+  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
