@@ -45,7 +45,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 INT8_OVER_BF16 = 2.0            # nominal dense int8 : bf16 tensor-core ratio (4.5 : 2.25 PFLOP/s)
 # the decode kernel's sources: a committed ncu summary's traffic figure is
 # reported only while these are unchanged since its capture
-KERNEL_SOURCES = ["common.cuh", "gemv.cu"]
+KERNEL_SOURCES = ["common.cuh", "resident.cu"]
 
 
 # ---------------------------------------------------------------- helpers
@@ -529,7 +529,7 @@ def run_ours(args, world, rank, local):
     alg_bytes = packed_bytes / n_mat + 2 * HIDDEN + 2 * INTER + 4
     launch_s = step_s / n_mat
     achieved = alg_bytes / launch_s / 1e9
-    traffic = profile_traffic("decode_gemv_2b_m1.md")
+    traffic = profile_traffic("decode_resident_2b_m1.md")
 
     # --------------------------------------------------- e2e through the API
     # per step: pinned host x -> device, one bitnet_linear_chain call through
@@ -585,7 +585,7 @@ def run_ours(args, world, rank, local):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
-                         "traffic": traffic, "kernel": "decode_kernel<Linear,1,1>",
+                         "traffic": traffic, "kernel": "resident_kernel (1 token)",
                          "peak_source": pk["source"],
                          "algorithmic_bytes_per_launch": alg_bytes,
                          "launch_us": round(launch_s * 1e6, 3)},

@@ -199,8 +199,8 @@ BITNET_API bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int
  * decode step runs them one after the other; the pages define no call that
  * runs several layers, this one only schedules them.
  *
- * The layers are launched one after the other on `stream`, each exactly as
- * bitnet_linear launches it (decode kernels start streaming their weights
+ * The layers are launched one after the other on `stream`, each with the
+ * kernel bitnet_linear would use (decode kernels start loading their weights
  * while the layer before them finishes).
  *
  * L        number of layers, >= 1.

@@ -234,25 +234,16 @@ size_t bitnet_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
   return linear_ws_layout(M, N, K).total;
 }
 
-bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N, int64_t K,
-                            const uint16_t* x, int64_t M, uint16_t* y, float* y_f32,
-                            int32_t* acc, void* workspace, size_t workspace_bytes,
-                            void* stream) {
-  if (!packed || !gamma || !x || !y) return BITNET_ERR_INVALID_ARG;
-  if (M < 1 || N < 1 || K < 4 || K % 4 != 0 || K > 524288 || M > 0x7fffffff || N > 0x7fffffff)
-    return BITNET_ERR_SHAPE;
-  if (!aligned16(packed) || !aligned16(x) || !aligned16(y) || ((uintptr_t)gamma & 3u) ||
-      ((uintptr_t)y_f32 & 3u) || ((uintptr_t)acc & 3u))
-    return BITNET_ERR_ALIGN;
-  const LinearWs L = linear_ws_layout(M, N, K);
-  if (L.total > 0) {
-    if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
-  }
-  DevInfo d;
-  bitnet_status st = device_info(&d);
-  if (st != BITNET_OK) return st;
-  cudaStream_t s = as_stream(stream);
+}  // extern "C"
+
+namespace {
+
+// Enqueue one validated BitLinear.
+bitnet_status linear_enqueue(const uint8_t* packed, const float* gamma, int64_t N, int64_t K,
+                             const uint16_t* x, int64_t M, uint16_t* y, float* y_f32,
+                             int32_t* acc, void* workspace, const LinearWs& L, const DevInfo& d,
+                             cudaStream_t s) {
+  bitnet_status st = BITNET_OK;
   const LinearPath p = linear_path(M, K);
   if (p == kPathGemv) {
     if (bitnet_resident_fits(M, N, K, d.num_sms))
@@ -295,6 +286,32 @@ bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N
       return BITNET_ERR_CUDA;
   }
   return bitnet_gemm_launch(0 /*linear*/, xq, packed, nullptr, a, bn, d.num_sms, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N, int64_t K,
+                            const uint16_t* x, int64_t M, uint16_t* y, float* y_f32,
+                            int32_t* acc, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (!packed || !gamma || !x || !y) return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 4 || K % 4 != 0 || K > 524288 || M > 0x7fffffff || N > 0x7fffffff)
+    return BITNET_ERR_SHAPE;
+  if (!aligned16(packed) || !aligned16(x) || !aligned16(y) || ((uintptr_t)gamma & 3u) ||
+      ((uintptr_t)y_f32 & 3u) || ((uintptr_t)acc & 3u))
+    return BITNET_ERR_ALIGN;
+  const LinearWs L = linear_ws_layout(M, N, K);
+  if (L.total > 0) {
+    if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  }
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  return linear_enqueue(packed, gamma, N, K, x, M, y, y_f32, acc, workspace, L, d,
+                        as_stream(stream));
 }
 
 size_t bitnet_ffn_workspace_size(int64_t M, int64_t H, int64_t I) {
@@ -437,11 +454,14 @@ bitnet_status bitnet_linear_chain(int64_t L, const uint8_t* const* packed,
   DevInfo d;
   bitnet_status st = device_info(&d);
   if (st != BITNET_OK) return st;
-  // one launch per layer, in order on the stream; each decode kernel starts
-  // streaming its weights while the previous layer finishes
+  // one launch per layer, in order on the stream (validated above, planned
+  // here); each decode kernel starts loading its weights while the layer
+  // before it finishes
+  const cudaStream_t s = as_stream(stream);
   for (int64_t l = 0; l < L; ++l) {
-    st = bitnet_linear(packed[l], gamma[l], N[l], K[l], l == 0 ? x : y[l - 1], M, y[l], nullptr,
-                       nullptr, workspace, workspace_bytes, stream);
+    const LinearWs lw = linear_ws_layout(M, N[l], K[l]);
+    st = linear_enqueue(packed[l], gamma[l], N[l], K[l], l == 0 ? x : y[l - 1], M, y[l], nullptr,
+                        nullptr, workspace, lw, d, s);
     if (st != BITNET_OK) return st;
   }
   return BITNET_OK;

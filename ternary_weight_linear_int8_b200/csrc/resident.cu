@@ -20,6 +20,10 @@
 // dequantised stores.
 #include "common.cuh"
 
+#ifndef RESIDENT_WARPS
+#define RESIDENT_WARPS 16
+#endif
+
 namespace bitnet {
 
 struct ResidentParams {
@@ -37,22 +41,26 @@ struct ResidentParams {
   uint32_t w_off;
 };
 
-constexpr int kResWarps = 16;
-constexpr int kResThreads = kResWarps * 32;
 constexpr int kResMaxTok = 8;
-// two CTAs per SM: 228 KB of shared memory per SM, 1 KB reserved per CTA
-constexpr uint32_t kResSmemMax = 112 * 1024;
-constexpr uint32_t kResHead = 1152;     // barriers, token scalars, warp partials
+constexpr int kResMaxWarps = 32;
+// 16 warps: two CTAs per SM (228 KB of shared memory per SM, 1 KB reserved
+// per CTA); 32 warps: one CTA per SM
+__host__ __device__ constexpr uint32_t res_smem_max(int nw) {
+  return nw == 16 ? 112u * 1024u : 200u * 1024u;
+}
+constexpr uint32_t kResHead = 2176;     // barriers, token scalars, warp partials
 
 extern __shared__ __align__(128) uint8_t g_res_smem[];
 
-template <int MT, int MM>
-__global__ void __launch_bounds__(kResThreads, 2)
+template <int MT, int MM, int NW>
+__global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
     resident_kernel(const __grid_constant__ ResidentParams p) {
+  constexpr int kResWarps = NW;
+  constexpr int kResThreads = NW * 32;
   uint64_t* bars = reinterpret_cast<uint64_t*>(g_res_smem);          // [4]
   float* tok_d = reinterpret_cast<float*>(g_res_smem + 64);          // [8]
-  float* red_f = reinterpret_cast<float*>(g_res_smem + 128);         // [16 warps][8]
-  int* red_i = reinterpret_cast<int*>(g_res_smem + 640);             // [16 warps][8]
+  float* red_f = reinterpret_cast<float*>(g_res_smem + 128);         // [32 warps][8]
+  int* red_i = reinterpret_cast<int*>(g_res_smem + 1152);            // [32 warps][8]
   uint8_t* xq = g_res_smem + p.x_off;                                // [Mpad][K], kernel order
   int* accs = reinterpret_cast<int*>(g_res_smem + p.acc_off);        // [rows][8] (wk > 1)
   uint8_t* wsm = g_res_smem + p.w_off;                               // [rows][K/4]
@@ -122,52 +130,44 @@ __global__ void __launch_bounds__(kResThreads, 2)
     return mx;
   };
   auto tok_of = [&](int pi) { return MM == 1 ? 0 : pi / Kh; };
-  if (keep) {
+  float sc[MM];
+  {
+    if (keep) {
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int pi = tid + i * kResThreads;
-      if (pi < npair) {
+      for (int i = 0; i < 2; ++i) {
+        const int pi = tid + i * kResThreads;
+        if (pi < npair) {
+          const int m = tok_of(pi);
+          kv[i] = *reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (pi - m * Kh) * 8);
+          const float mx = absmax8(kv[i]);
+#pragma unroll
+          for (int mm = 0; mm < MM; ++mm)
+            if (mm == m) am[mm] = fmaxf(am[mm], mx);
+        }
+      }
+    } else {
+      for (int pi = tid; pi < npair; pi += kResThreads) {
         const int m = tok_of(pi);
-        kv[i] = *reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (pi - m * Kh) * 8);
-        const float mx = absmax8(kv[i]);
+        const float mx =
+            absmax8(*reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (pi - m * Kh) * 8));
 #pragma unroll
         for (int mm = 0; mm < MM; ++mm)
           if (mm == m) am[mm] = fmaxf(am[mm], mx);
       }
     }
-  } else {
-    for (int pi = tid; pi < npair; pi += kResThreads) {
-      const int m = tok_of(pi);
-      const float mx =
-          absmax8(*reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (pi - m * Kh) * 8));
+    // warp maxima with one redux each (|x| >= 0, so the bit patterns order
+    // like the values), then every warp reduces the warp maxima the same way
 #pragma unroll
-      for (int mm = 0; mm < MM; ++mm)
-        if (mm == m) am[mm] = fmaxf(am[mm], mx);
+    for (int m = 0; m < MM; ++m) {
+      const uint32_t w = __reduce_max_sync(0xffffffffu, __float_as_uint(am[m]));
+      if (lane == 0 && m < M) red_f[warp * kResMaxTok + m] = __uint_as_float(w);
     }
-  }
-  // warp maxima with one redux each (|x| >= 0, so the bit patterns order
-  // like the values)
+    __syncthreads();
 #pragma unroll
-  for (int m = 0; m < MM; ++m) {
-    const uint32_t w = __reduce_max_sync(0xffffffffu, __float_as_uint(am[m]));
-    if (lane == 0 && m < M) red_f[warp * kResMaxTok + m] = __uint_as_float(w);
-  }
-  __syncthreads();
-  float sc[MM];
-#pragma unroll
-  for (int m = 0; m < MM; ++m) {
-    float a = 0.f;
-    if (m < M) {
-      float v[kResWarps];
-#pragma unroll
-      for (int w = 0; w < kResWarps; ++w) v[w] = red_f[w * kResMaxTok + m];
-#pragma unroll
-      for (int h = kResWarps / 2; h > 0; h >>= 1)
-#pragma unroll
-        for (int w = 0; w < h; ++w) v[w] = fmaxf(v[w], v[w + h]);
-      a = v[0];
+    for (int m = 0; m < MM; ++m) {
+      const uint32_t v = (m < M && lane < kResWarps) ? __float_as_uint(red_f[lane * kResMaxTok + m]) : 0u;
+      sc[m] = qscale(__uint_as_float(__reduce_max_sync(0xffffffffu, v)));
     }
-    sc[m] = qscale(a);
   }
   if (tid < M) {
     float s = sc[0];
@@ -228,12 +228,8 @@ __global__ void __launch_bounds__(kResThreads, 2)
   int rtot[MM];
 #pragma unroll
   for (int m = 0; m < MM; ++m) {
-    int t = 0;
-    if (m < M) {
-#pragma unroll
-      for (int w = 0; w < kResWarps; ++w) t += red_i[w * kResMaxTok + m];
-    }
-    rtot[m] = t;
+    const int v = (m < M && lane < kResWarps) ? red_i[lane * kResMaxTok + m] : 0;
+    rtot[m] = __reduce_add_sync(0xffffffffu, v);
   }
 
   // ---- products: items (4-row block b, K-slice q), dealt round robin to the
@@ -354,7 +350,7 @@ struct ResidentPlan {
 
 static uint32_t al128(uint64_t v) { return (uint32_t)((v + 127) & ~uint64_t(127)); }
 
-static bool plan_resident(int M, int N, int K, int num_sms, ResidentPlan* out) {
+static bool plan_resident(int M, int N, int K, int num_sms, int nw, ResidentPlan* out) {
   if (M < 1 || M > 3 || K % 64 != 0) return false;
   const int MT = M == 1 ? 1 : 2;
   const int Mpad = ((M + MT - 1) / MT) * MT;
@@ -368,7 +364,7 @@ static bool plan_resident(int M, int N, int K, int num_sms, ResidentPlan* out) {
   double best = 1e30;
   for (int c = 1; c <= 8; c *= 2) {
     if (c > 1 && Kw / c < 32) break;
-    const double rounds = (double)((nblk * c + kResWarps - 1) / kResWarps);
+    const double rounds = (double)((nblk * c + nw - 1) / nw);
     const double cost = rounds * ((double)((Kw / c + 31) / 32) + 2.0);
     if (cost < best - 1e-9) { best = cost; wk = c; }
   }
@@ -380,21 +376,21 @@ static bool plan_resident(int M, int N, int K, int num_sms, ResidentPlan* out) {
   p.acc_off = p.x_off + al128((uint64_t)Mpad * K);
   p.w_off = p.acc_off + (wk > 1 ? al128((uint64_t)nblk * 4 * kResMaxTok * 4) : 0u);
   const uint64_t total = (uint64_t)p.w_off + al128((uint64_t)nblk * 4 * (K / 4));
-  if (total > kResSmemMax) return false;
+  if (total > res_smem_max(nw)) return false;
   out->grid = grid;
   out->smem = (uint32_t)total;
   return true;
 }
 
-template <int MT, int MM>
+template <int MT, int MM, int NW>
 static cudaError_t launch_resident_t(const ResidentPlan& pl, cudaStream_t stream) {
   static std::atomic<uint64_t> configured{0};
-  cudaError_t e = set_smem_attr_once(configured, resident_kernel<MT, MM>, (int)kResSmemMax,
-                                     cudaSharedmemCarveoutMaxShared);
+  cudaError_t e = set_smem_attr_once(configured, resident_kernel<MT, MM, NW>,
+                                     (int)res_smem_max(NW), cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)pl.grid);
-  cfg.blockDim = dim3(kResThreads);
+  cfg.blockDim = dim3(NW * 32);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -402,29 +398,35 @@ static cudaError_t launch_resident_t(const ResidentPlan& pl, cudaStream_t stream
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, resident_kernel<MT, MM>, pl.p);
+  return cudaLaunchKernelEx(&cfg, resident_kernel<MT, MM, NW>, pl.p);
 }
 
 }  // namespace bitnet
 
 using namespace bitnet;
 
+// Warps per CTA of the resident kernel: 16, two CTAs per SM, so the next
+// layer's CTA loads its weights while this one computes (one CTA of 32 warps
+// per SM measured slower: 6.0 vs 3.4 us per 2B layer).
+constexpr int kResidentWarps = RESIDENT_WARPS;
+
 // Whether the resident kernel serves this BitLinear shape.
 bool bitnet_resident_fits(int64_t M, int64_t N, int64_t K, int num_sms) {
   if (M > 8 || N > 0x7fffffff || K > 0x7fffffff) return false;
   ResidentPlan pl;
-  return plan_resident((int)M, (int)N, (int)K, num_sms, &pl);
+  return plan_resident((int)M, (int)N, (int)K, num_sms, kResidentWarps, &pl);
 }
 
 bitnet_status bitnet_resident_launch(const uint8_t* w, const float* gamma, int N, int K,
                                      const uint16_t* x, int M, uint16_t* y, float* y_f32,
                                      int32_t* acc, int num_sms, cudaStream_t stream) {
+  constexpr int NW = kResidentWarps;
   ResidentPlan pl;
-  if (!plan_resident(M, N, K, num_sms, &pl)) return BITNET_ERR_UNSUPPORTED;
+  if (!plan_resident(M, N, K, num_sms, NW, &pl)) return BITNET_ERR_UNSUPPORTED;
   pl.p.w = w; pl.p.gamma = gamma; pl.p.x = x; pl.p.y = y; pl.p.y_f32 = y_f32; pl.p.acc = acc;
   cudaError_t e;
-  if (M == 1) e = launch_resident_t<1, 1>(pl, stream);
-  else if (M == 2) e = launch_resident_t<2, 2>(pl, stream);
-  else e = launch_resident_t<2, 4>(pl, stream);
+  if (M == 1) e = launch_resident_t<1, 1, NW>(pl, stream);
+  else if (M == 2) e = launch_resident_t<2, 2, NW>(pl, stream);
+  else e = launch_resident_t<2, 4, NW>(pl, stream);
   return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
