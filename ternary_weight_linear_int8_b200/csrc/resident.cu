@@ -52,6 +52,7 @@ constexpr uint32_t kResHead = 2176;     // barriers, token scalars, warp partial
 
 extern __shared__ __align__(128) uint8_t g_res_smem[];
 
+// MT: tokens per dp4a pass; MM: token count rounded up (loop bound); NW: warps.
 template <int MT, int MM, int NW>
 __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
     resident_kernel(const __grid_constant__ ResidentParams p) {
@@ -71,19 +72,20 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
   const int n0 = (int)(((int64_t)blockIdx.x * N) / gridDim.x);
   const int n1 = (int)(((int64_t)(blockIdx.x + 1) * N) / gridDim.x);
   const int R = n1 - n0;
-  const int nblk = (R + 3) >> 2;
+  constexpr int BR = 4;                // rows per block
+  const int nblk = (R + BR - 1) / BR;
   const int P = p.pieces;
-  const int cs = (nblk + P - 1) / P;   // 4-row blocks per piece
+  const int cs = (nblk + P - 1) / P;   // blocks per piece
 
-  // ---- weights: the whole slice, in P pieces of cs whole 4-row blocks
+  // ---- weights: the whole slice, in P pieces of cs whole row blocks
   if (tid == 0) {
     for (int i = 0; i < P; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
     pdl_launch_dependents();
     const uint64_t pol = policy_evict_first();
     for (int i = 0; i < P; ++i) {
-      const int r0 = min(R, 4 * i * cs);
-      const int r1 = min(R, 4 * (i + 1) * cs);
+      const int r0 = min(R, BR * i * cs);
+      const int r1 = min(R, BR * (i + 1) * cs);
       if (r1 <= r0) {            // empty piece: complete its phase at once
         mbar_arrive(&bars[i]);
         continue;
@@ -98,12 +100,13 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
       }
     }
   }
+  // dp4a passes read MT tokens at a time: the padding tokens are zero
   const int Mpad = ((M + MT - 1) / MT) * MT;
   for (int i = M * K + tid * 16; i < Mpad * K; i += kResThreads * 16)
     sts_v4(smem_u32(xq + i), make_uint4(0, 0, 0, 0));
   const int WK = p.wk;
   if (WK > 1)
-    for (int i = tid; i < nblk * 4 * kResMaxTok; i += kResThreads) accs[i] = 0;
+    for (int i = tid; i < nblk * BR * kResMaxTok; i += kResThreads) accs[i] = 0;
 
   pdl_wait();
 
@@ -246,12 +249,13 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
     if (p.y_f32) p.y_f32[o] = y32;
     if (p.acc) p.acc[o] = ac;
   };
-  constexpr int kUnroll = MT == 1 ? 4 : 2;
-  const int wkl = __ffs(WK) - 1;
-  const int nitems = nblk * WK;
   const uint32_t x_addr = smem_u32(xq), w_addr = smem_u32(wsm);
   bool ok = true;
   int pc = 0;            // weight piece of the current block (blocks only grow)
+  {
+  constexpr int kUnroll = MT == 1 ? 4 : 2;
+  const int wkl = __ffs(WK) - 1;
+  const int nitems = nblk * WK;
   for (int it = warp; it < nitems; it += kResWarps) {
     const int b = it >> wkl, qs = it & (WK - 1);
     while ((pc + 1) * cs <= b) ++pc;
@@ -326,6 +330,7 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
         }
       }
     }
+  }
   }
   if (WK > 1) {
     __syncthreads();
@@ -407,7 +412,9 @@ using namespace bitnet;
 
 // Warps per CTA of the resident kernel: 16, two CTAs per SM, so the next
 // layer's CTA loads its weights while this one computes (one CTA of 32 warps
-// per SM measured slower: 6.0 vs 3.4 us per 2B layer).
+// per SM measured slower: 6.0 vs 3.4 us per 2B layer).  The products are
+// dp4a items: warp-level int8 MMA items (16-row tiles) measured slower here,
+// 4.27 vs 2.94 us per 2B layer at one token and 6.36 vs 5.39 at two.
 constexpr int kResidentWarps = RESIDENT_WARPS;
 
 // Whether the resident kernel serves this BitLinear shape.
