@@ -276,21 +276,15 @@ def chain_calls(B, packs, x, bufs):
 
 
 class ChainCall:
-    """The chain as one bitnet_linear_chain call (outputs ping-pong in bufs)."""
+    """The chain as one bitnet_linear_chain call (outputs ping-pong in bufs),
+    through the binding's prepared chain (argument arrays built once)."""
 
     def __init__(self, B, torch, packs, bufs, dev):
-        self.B = B
-        self.P = [p for p, _ in packs]
-        self.G = [g for _, g in packs]
-        self.ys = [bufs[l % 2] for l in range(len(packs))]
-        M = bufs[0].shape[0]
-        nb = B.bitnet_linear_chain_workspace_size([p.shape[0] for p in self.P],
-                                                  [p.shape[1] * 4 for p in self.P], M)
-        self.ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+        self.prep = B.PreparedChain([p for p, _ in packs], [g for _, g in packs],
+                                    [bufs[l % 2] for l in range(len(packs))])
 
     def __call__(self, x):
-        self.B.bitnet_linear_chain(self.P, self.G, x, ys=self.ys, workspace=self.ws)
-        return self.ys[-1]
+        return self.prep(x)
 
 
 def capture(torch, fn, stream):
@@ -396,6 +390,44 @@ def secondary_measurements(B, inputs, torch, dev, stream, pk):
                                      "frac_hbm": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4),
                                      "us_per_step": round(t * 1e6, 1)}
         del g
+    # variants on the same 2B decode chain (M = 1), one launch per layer in a
+    # graph: BitNet v1 sign weights (1 bit each) and the pair-lookup-table
+    # inner loop on the ternary weights
+    x1 = torch.from_numpy(inputs.activations((1, HIDDEN), seed=0).view(np.int16)).to(dev)
+    bufs = [torch.empty((1, INTER), dtype=torch.bfloat16, device=dev),
+            torch.empty((1, HIDDEN), dtype=torch.bfloat16, device=dev)]
+    w1 = []
+    for l in range(2 * LAYERS):
+        N, K = (INTER, HIDDEN) if l % 2 == 0 else (HIDDEN, INTER)
+        W = torch.from_numpy(inputs.weights(N, K, seed=inputs.layer_seed(l))).to(dev)
+        w1.append(B.bitnet_pack_weights_w1(W))
+        del W
+    wsw = torch.empty(max(B.bitnet_linear_w1_workspace_size(1, INTER, HIDDEN),
+                          B.bitnet_linear_w1_workspace_size(1, HIDDEN, INTER)),
+                      dtype=torch.uint8, device=dev)
+
+    def run_w1():
+        cur = x1
+        for l, (p, a) in enumerate(w1):
+            B.bitnet_linear_w1(p, a, cur, y=bufs[l % 2], workspace=wsw)
+            cur = bufs[l % 2]
+
+    def run_tl2():
+        cur = x1
+        for l, (p, g) in enumerate(packs):
+            B.bitnet_linear_tl2(p, g, cur, y=bufs[l % 2])
+            cur = bufs[l % 2]
+    for name, fn, nbytes in (("decode_chain_w1_M1", run_w1, sum(p.numel() for p, _ in w1)),
+                             ("decode_chain_tl2_M1", run_tl2, sum(p.numel() for p, _ in packs))):
+        g = capture(torch, fn, stream)
+        ms, _, _ = time_graph(torch, g, stream, 50, 3)
+        t = ms / 50 * 1e-3
+        out[name] = {"GB/s": round(nbytes / t / 1e9, 1), "us_per_layer": round(t / 60 * 1e6, 3),
+                     "weights_per_s": round(2 * LAYERS * HIDDEN * INTER / t / 1e12, 3),
+                     "frac_hbm": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4),
+                     "bytes": "packed weights streamed per step (1 bit per weight for w1)"}
+        del g
+    del w1, wsw
     # FFN 100B-class: two distinct blocks rotated
     H, I = 8192, 28672
     blocks = []
@@ -560,7 +592,8 @@ def run_ours(args, world, rank, local):
            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
            "ms_per_step": e2e_ms,
            "how": "pinned host x -> device, one eager bitnet_linear_chain call (60 layers) "
-                  "through the Python binding, device -> pinned host y; CUDA events"}
+                  "through the Python binding's prepared chain, device -> pinned host y; "
+                  "CUDA events"}
 
     secondary = None
     if not args.no_secondary and rank == 0:

@@ -258,6 +258,64 @@ BITNET_API bitnet_status bitnet_linear_noalloc(const uint8_t* packed, const floa
                                                uint16_t* y, void* stream);
 
 /*
+ * BitNet v1 W1A8: sign weights, one bit each.
+ *   [Y] section "BitNet v1：BitLinearの誕生" > "1-Bit重みとSign関数"
+ *       (W_b = +1 where W >= 0, -1 where W < 0; alpha = mean |W_ij|; the
+ *       output is restored with alpha and the activation scale).
+ *
+ * bitnet_pack_weights_w1:
+ * W       [N,K] fp32, device, read only.  Must be finite.
+ * packed  [N,K/8] uint8, device, written: bit (k % 8) of byte n*K/8 + k/8 is
+ *         1 where W[n,k] >= 0 (including -0.0) and 0 where W[n,k] < 0.
+ * alpha   one fp32 on the device, written: the fp32 value nearest (ties to
+ *         even) to the exact mean of |W| (the same value bitnet_pack_weights
+ *         writes as gamma).
+ * workspace  >= bitnet_pack_w1_workspace_size(N, K) bytes.
+ * Requires K % 8 == 0, N >= 1, K >= 8, N*K < 2^39.  A non-finite weight sets
+ * alpha to NaN and records BITNET_ERR_NONFINITE.
+ *
+ * bitnet_linear_w1:  the activations are quantised exactly as in
+ * bitnet_linear (per token, s_t = 127 / max(max|x|, 1e-5)); then
+ *   acc[t,n] = sum_k xq[t,k] * W_b[n,k]   (exact int32)
+ *   y32      = fp32(acc) * (alpha / s_t);  y = bf16(y32), nearest even.
+ * (The page's v1 listing takes the absmax over the whole tensor; the library
+ * keeps its per-token quantiser, identical for one token.)
+ * Arguments as bitnet_linear, with packed [N,K/8] and alpha.
+ * workspace  >= bitnet_linear_w1_workspace_size(M, N, K) bytes.  With 1-3
+ * tokens, K % 128 == 0 and a per-SM slice that fits in shared memory the
+ * decode kernel reads the sign bits directly and the workspace is unused;
+ * otherwise the +-1 matrix is written into the workspace as I2_S codes
+ * (a +-1 matrix is a ternary one) and bitnet_linear's kernels run on it.
+ * Requires K % 8 == 0, K <= 524288.
+ */
+BITNET_API size_t bitnet_pack_w1_workspace_size(int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_pack_weights_w1(const float* W, int64_t N, int64_t K,
+                                                uint8_t* packed, float* alpha, void* workspace,
+                                                size_t workspace_bytes, void* stream);
+BITNET_API size_t bitnet_linear_w1_workspace_size(int64_t M, int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_linear_w1(const uint8_t* packed, const float* alpha, int64_t N,
+                                          int64_t K, const uint16_t* x, int64_t M, uint16_t* y,
+                                          float* y_f32, int32_t* acc, void* workspace,
+                                          size_t workspace_bytes, void* stream);
+
+/*
+ * BitLinear for one token through pair lookup tables instead of dp4a: the
+ * same result as bitnet_linear (same codes, accumulators and outputs).
+ *   [Y] section "I2_Sカーネルの内部動作" (TL2: two ternary weights, 3 x 3 = 9
+ *       combinations, index one table entry).
+ * For every activation pair (x_q[2i], x_q[2i+1]) a 16-entry table of
+ * x0 (c0 - 1) + x1 (c1 - 1) is built in shared memory, indexed by the packed
+ * nibble c0 + 4 c1 of two I2_S codes; a packed byte costs two lookups.
+ * x [1,K] bf16 bits; y [1,N]; y_f32, acc optional [1,N].  No workspace.
+ * Requires K % 64 == 0 and a per-SM slice of weights plus 16 K bytes of
+ * tables that fits in shared memory (else BITNET_ERR_UNSUPPORTED).  Kept as
+ * a measured alternative to the dp4a inner loop.
+ */
+BITNET_API bitnet_status bitnet_linear_tl2(const uint8_t* packed, const float* gamma, int64_t N,
+                                           int64_t K, const uint16_t* x, uint16_t* y,
+                                           float* y_f32, int32_t* acc, void* stream);
+
+/*
  * Synchronise `stream`, then return and clear the device status word of the
  * current device: BITNET_OK, BITNET_ERR_TIMEOUT (a bounded wait expired; the
  * affected outputs are unspecified) or BITNET_ERR_NONFINITE.  A failing

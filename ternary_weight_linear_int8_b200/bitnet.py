@@ -43,6 +43,11 @@ SIGNATURES = {
     "bitnet_linear_noalloc": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I64, _P, _P]),
     "bitnet_linear_chain_workspace_size": (_SZ, [_I64, _P, _P, _I64]),
     "bitnet_linear_chain": (ctypes.c_int, [_I64, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
+    "bitnet_pack_w1_workspace_size": (_SZ, [_I64, _I64]),
+    "bitnet_pack_weights_w1": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
+    "bitnet_linear_w1_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "bitnet_linear_w1": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I64, _P, _P, _P, _P, _SZ, _P]),
+    "bitnet_linear_tl2": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _P, _P, _P, _P]),
 }
 
 
@@ -278,6 +283,39 @@ def bitnet_linear_chain(packs, gammas, x: torch.Tensor, ys=None, workspace=None)
     return ys
 
 
+class PreparedChain:
+    """bitnet_linear_chain with its argument arrays and workspace built once:
+    calling it enqueues the whole chain with one C call (the layers' device
+    pointers, shapes and output buffers are fixed; only x and the stream
+    change from call to call)."""
+
+    def __init__(self, packs, gammas, ys, workspace=None):
+        if len(packs) != len(gammas) or len(packs) != len(ys) or not packs:
+            raise ValueError("packs, gammas and ys must be non-empty lists of equal length")
+        for p, g, y in zip(packs, gammas, ys):
+            _dev(p, "packed")
+            _dev(g, "gamma")
+            _bits16(y, "y")
+        self.M = ys[0].shape[0]
+        self.K0 = packs[0].shape[1] * 4
+        self._keep = (list(packs), list(gammas), list(ys))
+        self.L, self.Ns, self.Ks, self.P, self.G, self.Y = _host_arrays(packs, gammas, ys, None)
+        nb = lib().bitnet_linear_chain_workspace_size(self.L, self.Ns, self.Ks, self.M)
+        self.nb = nb
+        self.ws = _workspace(nb, ys[0].device, workspace)
+        self.ys = ys
+        self._fn = lib().bitnet_linear_chain
+        self._ws_ptr = _ptr(self.ws)
+
+    def __call__(self, x: torch.Tensor):
+        if x.shape[0] != self.M or x.shape[1] != self.K0:
+            raise ValueError("x does not match the prepared chain")
+        st = self._fn(self.L, self.P, self.G, self.Ns, self.Ks, ctypes.c_void_p(x.data_ptr()),
+                      self.M, self.Y, self._ws_ptr, self.nb, _stream())
+        _check("bitnet_linear_chain", st)
+        return self.ys[-1]
+
+
 def bitnet_linear_noalloc(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, y=None):
     """BitLinear using the library's fixed device scratch array instead of a
     workspace (for callers that cannot allocate).  Returns y bf16 [M,N]."""
@@ -293,6 +331,71 @@ def bitnet_linear_noalloc(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Te
                                      _stream())
     _check("bitnet_linear_noalloc", st)
     return y
+
+
+def bitnet_linear_w1_workspace_size(M: int, N: int, K: int) -> int:
+    return lib().bitnet_linear_w1_workspace_size(M, N, K)
+
+
+def bitnet_pack_weights_w1(W: torch.Tensor, packed=None, alpha=None, workspace=None):
+    """BitNet v1 sign weights: W fp32 [N,K] -> (packed uint8 [N,K/8], alpha fp32 [1])."""
+    _dev(W, "W")
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float32 tensor")
+    N, K = W.shape
+    packed = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device) if packed is None else packed
+    alpha = torch.empty(1, dtype=torch.float32, device=W.device) if alpha is None else alpha
+    nb = lib().bitnet_pack_w1_workspace_size(N, K)
+    ws = _workspace(nb, W.device, workspace)
+    st = lib().bitnet_pack_weights_w1(_ptr(W), N, K, _ptr(packed), _ptr(alpha), _ptr(ws), nb,
+                                      _stream())
+    _check("bitnet_pack_weights_w1", st)
+    return packed, alpha
+
+
+def bitnet_linear_w1(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, y=None,
+                     want_f32: bool = False, want_acc: bool = False, workspace=None,
+                     y_f32=None, acc=None):
+    """W1A8 BitLinear on sign-packed weights.  Returns (y bf16 [M,N], y_f32, acc)."""
+    _dev(packed, "packed")
+    _dev(alpha, "alpha")
+    _bits16(x, "x")
+    N, Kb = packed.shape
+    M, K = x.shape
+    if K != 8 * Kb:
+        raise ValueError("x and packed disagree on K")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    y32 = y_f32 if y_f32 is not None else (
+        torch.empty((M, N), dtype=torch.float32, device=x.device) if want_f32 else None)
+    acc = acc if acc is not None else (
+        torch.empty((M, N), dtype=torch.int32, device=x.device) if want_acc else None)
+    nb = lib().bitnet_linear_w1_workspace_size(M, N, K)
+    ws = _workspace(nb, x.device, workspace)
+    st = lib().bitnet_linear_w1(_ptr(packed), _ptr(alpha), N, K, _ptr(x), M, _ptr(y), _ptr(y32),
+                                _ptr(acc), _ptr(ws), nb, _stream())
+    _check("bitnet_linear_w1", st)
+    return y, y32, acc
+
+
+def bitnet_linear_tl2(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, y=None,
+                      want_f32: bool = False, want_acc: bool = False, y_f32=None, acc=None):
+    """One-token BitLinear through pair lookup tables (same result as bitnet_linear)."""
+    _dev(packed, "packed")
+    _dev(gamma, "gamma")
+    _bits16(x, "x")
+    N, Kb = packed.shape
+    M, K = x.shape
+    if M != 1 or K != 4 * Kb:
+        raise ValueError("x must be [1, K] with K = 4 * packed.shape[1]")
+    y = torch.empty((1, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    y32 = y_f32 if y_f32 is not None else (
+        torch.empty((1, N), dtype=torch.float32, device=x.device) if want_f32 else None)
+    acc = acc if acc is not None else (
+        torch.empty((1, N), dtype=torch.int32, device=x.device) if want_acc else None)
+    st = lib().bitnet_linear_tl2(_ptr(packed), _ptr(gamma), N, K, _ptr(x), _ptr(y), _ptr(y32),
+                                 _ptr(acc), _stream())
+    _check("bitnet_linear_tl2", st)
+    return y, y32, acc
 
 
 def bitnet_last_device_status() -> int:

@@ -16,10 +16,15 @@ bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* ga
                                   int32_t* rowsum, double* sumsq, int8_t* xq_natural,
                                   cudaStream_t stream);
 bitnet_status bitnet_decode_launch(const DecodeOp& op, int M, int num_sms, cudaStream_t stream);
-bool bitnet_resident_fits(int64_t M, int64_t N, int64_t K, int num_sms);
-bitnet_status bitnet_resident_launch(const uint8_t* w, const float* gamma, int N, int K,
+bool bitnet_resident_fits(int fmt, int64_t M, int64_t N, int64_t K, int num_sms);
+bitnet_status bitnet_resident_launch(int fmt, const uint8_t* w, const float* gamma, int N, int K,
                                      const uint16_t* x, int M, uint16_t* y, float* y_f32,
                                      int32_t* acc, int num_sms, cudaStream_t stream);
+bitnet_status bitnet_pack_w1_launch(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                                    float* alpha, void* workspace, cudaStream_t stream,
+                                    int num_sms);
+bitnet_status bitnet_sign_to_i2s_launch(const uint8_t* sign, int64_t nbytes, uint8_t* codes,
+                                        int num_sms, cudaStream_t stream);
 bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
                                  const uint8_t* w1, GemmArgs a, int bn, int num_sms,
                                  cudaStream_t stream);
@@ -246,8 +251,8 @@ bitnet_status linear_enqueue(const uint8_t* packed, const float* gamma, int64_t 
   bitnet_status st = BITNET_OK;
   const LinearPath p = linear_path(M, K);
   if (p == kPathGemv) {
-    if (bitnet_resident_fits(M, N, K, d.num_sms))
-      return bitnet_resident_launch(packed, gamma, (int)N, (int)K, x, (int)M, y, y_f32, acc,
+    if (bitnet_resident_fits(0, M, N, K, d.num_sms))
+      return bitnet_resident_launch(0, packed, gamma, (int)N, (int)K, x, (int)M, y, y_f32, acc,
                                     d.num_sms, s);
     DecodeOp a{};
     a.mode = kLinear;
@@ -465,6 +470,80 @@ bitnet_status bitnet_linear_chain(int64_t L, const uint8_t* const* packed,
     if (st != BITNET_OK) return st;
   }
   return BITNET_OK;
+}
+
+size_t bitnet_pack_w1_workspace_size(int64_t N, int64_t K) {
+  (void)N;
+  (void)K;
+  return bitnet_pack_workspace_size_impl();
+}
+
+bitnet_status bitnet_pack_weights_w1(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                                     float* alpha, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  if (!W || !packed || !alpha) return BITNET_ERR_INVALID_ARG;
+  if (N < 1 || K < 8 || K % 8 != 0 || N > (int64_t(1) << 39) / K) return BITNET_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(packed) || ((uintptr_t)alpha & 3u)) return BITNET_ERR_ALIGN;
+  if (!workspace || workspace_bytes < bitnet_pack_w1_workspace_size(N, K))
+    return BITNET_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  return bitnet_pack_w1_launch(W, N, K, packed, alpha, workspace, as_stream(stream), d.num_sms);
+}
+
+size_t bitnet_linear_w1_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 8) return 0;
+  return al256((size_t)N * (size_t)(K / 4)) + linear_ws_layout(M, N, K).total;
+}
+
+bitnet_status bitnet_linear_w1(const uint8_t* packed, const float* alpha, int64_t N, int64_t K,
+                               const uint16_t* x, int64_t M, uint16_t* y, float* y_f32,
+                               int32_t* acc, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (!packed || !alpha || !x || !y) return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 8 || K % 8 != 0 || K > 524288 || M > 0x7fffffff || N > 0x7fffffff)
+    return BITNET_ERR_SHAPE;
+  if (!aligned16(packed) || !aligned16(x) || !aligned16(y) || ((uintptr_t)alpha & 3u) ||
+      ((uintptr_t)y_f32 & 3u) || ((uintptr_t)acc & 3u))
+    return BITNET_ERR_ALIGN;
+  const size_t need = bitnet_linear_w1_workspace_size(M, N, K);
+  if (!workspace || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  // one to three tokens, packed rows a multiple of 16 bytes: the decode kernel
+  // on the sign bits themselves
+  if (K % 128 == 0 && bitnet_resident_fits(1, M, N, K, d.num_sms))
+    return bitnet_resident_launch(1, packed, alpha, (int)N, (int)K, x, (int)M, y, y_f32, acc,
+                                  d.num_sms, s);
+  // otherwise the same +-1 matrix as ternary I2_S codes, then BitLinear with
+  // gamma = alpha
+  uint8_t* codes = static_cast<uint8_t*>(workspace);
+  st = bitnet_sign_to_i2s_launch(packed, N * (K / 8), codes, d.num_sms, s);
+  if (st != BITNET_OK) return st;
+  const LinearWs L = linear_ws_layout(M, N, K);
+  return linear_enqueue(codes, alpha, N, K, x, M, y, y_f32, acc,
+                        codes + al256((size_t)N * (size_t)(K / 4)), L, d, s);
+}
+
+bitnet_status bitnet_linear_tl2(const uint8_t* packed, const float* gamma, int64_t N, int64_t K,
+                                const uint16_t* x, uint16_t* y, float* y_f32, int32_t* acc,
+                                void* stream) {
+  if (!packed || !gamma || !x || !y) return BITNET_ERR_INVALID_ARG;
+  if (N < 1 || K < 64 || K % 64 != 0 || K > 524288 || N > 0x7fffffff) return BITNET_ERR_SHAPE;
+  if (!aligned16(packed) || !aligned16(x) || !aligned16(y) || ((uintptr_t)gamma & 3u) ||
+      ((uintptr_t)y_f32 & 3u) || ((uintptr_t)acc & 3u))
+    return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  if (!bitnet_resident_fits(2, 1, N, K, d.num_sms)) return BITNET_ERR_UNSUPPORTED;
+  return bitnet_resident_launch(2, packed, gamma, (int)N, (int)K, x, 1, y, y_f32, acc, d.num_sms,
+                                as_stream(stream));
 }
 
 bitnet_status bitnet_last_device_status(void* stream) {

@@ -173,11 +173,72 @@ __global__ void __launch_bounds__(256) ternary_pack_kernel(const float4* __restr
   }
 }
 
+// BitNet v1 sign weights (youngju.dev page, section "BitNet v1：BitLinearの誕生"
+// > "1-Bit重みとSign関数": W_b = +1 where W >= 0, -1 where W < 0): one output
+// byte (eight weights along K, bit i for weight 8j + i, 1 for +1) per thread.
+__global__ void __launch_bounds__(256) sign_pack_kernel(const float4* __restrict__ W,
+                                                         int64_t nbytes,
+                                                         uint8_t* __restrict__ packed) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nbytes;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = __ldcs(&W[2 * i]), b = __ldcs(&W[2 * i + 1]);
+    const float e8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t byte = 0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) byte |= (e8[c] >= 0.0f ? 1u : 0u) << c;
+    packed[i] = (uint8_t)byte;
+  }
+}
+
+// Sign bits -> I2_S codes of the same +-1 matrix (a +-1 matrix is a ternary
+// one): bit 1 -> code 10 (+1), bit 0 -> code 00 (-1).  One sign byte becomes
+// two code bytes.
+__global__ void __launch_bounds__(256) sign_to_i2s_kernel(const uint8_t* __restrict__ sign,
+                                                           int64_t nbytes,
+                                                           uint8_t* __restrict__ codes) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nbytes;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint32_t v = sign[i];
+    uint32_t out = 0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) out |= ((v >> c) & 1u) << (2 * c + 1);
+    codes[2 * i] = (uint8_t)(out & 0xffu);
+    codes[2 * i + 1] = (uint8_t)(out >> 8);
+  }
+}
+
 }  // namespace bitnet
 
 using namespace bitnet;
 
 size_t bitnet_pack_workspace_size_impl() { return 4096; }
+
+bitnet_status bitnet_pack_w1_launch(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                                    float* alpha, void* workspace, cudaStream_t stream,
+                                    int num_sms) {
+  PackWs* ws = reinterpret_cast<PackWs*>(workspace);
+  if (cudaMemsetAsync(ws, 0, sizeof(PackWs), stream) != cudaSuccess) return BITNET_ERR_CUDA;
+  const int64_t total = N * K;
+  const int64_t n4 = total / 4;
+  int grid = num_sms * 4;
+  const int64_t need = (n4 + 255) / 256;
+  if (need < grid) grid = (int)(need > 0 ? need : 1);
+  // alpha = mean |W|: the same exact mean as gamma
+  gamma_bucket_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(W), n4, ws);
+  gamma_finalize_kernel<<<1, 32, 0, stream>>>(ws, (unsigned long long)total, alpha);
+  sign_pack_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(W), total / 8,
+                                             packed);
+  return cudaGetLastError() == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
+
+bitnet_status bitnet_sign_to_i2s_launch(const uint8_t* sign, int64_t nbytes, uint8_t* codes,
+                                        int num_sms, cudaStream_t stream) {
+  int grid = num_sms * 4;
+  const int64_t need = (nbytes + 255) / 256;
+  if (need < grid) grid = (int)(need > 0 ? need : 1);
+  sign_to_i2s_kernel<<<grid, 256, 0, stream>>>(sign, nbytes, codes);
+  return cudaGetLastError() == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
 
 bitnet_status bitnet_pack_launch(const float* W, int64_t N, int64_t K, uint8_t* packed,
                                  float* gamma, void* workspace, cudaStream_t stream,

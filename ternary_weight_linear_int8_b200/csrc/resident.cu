@@ -18,17 +18,31 @@
 // dependent sequence remains: activation loads, per-token absmax and
 // quantisation into shared memory, the products from shared memory and the
 // dequantised stores.
+//
+// Two more weight formats share the schedule (template parameter FMT):
+//  * kResW1 -- BitNet v1 sign weights, one bit each (youngju.dev page,
+//    section "BitNet v1：BitLinearの誕生" > "1-Bit重みとSign関数"): bit 1 for
+//    +1, 0 for -1, 8 weights per byte along K, least significant bit first.
+//    Plane p of a 32-bit word, (w >> p) & 0x01010101, holds in byte b the bit
+//    of k = 32j + 8b + p, and the activations sit in the matching order (in
+//    each group of 32, slot 4p + b holds k = 8b + p), so dp4a gives the sum
+//    of x over the +1 weights, S; then x . W_b = 2 S - sum x.
+//  * kResTL2 -- the ternary I2_S weights through pair lookup tables instead
+//    of dp4a (the TL2 idea of the youngju.dev page, section
+//    "I2_Sカーネルの内部動作": two ternary weights index one table entry).  For
+//    every activation pair (x0, x1) = (x_q[2i], x_q[2i+1]) a 16-entry table
+//    holds x0 (c0 - 1) + x1 (c1 - 1) at c0 + 4 c1; a packed nibble is exactly
+//    that index, so a byte costs two lookups.  One token; one CTA per SM (the
+//    tables take 16 K bytes).
 #include "common.cuh"
-
-#ifndef RESIDENT_WARPS
-#define RESIDENT_WARPS 16
-#endif
 
 namespace bitnet {
 
+enum ResFmt : int { kResI2S = 0, kResW1 = 1, kResTL2 = 2 };
+
 struct ResidentParams {
-  const uint8_t* w;        // packed [N, K/4]
-  const float* gamma;
+  const uint8_t* w;        // packed [N, K/4] (I2_S) or [N, K/8] (sign bits)
+  const float* gamma;      // gamma (I2_S) or alpha (sign weights)
   const uint16_t* x;       // bf16 [M, K]
   uint16_t* y;             // bf16 [M, N]
   float* y_f32;            // optional [M, N]
@@ -37,63 +51,63 @@ struct ResidentParams {
   int wk;                  // K-slices per 4-row block (1, 2, 4 or 8)
   int pieces;              // weight copy groups (1..4), one mbarrier each
   uint32_t x_off;          // shared-memory offsets (bytes, multiples of 128)
+  uint32_t lut_off;        // pair tables (kResTL2)
   uint32_t acc_off;
   uint32_t w_off;
 };
 
+constexpr int kResWarps = 16;
+constexpr int kResThreads = kResWarps * 32;
 constexpr int kResMaxTok = 8;
-constexpr int kResMaxWarps = 32;
-// 16 warps: two CTAs per SM (228 KB of shared memory per SM, 1 KB reserved
-// per CTA); 32 warps: one CTA per SM
-__host__ __device__ constexpr uint32_t res_smem_max(int nw) {
-  return nw == 16 ? 112u * 1024u : 200u * 1024u;
+// two CTAs per SM: 228 KB of shared memory per SM, 1 KB reserved per CTA;
+// the pair tables need one CTA per SM
+__host__ __device__ constexpr uint32_t res_smem_max(int fmt) {
+  return fmt == kResTL2 ? 200u * 1024u : 112u * 1024u;
 }
-constexpr uint32_t kResHead = 2176;     // barriers, token scalars, warp partials
+constexpr uint32_t kResHead = 1152;     // barriers, token scalars, warp partials
 
 extern __shared__ __align__(128) uint8_t g_res_smem[];
 
-// MT: tokens per dp4a pass; MM: token count rounded up (loop bound); NW: warps.
-template <int MT, int MM, int NW>
-__global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
+// MT: tokens per dp4a pass; MM: token count rounded up (loop bound).
+template <int FMT, int MT, int MM>
+__global__ void __launch_bounds__(kResThreads, FMT == kResTL2 ? 1 : 2)
     resident_kernel(const __grid_constant__ ResidentParams p) {
-  constexpr int kResWarps = NW;
-  constexpr int kResThreads = NW * 32;
   uint64_t* bars = reinterpret_cast<uint64_t*>(g_res_smem);          // [4]
   float* tok_d = reinterpret_cast<float*>(g_res_smem + 64);          // [8]
-  float* red_f = reinterpret_cast<float*>(g_res_smem + 128);         // [32 warps][8]
-  int* red_i = reinterpret_cast<int*>(g_res_smem + 1152);            // [32 warps][8]
-  uint8_t* xq = g_res_smem + p.x_off;                                // [Mpad][K], kernel order
+  float* red_f = reinterpret_cast<float*>(g_res_smem + 128);         // [16 warps][8]
+  int* red_i = reinterpret_cast<int*>(g_res_smem + 640);             // [16 warps][8]
+  uint8_t* xq = g_res_smem + p.x_off;                                // [Mpad][K]
   int* accs = reinterpret_cast<int*>(g_res_smem + p.acc_off);        // [rows][8] (wk > 1)
-  uint8_t* wsm = g_res_smem + p.w_off;                               // [rows][K/4]
+  uint8_t* wsm = g_res_smem + p.w_off;                               // [rows][Rb]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int K = p.K, N = p.N, M = p.M;
-  const int Kb = K >> 2, Kw = K >> 4;
+  const int Rb = FMT == kResW1 ? K >> 3 : K >> 2;   // packed bytes per row
+  const int Ww = FMT == kResW1 ? K >> 5 : K >> 4;   // 32-bit words per row
   const int n0 = (int)(((int64_t)blockIdx.x * N) / gridDim.x);
   const int n1 = (int)(((int64_t)(blockIdx.x + 1) * N) / gridDim.x);
   const int R = n1 - n0;
-  constexpr int BR = 4;                // rows per block
-  const int nblk = (R + BR - 1) / BR;
+  const int nblk = (R + 3) >> 2;       // 4-row blocks
   const int P = p.pieces;
   const int cs = (nblk + P - 1) / P;   // blocks per piece
 
-  // ---- weights: the whole slice, in P pieces of cs whole row blocks
+  // ---- weights: the whole slice, in P pieces of cs whole 4-row blocks
   if (tid == 0) {
     for (int i = 0; i < P; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
     pdl_launch_dependents();
     const uint64_t pol = policy_evict_first();
     for (int i = 0; i < P; ++i) {
-      const int r0 = min(R, BR * i * cs);
-      const int r1 = min(R, BR * (i + 1) * cs);
+      const int r0 = min(R, 4 * i * cs);
+      const int r1 = min(R, 4 * (i + 1) * cs);
       if (r1 <= r0) {            // empty piece: complete its phase at once
         mbar_arrive(&bars[i]);
         continue;
       }
-      const uint32_t bytes = (uint32_t)(r1 - r0) * (uint32_t)Kb;
+      const uint32_t bytes = (uint32_t)(r1 - r0) * (uint32_t)Rb;
       mbar_arrive_expect_tx(&bars[i], bytes);
-      const uint8_t* src = p.w + (int64_t)(n0 + r0) * Kb;
-      uint8_t* dst = wsm + (size_t)r0 * Kb;
+      const uint8_t* src = p.w + (int64_t)(n0 + r0) * Rb;
+      uint8_t* dst = wsm + (size_t)r0 * Rb;
       for (uint32_t off = 0; off < bytes; off += 4096u) {
         const uint32_t nb = bytes - off < 4096u ? bytes - off : 4096u;
         bulk_g2s(dst + off, src + off, nb, &bars[i], pol);
@@ -106,7 +120,7 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
     sts_v4(smem_u32(xq + i), make_uint4(0, 0, 0, 0));
   const int WK = p.wk;
   if (WK > 1)
-    for (int i = tid; i < nblk * BR * kResMaxTok; i += kResThreads) accs[i] = 0;
+    for (int i = tid; i < nblk * 4 * kResMaxTok; i += kResThreads) accs[i] = 0;
 
   pdl_wait();
 
@@ -115,7 +129,7 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
   // registers between the passes, otherwise pass 2 loads them again.
   float gam = 0.f;
   if (tid < M) gam = *p.gamma;
-  const int Kh = Kw * 2;                 // 8-value pieces per token
+  const int Kh = K >> 3;                 // 8-value pieces per token
   const int npair = M * Kh;
   const bool keep = npair <= 2 * kResThreads;
   uint4 kv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
@@ -133,44 +147,43 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
     return mx;
   };
   auto tok_of = [&](int pi) { return MM == 1 ? 0 : pi / Kh; };
-  float sc[MM];
-  {
-    if (keep) {
+  if (keep) {
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int pi = tid + i * kResThreads;
-        if (pi < npair) {
-          const int m = tok_of(pi);
-          kv[i] = *reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (pi - m * Kh) * 8);
-          const float mx = absmax8(kv[i]);
-#pragma unroll
-          for (int mm = 0; mm < MM; ++mm)
-            if (mm == m) am[mm] = fmaxf(am[mm], mx);
-        }
-      }
-    } else {
-      for (int pi = tid; pi < npair; pi += kResThreads) {
+    for (int i = 0; i < 2; ++i) {
+      const int pi = tid + i * kResThreads;
+      if (pi < npair) {
         const int m = tok_of(pi);
-        const float mx =
-            absmax8(*reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (pi - m * Kh) * 8));
+        kv[i] = *reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (pi - m * Kh) * 8);
+        const float mx = absmax8(kv[i]);
 #pragma unroll
         for (int mm = 0; mm < MM; ++mm)
           if (mm == m) am[mm] = fmaxf(am[mm], mx);
       }
     }
-    // warp maxima with one redux each (|x| >= 0, so the bit patterns order
-    // like the values), then every warp reduces the warp maxima the same way
+  } else {
+    for (int pi = tid; pi < npair; pi += kResThreads) {
+      const int m = tok_of(pi);
+      const float mx =
+          absmax8(*reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + (pi - m * Kh) * 8));
 #pragma unroll
-    for (int m = 0; m < MM; ++m) {
-      const uint32_t w = __reduce_max_sync(0xffffffffu, __float_as_uint(am[m]));
-      if (lane == 0 && m < M) red_f[warp * kResMaxTok + m] = __uint_as_float(w);
+      for (int mm = 0; mm < MM; ++mm)
+        if (mm == m) am[mm] = fmaxf(am[mm], mx);
     }
-    __syncthreads();
+  }
+  // warp maxima with one redux each (|x| >= 0, so the bit patterns order
+  // like the values), then every warp reduces the warp maxima the same way
 #pragma unroll
-    for (int m = 0; m < MM; ++m) {
-      const uint32_t v = (m < M && lane < kResWarps) ? __float_as_uint(red_f[lane * kResMaxTok + m]) : 0u;
-      sc[m] = qscale(__uint_as_float(__reduce_max_sync(0xffffffffu, v)));
-    }
+  for (int m = 0; m < MM; ++m) {
+    const uint32_t w = __reduce_max_sync(0xffffffffu, __float_as_uint(am[m]));
+    if (lane == 0 && m < M) red_f[warp * kResMaxTok + m] = __uint_as_float(w);
+  }
+  __syncthreads();
+  float sc[MM];
+#pragma unroll
+  for (int m = 0; m < MM; ++m) {
+    const uint32_t v =
+        (m < M && lane < kResWarps) ? __float_as_uint(red_f[lane * kResMaxTok + m]) : 0u;
+    sc[m] = qscale(__uint_as_float(__reduce_max_sync(0xffffffffu, v)));
   }
   if (tid < M) {
     float s = sc[0];
@@ -182,8 +195,6 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
   int rs[MM];
 #pragma unroll
   for (int m = 0; m < MM; ++m) rs[m] = 0;
-  // 8 values k = 16g + 8h + i (i = 0..7) land at slots 4(i%4) + 2h + i/4 of
-  // group g: per code plane t one 16-bit half (values t and t + 4)
   auto quant8 = [&](int pi, const uint4& v) {
     const int m = tok_of(pi), hg = pi - m * Kh;
     float s = sc[0];
@@ -197,13 +208,29 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
       q[2 * i] = quant_code_sat(__uint_as_float(w[i] << 16), s);
       q[2 * i + 1] = quant_code_sat(__uint_as_float(w[i] & 0xffff0000u), s);
     }
-    const uint32_t base =
-        smem_u32(xq) + (uint32_t)(m * K + (hg >> 1) * 16 + 2 * (hg & 1));
     int sum = 0;
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      sts_u16(base + 4 * t, (uint16_t)__byte_perm((uint32_t)q[t], (uint32_t)q[4 + t], 0x0040));
-      sum += q[t] + q[4 + t];
+    for (int i = 0; i < 8; ++i) sum += q[i];
+    const uint32_t row = smem_u32(xq) + (uint32_t)(m * K);
+    if constexpr (FMT == kResI2S) {
+      // k = 16g + 8h + i lands at slot 4 (i % 4) + 2h + i / 4 of group g: per
+      // code plane t one 16-bit half (values t and t + 4)
+      const uint32_t base = row + (uint32_t)((hg >> 1) * 16 + 2 * (hg & 1));
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        sts_u16(base + 4 * t, (uint16_t)__byte_perm((uint32_t)q[t], (uint32_t)q[4 + t], 0x0040));
+    } else if constexpr (FMT == kResW1) {
+      // k = 32G + 8h + i lands at slot 4i + h of group G
+      const uint32_t base = row + (uint32_t)((hg >> 2) * 32 + (hg & 3));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sts_u8(base + 4 * i, (uint8_t)q[i]);
+    } else {
+      // natural order (the pair tables are built from it)
+      const uint32_t lo = __byte_perm(__byte_perm((uint32_t)q[0], (uint32_t)q[1], 0x0040),
+                                      __byte_perm((uint32_t)q[2], (uint32_t)q[3], 0x0040), 0x5410);
+      const uint32_t hi = __byte_perm(__byte_perm((uint32_t)q[4], (uint32_t)q[5], 0x0040),
+                                      __byte_perm((uint32_t)q[6], (uint32_t)q[7], 0x0040), 0x5410);
+      sts_v2(row + (uint32_t)(hg * 8), lo, hi);
     }
 #pragma unroll
     for (int mm = 0; mm < MM; ++mm)
@@ -227,6 +254,28 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
     if (lane == 0 && m < M) red_i[warp * kResMaxTok + m] = t;
   }
   __syncthreads();
+  if constexpr (FMT == kResTL2) {
+    // pair tables: entry c0 + 4 c1 of pair i is x0 (c0 - 1) + x1 (c1 - 1)
+    // (code 3 never occurs; its entries are 0); 16 int16 = 32 bytes a pair
+    const uint32_t lut = smem_u32(g_res_smem + p.lut_off);
+    for (int pr = tid; pr < (K >> 1); pr += kResThreads) {
+      const int x0 = (int)(int8_t)xq[2 * pr], x1 = (int)(int8_t)xq[2 * pr + 1];
+      uint32_t e[8];
+#pragma unroll
+      for (int w2 = 0; w2 < 8; ++w2) {
+        int v2[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int idx = 2 * w2 + h, c0 = idx & 3, c1 = idx >> 2;
+          v2[h] = (c0 == 3 || c1 == 3) ? 0 : x0 * (c0 - 1) + x1 * (c1 - 1);
+        }
+        e[w2] = ((uint32_t)v2[0] & 0xffffu) | ((uint32_t)v2[1] << 16);
+      }
+      sts_v4(lut + 32u * pr, make_uint4(e[0], e[1], e[2], e[3]));
+      sts_v4(lut + 32u * pr + 16u, make_uint4(e[4], e[5], e[6], e[7]));
+    }
+    __syncthreads();
+  }
   // each token's row sum (identical in every thread)
   int rtot[MM];
 #pragma unroll
@@ -242,7 +291,7 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
 #pragma unroll
     for (int mm = 1; mm < MM; ++mm)
       if (mm == m) rsum = rtot[mm];
-    const int ac = v - rsum;
+    const int ac = FMT == kResTL2 ? v : (FMT == kResW1 ? 2 * v - rsum : v - rsum);
     const float y32 = __fmul_rn(__int2float_rn(ac), tok_d[m]);
     const int64_t o = (int64_t)m * N + n0 + r;
     p.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
@@ -250,20 +299,20 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
     if (p.acc) p.acc[o] = ac;
   };
   const uint32_t x_addr = smem_u32(xq), w_addr = smem_u32(wsm);
+  const uint32_t lut_addr = smem_u32(g_res_smem + p.lut_off);
   bool ok = true;
   int pc = 0;            // weight piece of the current block (blocks only grow)
-  {
-  constexpr int kUnroll = MT == 1 ? 4 : 2;
+  constexpr int kUnroll = (MT == 1 && FMT == kResI2S) ? 4 : 2;
   const int wkl = __ffs(WK) - 1;
   const int nitems = nblk * WK;
   for (int it = warp; it < nitems; it += kResWarps) {
     const int b = it >> wkl, qs = it & (WK - 1);
     while ((pc + 1) * cs <= b) ++pc;
     if (!mbar_wait(&bars[pc], 0)) { ok = false; break; }
-    const int j0 = (qs * Kw) >> wkl, j1 = ((qs + 1) * Kw) >> wkl;
+    const int j0 = (qs * Ww) >> wkl, j1 = ((qs + 1) * Ww) >> wkl;
     uint32_t rowa[4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) rowa[r] = w_addr + (uint32_t)(min(4 * b + r, R - 1) * Kb);
+    for (int r = 0; r < 4; ++r) rowa[r] = w_addr + (uint32_t)(min(4 * b + r, R - 1) * Rb);
     for (int tg = 0; tg < M; tg += MT) {
       int acc_r[4][MT];
       int acc4[4][4];
@@ -280,34 +329,66 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
         uint32_t w[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) w[r] = lds_u32(rowa[r] + 4u * j);
-        uint4 xv[MT];
+        if constexpr (FMT == kResI2S) {
+          uint4 xv[MT];
 #pragma unroll
-        for (int t = 0; t < MT; ++t) xv[t] = lds_v4(xt + (uint32_t)(t * K) + 16u * j);
+          for (int t = 0; t < MT; ++t) xv[t] = lds_v4(xt + (uint32_t)(t * K) + 16u * j);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          if constexpr (MT == 1) {
-            acc4[r][0] = dp4a_su((int)xv[0].x, w[r] & 0x03030303u, acc4[r][0]);
-            acc4[r][1] = dp4a_su((int)xv[0].y, w[r] & 0x0c0c0c0cu, acc4[r][1]);
-            acc4[r][2] = dp4a_su((int)xv[0].z, w[r] & 0x30303030u, acc4[r][2]);
-            acc4[r][3] = dp4a_su((int)xv[0].w, w[r] & 0xc0c0c0c0u, acc4[r][3]);
-          } else {
-            const uint32_t c0 = w[r] & 0x03030303u;
-            const uint32_t c1 = (w[r] >> 2) & 0x03030303u;
-            const uint32_t c2 = (w[r] >> 4) & 0x03030303u;
-            const uint32_t c3 = (w[r] >> 6) & 0x03030303u;
+          for (int r = 0; r < 4; ++r) {
+            if constexpr (MT == 1) {
+              acc4[r][0] = dp4a_su((int)xv[0].x, w[r] & 0x03030303u, acc4[r][0]);
+              acc4[r][1] = dp4a_su((int)xv[0].y, w[r] & 0x0c0c0c0cu, acc4[r][1]);
+              acc4[r][2] = dp4a_su((int)xv[0].z, w[r] & 0x30303030u, acc4[r][2]);
+              acc4[r][3] = dp4a_su((int)xv[0].w, w[r] & 0xc0c0c0c0u, acc4[r][3]);
+            } else {
+              const uint32_t c0 = w[r] & 0x03030303u;
+              const uint32_t c1 = (w[r] >> 2) & 0x03030303u;
+              const uint32_t c2 = (w[r] >> 4) & 0x03030303u;
+              const uint32_t c3 = (w[r] >> 6) & 0x03030303u;
 #pragma unroll
-            for (int t = 0; t < MT; ++t) {
+              for (int t = 0; t < MT; ++t) {
+                int v = acc_r[r][t];
+                v = dp4a_su((int)xv[t].x, c0, v);
+                v = dp4a_su((int)xv[t].y, c1, v);
+                v = dp4a_su((int)xv[t].z, c2, v);
+                v = dp4a_su((int)xv[t].w, c3, v);
+                acc_r[r][t] = v;
+              }
+            }
+          }
+        } else if constexpr (FMT == kResW1) {
+          // 32 activations per word: planes p = 0..7 against words p of the group
+#pragma unroll
+          for (int t = 0; t < MT; ++t) {
+            const uint4 xa = lds_v4(xt + (uint32_t)(t * K) + 32u * j);
+            const uint4 xb = lds_v4(xt + (uint32_t)(t * K) + 32u * j + 16u);
+            const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
               int v = acc_r[r][t];
-              v = dp4a_su((int)xv[t].x, c0, v);
-              v = dp4a_su((int)xv[t].y, c1, v);
-              v = dp4a_su((int)xv[t].z, c2, v);
-              v = dp4a_su((int)xv[t].w, c3, v);
+#pragma unroll
+              for (int pl = 0; pl < 8; ++pl)
+                v = dp4a_su((int)xw[pl], (w[r] >> pl) & 0x01010101u, v);
               acc_r[r][t] = v;
             }
           }
+        } else {
+          // pair tables: byte q of the word holds pairs 2q (low nibble) and
+          // 2q + 1 (high nibble) of this word's 8 pairs
+          const uint32_t tb = lut_addr + 256u * (uint32_t)j;
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            int v = acc_r[r][0];
+#pragma unroll
+            for (int q2 = 0; q2 < 8; ++q2) {
+              const uint32_t nib = (w[r] >> (4 * q2)) & 15u;
+              v += lds_s16(tb + 32u * q2 + 2u * nib);
+            }
+            acc_r[r][0] = v;
+          }
         }
       }
-      if constexpr (MT == 1) {
+      if constexpr (MT == 1 && FMT == kResI2S) {
 #pragma unroll
         for (int r = 0; r < 4; ++r)
           acc_r[r][0] = acc4[r][0] + (acc4[r][1] >> 2) + (acc4[r][2] >> 4) + (acc4[r][3] >> 6);
@@ -330,7 +411,6 @@ __global__ void __launch_bounds__(NW * 32, NW == 16 ? 2 : 1)
         }
       }
     }
-  }
   }
   if (WK > 1) {
     __syncthreads();
@@ -355,22 +435,24 @@ struct ResidentPlan {
 
 static uint32_t al128(uint64_t v) { return (uint32_t)((v + 127) & ~uint64_t(127)); }
 
-static bool plan_resident(int M, int N, int K, int num_sms, int nw, ResidentPlan* out) {
-  if (M < 1 || M > 3 || K % 64 != 0) return false;
+static bool plan_resident(int fmt, int M, int N, int K, int num_sms, ResidentPlan* out) {
+  if (M < 1 || M > (fmt == kResTL2 ? 1 : 3) || K % 64 != 0 || N < 1) return false;
+  if (fmt == kResW1 && K % 128 != 0) return false;   // 16-byte packed rows
   const int MT = M == 1 ? 1 : 2;
   const int Mpad = ((M + MT - 1) / MT) * MT;
   const int grid = (N + 3) / 4 < num_sms ? (N + 3) / 4 : num_sms;
   const int rows_max = (N + grid - 1) / grid;
   const int nblk = (rows_max + 3) / 4;
-  const int Kw = K / 16;
+  const int Ww = fmt == kResW1 ? K / 32 : K / 16;
+  const int Rb = fmt == kResW1 ? K / 8 : K / 4;
   // K-slices: rounds of items over the warps x (32-word steps + a fixed
   // per-item cost of about two steps)
   int wk = 1;
   double best = 1e30;
   for (int c = 1; c <= 8; c *= 2) {
-    if (c > 1 && Kw / c < 32) break;
-    const double rounds = (double)((nblk * c + nw - 1) / nw);
-    const double cost = rounds * ((double)((Kw / c + 31) / 32) + 2.0);
+    if (c > 1 && Ww / c < 32) break;
+    const double rounds = (double)((nblk * c + kResWarps - 1) / kResWarps);
+    const double cost = rounds * ((double)((Ww / c + 31) / 32) + 2.0);
     if (cost < best - 1e-9) { best = cost; wk = c; }
   }
   ResidentParams& p = out->p;
@@ -378,24 +460,25 @@ static bool plan_resident(int M, int N, int K, int num_sms, int nw, ResidentPlan
   p.N = N; p.K = K; p.M = M; p.wk = wk;
   p.pieces = nblk < 4 ? nblk : 4;
   p.x_off = kResHead;
-  p.acc_off = p.x_off + al128((uint64_t)Mpad * K);
+  p.lut_off = p.x_off + al128((uint64_t)Mpad * K);
+  p.acc_off = p.lut_off + (fmt == kResTL2 ? al128((uint64_t)K * 16) : 0u);
   p.w_off = p.acc_off + (wk > 1 ? al128((uint64_t)nblk * 4 * kResMaxTok * 4) : 0u);
-  const uint64_t total = (uint64_t)p.w_off + al128((uint64_t)nblk * 4 * (K / 4));
-  if (total > res_smem_max(nw)) return false;
+  const uint64_t total = (uint64_t)p.w_off + al128((uint64_t)nblk * 4 * Rb);
+  if (total > res_smem_max(fmt)) return false;
   out->grid = grid;
   out->smem = (uint32_t)total;
   return true;
 }
 
-template <int MT, int MM, int NW>
+template <int FMT, int MT, int MM>
 static cudaError_t launch_resident_t(const ResidentPlan& pl, cudaStream_t stream) {
   static std::atomic<uint64_t> configured{0};
-  cudaError_t e = set_smem_attr_once(configured, resident_kernel<MT, MM, NW>,
-                                     (int)res_smem_max(NW), cudaSharedmemCarveoutMaxShared);
+  cudaError_t e = set_smem_attr_once(configured, resident_kernel<FMT, MT, MM>,
+                                     (int)res_smem_max(FMT), cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)pl.grid);
-  cfg.blockDim = dim3(NW * 32);
+  cfg.blockDim = dim3(kResThreads);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -403,37 +486,44 @@ static cudaError_t launch_resident_t(const ResidentPlan& pl, cudaStream_t stream
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, resident_kernel<MT, MM, NW>, pl.p);
+  return cudaLaunchKernelEx(&cfg, resident_kernel<FMT, MT, MM>, pl.p);
 }
 
 }  // namespace bitnet
 
 using namespace bitnet;
 
-// Warps per CTA of the resident kernel: 16, two CTAs per SM, so the next
+// The resident kernel runs 16 warps per CTA, two CTAs per SM, so the next
 // layer's CTA loads its weights while this one computes (one CTA of 32 warps
 // per SM measured slower: 6.0 vs 3.4 us per 2B layer).  The products are
 // dp4a items: warp-level int8 MMA items (16-row tiles) measured slower here,
 // 4.27 vs 2.94 us per 2B layer at one token and 6.36 vs 5.39 at two.
-constexpr int kResidentWarps = RESIDENT_WARPS;
 
-// Whether the resident kernel serves this BitLinear shape.
-bool bitnet_resident_fits(int64_t M, int64_t N, int64_t K, int num_sms) {
+// Whether the resident kernel serves this shape in format fmt (0: I2_S
+// ternary, 1: sign bits, 2: I2_S through pair tables).
+bool bitnet_resident_fits(int fmt, int64_t M, int64_t N, int64_t K, int num_sms) {
   if (M > 8 || N > 0x7fffffff || K > 0x7fffffff) return false;
   ResidentPlan pl;
-  return plan_resident((int)M, (int)N, (int)K, num_sms, kResidentWarps, &pl);
+  return plan_resident(fmt, (int)M, (int)N, (int)K, num_sms, &pl);
 }
 
-bitnet_status bitnet_resident_launch(const uint8_t* w, const float* gamma, int N, int K,
+bitnet_status bitnet_resident_launch(int fmt, const uint8_t* w, const float* gamma, int N, int K,
                                      const uint16_t* x, int M, uint16_t* y, float* y_f32,
                                      int32_t* acc, int num_sms, cudaStream_t stream) {
-  constexpr int NW = kResidentWarps;
   ResidentPlan pl;
-  if (!plan_resident(M, N, K, num_sms, NW, &pl)) return BITNET_ERR_UNSUPPORTED;
+  if (!plan_resident(fmt, M, N, K, num_sms, &pl)) return BITNET_ERR_UNSUPPORTED;
   pl.p.w = w; pl.p.gamma = gamma; pl.p.x = x; pl.p.y = y; pl.p.y_f32 = y_f32; pl.p.acc = acc;
   cudaError_t e;
-  if (M == 1) e = launch_resident_t<1, 1, NW>(pl, stream);
-  else if (M == 2) e = launch_resident_t<2, 2, NW>(pl, stream);
-  else e = launch_resident_t<2, 4, NW>(pl, stream);
+  if (fmt == kResTL2) {
+    e = launch_resident_t<kResTL2, 1, 1>(pl, stream);
+  } else if (fmt == kResW1) {
+    if (M == 1) e = launch_resident_t<kResW1, 1, 1>(pl, stream);
+    else if (M == 2) e = launch_resident_t<kResW1, 2, 2>(pl, stream);
+    else e = launch_resident_t<kResW1, 2, 4>(pl, stream);
+  } else {
+    if (M == 1) e = launch_resident_t<kResI2S, 1, 1>(pl, stream);
+    else if (M == 2) e = launch_resident_t<kResI2S, 2, 2>(pl, stream);
+    else e = launch_resident_t<kResI2S, 2, 4>(pl, stream);
+  }
   return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
