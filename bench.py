@@ -428,6 +428,28 @@ def secondary_measurements(B, inputs, torch, dev, stream, pk):
                      "bytes": "packed weights streamed per step (1 bit per weight for w1)"}
         del g
     del w1, wsw
+    # a4.8 (4-bit activations, the round(0.01 K) largest values at 8 bits) on
+    # the same chain: quantiser, tensor-core kernel on 2 rows, combine
+    n_out = {K: int(round(0.01 * K)) for K in (HIDDEN, INTER)}
+    wsa = torch.empty(max(B.bitnet_linear_a48_workspace_size(1, INTER, HIDDEN),
+                          B.bitnet_linear_a48_workspace_size(1, HIDDEN, INTER)),
+                      dtype=torch.uint8, device=dev)
+
+    def run_a48():
+        cur = x1
+        for l, (p, g) in enumerate(packs):
+            B.bitnet_linear_a48(p, g, cur, n_out[p.shape[1] * 4], y=bufs[l % 2], workspace=wsa)
+            cur = bufs[l % 2]
+    g = capture(torch, run_a48, stream)
+    ms, _, _ = time_graph(torch, g, stream, 20, 3)
+    t = ms / 20 * 1e-3
+    nbytes = sum(p.numel() for p, _ in packs)
+    out["decode_chain_a48_M1"] = {"GB/s": round(nbytes / t / 1e9, 1),
+                                  "us_per_layer": round(t / 60 * 1e6, 3),
+                                  "frac_hbm": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4),
+                                  "launches_per_layer": "quantiser, split-K clear, tensor-core "
+                                                        "kernel, finaliser, combine"}
+    del g, wsa
     # FFN 100B-class: two distinct blocks rotated
     H, I = 8192, 28672
     blocks = []

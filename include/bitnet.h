@@ -316,6 +316,42 @@ BITNET_API bitnet_status bitnet_linear_tl2(const uint8_t* packed, const float* g
                                            float* y_f32, int32_t* acc, void* stream);
 
 /*
+ * BitNet a4.8: 4-bit activations with the largest values at 8 bits, on the
+ * ternary I2_S weights.
+ *   [Y] section "BitNet a4.8：ハイブリッド量子化戦略" (the top fraction of the
+ *       activation values is split off and processed at 8 bits, the rest is
+ *       quantised to 4 bits).
+ * The pages give neither the fraction nor the scales.  Per token, the n_out
+ * values of largest |x| (ties between equal |x| go to the lower channel) are
+ * the 8-bit part, the rest the 4-bit part, each with its own absmax scale:
+ *   s4 = 7 / max(max|x_in|, 1e-5),    q4 = clamp(rint(x s4), -8, 7) on inliers, 0 else
+ *   s8 = 127 / max(max|x_out|, 1e-5), q8 = clamp(rint(x s8), -128, 127) on outliers, 0 else
+ *   acc4 = q4 . W_q, acc8 = q8 . W_q   (exact int32)
+ *   y32 = fp32(acc4) (gamma / s4) + fp32(acc8) (gamma / s8)  (two fp32
+ *         products, one fp32 sum);  y = bf16(y32), nearest even.
+ * The page's second technique, per-channel scaling, comes with no formula and
+ * is not applied.
+ *
+ * bitnet_quant_act_a48: x [M,K] bf16 bits; q4, q8 [M,K] int8 (natural
+ * order) and s4, s8 [M] fp32, device, written.  Requires K % 8 == 0,
+ * 0 <= n_out <= K.
+ * bitnet_linear_a48: packed [N,K/4], gamma as bitnet_linear; y [M,N] bf16
+ * bits; y_f32, acc4, acc8 optional [M,N]; workspace >=
+ * bitnet_linear_a48_workspace_size(M, N, K) bytes.  Requires K % 64 == 0,
+ * 0 <= n_out <= K.  Runs the a4.8 quantiser (one CTA per token), the
+ * tensor-core kernel on the 2M code rows, and a combine kernel.
+ */
+BITNET_API bitnet_status bitnet_quant_act_a48(const uint16_t* x, int64_t M, int64_t K,
+                                              int64_t n_out, int8_t* q4, float* s4, int8_t* q8,
+                                              float* s8, void* stream);
+BITNET_API size_t bitnet_linear_a48_workspace_size(int64_t M, int64_t N, int64_t K);
+BITNET_API bitnet_status bitnet_linear_a48(const uint8_t* packed, const float* gamma, int64_t N,
+                                           int64_t K, const uint16_t* x, int64_t M,
+                                           int64_t n_out, uint16_t* y, float* y_f32,
+                                           int32_t* acc4, int32_t* acc8, void* workspace,
+                                           size_t workspace_bytes, void* stream);
+
+/*
  * Synchronise `stream`, then return and clear the device status word of the
  * current device: BITNET_OK, BITNET_ERR_TIMEOUT (a bounded wait expired; the
  * affected outputs are unspecified) or BITNET_ERR_NONFINITE.  A failing

@@ -48,6 +48,10 @@ SIGNATURES = {
     "bitnet_linear_w1_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "bitnet_linear_w1": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I64, _P, _P, _P, _P, _SZ, _P]),
     "bitnet_linear_tl2": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _P, _P, _P, _P]),
+    "bitnet_quant_act_a48": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
+    "bitnet_linear_a48_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "bitnet_linear_a48": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I64, _I64, _P, _P, _P, _P, _P,
+                                         _SZ, _P]),
 }
 
 
@@ -396,6 +400,50 @@ def bitnet_linear_tl2(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor
                                  _ptr(acc), _stream())
     _check("bitnet_linear_tl2", st)
     return y, y32, acc
+
+
+def bitnet_quant_act_a48(x: torch.Tensor, n_out: int):
+    """a4.8 activations: x bf16 [M,K] -> (q4 int8 [M,K], s4 [M], q8 int8 [M,K], s8 [M])."""
+    _bits16(x, "x")
+    M, K = x.shape
+    q4 = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    q8 = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s4 = torch.empty(M, dtype=torch.float32, device=x.device)
+    s8 = torch.empty(M, dtype=torch.float32, device=x.device)
+    st = lib().bitnet_quant_act_a48(_ptr(x), M, K, int(n_out), _ptr(q4), _ptr(s4), _ptr(q8),
+                                    _ptr(s8), _stream())
+    _check("bitnet_quant_act_a48", st)
+    return q4, s4, q8, s8
+
+
+def bitnet_linear_a48_workspace_size(M: int, N: int, K: int) -> int:
+    return lib().bitnet_linear_a48_workspace_size(M, N, K)
+
+
+def bitnet_linear_a48(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, n_out: int,
+                      y=None, want_f32: bool = False, want_acc: bool = False, workspace=None,
+                      y_f32=None, acc4=None, acc8=None):
+    """a4.8 BitLinear.  Returns (y bf16 [M,N], y_f32, acc4, acc8)."""
+    _dev(packed, "packed")
+    _dev(gamma, "gamma")
+    _bits16(x, "x")
+    N, Kb = packed.shape
+    M, K = x.shape
+    if K != 4 * Kb:
+        raise ValueError("x and packed disagree on K")
+    dev = x.device
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if y is None else y
+    y32 = y_f32 if y_f32 is not None else (
+        torch.empty((M, N), dtype=torch.float32, device=dev) if want_f32 else None)
+    if want_acc:
+        acc4 = torch.empty((M, N), dtype=torch.int32, device=dev) if acc4 is None else acc4
+        acc8 = torch.empty((M, N), dtype=torch.int32, device=dev) if acc8 is None else acc8
+    nb = lib().bitnet_linear_a48_workspace_size(M, N, K)
+    ws = _workspace(nb, dev, workspace)
+    st = lib().bitnet_linear_a48(_ptr(packed), _ptr(gamma), N, K, _ptr(x), M, int(n_out), _ptr(y),
+                                 _ptr(y32), _ptr(acc4), _ptr(acc8), _ptr(ws), nb, _stream())
+    _check("bitnet_linear_a48", st)
+    return y, y32, acc4, acc8
 
 
 def bitnet_last_device_status() -> int:

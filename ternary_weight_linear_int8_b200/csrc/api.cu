@@ -25,6 +25,13 @@ bitnet_status bitnet_pack_w1_launch(const float* W, int64_t N, int64_t K, uint8_
                                     int num_sms);
 bitnet_status bitnet_sign_to_i2s_launch(const uint8_t* sign, int64_t nbytes, uint8_t* codes,
                                         int num_sms, cudaStream_t stream);
+bitnet_status bitnet_a48_quant_launch(const uint16_t* x, int64_t M, int64_t K, int64_t n_out,
+                                      int8_t* rows, float* scale, int32_t* rowsum, int8_t* q4n,
+                                      int8_t* q8n, float* s4, float* s8, cudaStream_t stream);
+bitnet_status bitnet_a48_combine_launch(const int32_t* acc2, const float* scale,
+                                        const float* gamma, int64_t M, int64_t N, uint16_t* y,
+                                        float* y_f32, int32_t* acc4, int32_t* acc8, int num_sms,
+                                        cudaStream_t stream);
 bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
                                  const uint8_t* w1, GemmArgs a, int bn, int num_sms,
                                  cudaStream_t stream);
@@ -177,6 +184,29 @@ FfnWs ffn_ws_layout(int64_t M, int64_t H, int64_t I) {
 }
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Workspace of bitnet_linear_a48: the 2M code rows (q4 of token m at row 2m,
+// q8 at 2m + 1, kernel K order), their scales and row sums, the exact
+// accumulators of the 2M rows, the tensor-core kernel's (unused) bf16 rows,
+// and its split-K accumulators for small M.
+struct A48Ws {
+  size_t rows, scale, rowsum, acc2, yscr, acc, total;
+};
+
+A48Ws a48_ws_layout(int64_t M, int64_t N, int64_t K) {
+  A48Ws w{};
+  const int64_t M2 = 2 * M;
+  size_t off = 0;
+  w.rows = off; off += al256((size_t)M2 * K);
+  w.scale = off; off += al256((size_t)M2 * 4);
+  w.rowsum = off; off += al256((size_t)M2 * 4);
+  w.acc2 = off; off += al256((size_t)M2 * N * 4);
+  w.yscr = off; off += al256((size_t)M2 * N * 2);
+  w.acc = off;
+  if (M2 <= 256) off += splitk_acc_bytes(M2, N) + splitk_cnt_bytes(M2, N);
+  w.total = off;
+  return w;
+}
 
 }  // namespace
 
@@ -544,6 +574,72 @@ bitnet_status bitnet_linear_tl2(const uint8_t* packed, const float* gamma, int64
   if (!bitnet_resident_fits(2, 1, N, K, d.num_sms)) return BITNET_ERR_UNSUPPORTED;
   return bitnet_resident_launch(2, packed, gamma, (int)N, (int)K, x, 1, y, y_f32, acc, d.num_sms,
                                 as_stream(stream));
+}
+
+bitnet_status bitnet_quant_act_a48(const uint16_t* x, int64_t M, int64_t K, int64_t n_out,
+                                   int8_t* q4, float* s4, int8_t* q8, float* s8, void* stream) {
+  if (!x || !q4 || !s4 || !q8 || !s8) return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || K < 8 || K % 8 != 0 || M > 0x7fffffff || K > 524288) return BITNET_ERR_SHAPE;
+  if (n_out < 0 || n_out > K) return BITNET_ERR_INVALID_ARG;
+  if (!aligned16(x) || ((uintptr_t)s4 & 3u) || ((uintptr_t)s8 & 3u)) return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  return bitnet_a48_quant_launch(x, M, K, n_out, nullptr, nullptr, nullptr, q4, q8, s4, s8,
+                                 as_stream(stream));
+}
+
+size_t bitnet_linear_a48_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 8) return 0;
+  return a48_ws_layout(M, N, K).total;
+}
+
+bitnet_status bitnet_linear_a48(const uint8_t* packed, const float* gamma, int64_t N, int64_t K,
+                                const uint16_t* x, int64_t M, int64_t n_out, uint16_t* y,
+                                float* y_f32, int32_t* acc4, int32_t* acc8, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!packed || !gamma || !x || !y) return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 64 || K % 64 != 0 || K > 524288 || M > 0x3fffffff ||
+      N > 0x7fffffff)
+    return BITNET_ERR_SHAPE;
+  if (n_out < 0 || n_out > K) return BITNET_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(x) || !aligned16(y) || ((uintptr_t)gamma & 3u) ||
+      ((uintptr_t)y_f32 & 3u) || ((uintptr_t)acc4 & 3u) || ((uintptr_t)acc8 & 3u))
+    return BITNET_ERR_ALIGN;
+  const A48Ws L = a48_ws_layout(M, N, K);
+  if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* rows = reinterpret_cast<int8_t*>(ws + L.rows);
+  float* sc = reinterpret_cast<float*>(ws + L.scale);
+  int32_t* rs = reinterpret_cast<int32_t*>(ws + L.rowsum);
+  int32_t* acc2 = reinterpret_cast<int32_t*>(ws + L.acc2);
+  st = bitnet_a48_quant_launch(x, M, K, n_out, rows, sc, rs, nullptr, nullptr, nullptr, nullptr,
+                               s);
+  if (st != BITNET_OK) return st;
+  // the integer products of all 2M code rows on the tensor-core kernel
+  const int64_t M2 = 2 * M;
+  const int bn = bitnet_gemm_pick_bn((int)M2, (int)N, d.num_sms);
+  GemmArgs a{};
+  a.M = (int)M2; a.N = (int)N; a.K = (int)K;
+  a.ksplit = plan_ksplit(M2, N, K, bn, d.num_sms);
+  a.scale = sc; a.rowsum = rs; a.gamma0 = gamma;
+  a.y = reinterpret_cast<uint16_t*>(ws + L.yscr);
+  a.acc0 = acc2;
+  if (a.ksplit > 1) {
+    a.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc);
+    a.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc + splitk_acc_bytes(M2, N));
+    if (cudaMemsetAsync(a.acc_ws0, 0, splitk_acc_bytes(M2, N) + splitk_cnt_bytes(M2, N), s) !=
+        cudaSuccess)
+      return BITNET_ERR_CUDA;
+  }
+  st = bitnet_gemm_launch(0 /*linear*/, rows, packed, nullptr, a, bn, d.num_sms, s);
+  if (st != BITNET_OK) return st;
+  return bitnet_a48_combine_launch(acc2, sc, gamma, M, N, y, y_f32, acc4, acc8, d.num_sms, s);
 }
 
 bitnet_status bitnet_last_device_status(void* stream) {

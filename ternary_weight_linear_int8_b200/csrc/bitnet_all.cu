@@ -6,5 +6,6 @@
 #include "gemv.cu"
 #include "resident.cu"
 #include "gemm.cu"
+#include "a48.cu"
 #include "api.cu"
 #include "noalloc.cu"

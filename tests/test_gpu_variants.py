@@ -99,3 +99,47 @@ def test_linear_tl2_matches_oracle(N, K):
     assert np.array_equal(host_bits(y), ref["y"])
     for o in outs:
         o.check()
+
+
+# ------------------------------------------------------------------- a4.8
+def _a48_tokens(M, K, seed):
+    """Outlier-channel activations, plus a token with many equal magnitudes
+    (ties at the selection threshold must go to the lower channels)."""
+    x = inputs.activations((M, K), seed=seed, outliers=True)
+    if M > 1:
+        xf = np.tile(np.array([4.0, -4.0, 4.0, 1.0, -2.0, 2.0, 2.0, -2.0], np.float32), K // 8)
+        x[1] = O.f32_to_bf16_bits(xf)
+    return x
+
+
+@pytest.mark.parametrize("M,K,n_out", [(1, 2560, 26), (4, 6912, 69), (3, 512, 0), (2, 512, 512),
+                                       (5, 64, 3), (2, 1024, 257), (8, 2560, 1)])
+def test_quant_act_a48_matches_oracle(M, K, n_out):
+    x = _a48_tokens(M, K, seed=M + K + n_out)
+    q4r, s4r, q8r, s8r, _ = V.act_quant_a48(x, n_out)
+    q4, s4, q8, s8 = B.bitnet_quant_act_a48(dev_bits(x), n_out)
+    assert np.array_equal(q4.cpu().numpy(), q4r)
+    assert np.array_equal(q8.cpu().numpy(), q8r)
+    assert np.array_equal(f32_bits(s4.cpu().numpy()), f32_bits(s4r))
+    assert np.array_equal(f32_bits(s8.cpu().numpy()), f32_bits(s8r))
+
+
+@pytest.mark.parametrize("M,N,K,n_out", [(1, 6912, 2560, 26), (1, 2560, 6912, 69),
+                                         (4, 400, 512, 5), (16, 300, 1024, 10),
+                                         (64, 2560, 6912, 69), (3, 257, 128, 0), (2, 100, 128, 128)])
+def test_linear_a48_matches_oracle(M, N, K, n_out):
+    x = _a48_tokens(M, K, seed=N + K)
+    W = inputs.weights(N, K, seed=K + 3)
+    p_ref, g_ref = O.pack_weights(W)
+    ref = V.linear_a48(p_ref, g_ref, x, n_out)
+    p, g = B.bitnet_pack_weights(dev_f32(W))
+    outs = [guarded((M, N), torch.bfloat16), guarded((M, N), torch.float32),
+            guarded((M, N), torch.int32), guarded((M, N), torch.int32)]
+    y, y32, a4, a8 = B.bitnet_linear_a48(p, g, dev_bits(x), n_out, y=outs[0].t, y_f32=outs[1].t,
+                                         acc4=outs[2].t, acc8=outs[3].t)
+    assert np.array_equal(a4.cpu().numpy(), ref["acc4"].astype(np.int32))
+    assert np.array_equal(a8.cpu().numpy(), ref["acc8"].astype(np.int32))
+    assert np.array_equal(f32_bits(y32.cpu().numpy()), f32_bits(ref["y32"]))
+    assert np.array_equal(host_bits(y), ref["y"])
+    for o in outs:
+        o.check()
