@@ -503,6 +503,16 @@ def profile_case(case):
         call = ChainCall(B, torch, packs, bufs, dev)
         for _ in range(3):
             call(x)
+    elif case == "tl2":
+        # one up and one down 2B layer, dp4a inner loop then pair tables
+        x = torch.from_numpy(inputs.activations((1, HIDDEN), seed=0).view(np.int16)).to(dev)
+        for l, (N, K) in enumerate(((INTER, HIDDEN), (HIDDEN, INTER))):
+            W = torch.from_numpy(inputs.weights(N, K, seed=inputs.layer_seed(l))).to(dev)
+            p, g = B.bitnet_pack_weights(W)
+            xi = x if l == 0 else torch.zeros((1, K), dtype=torch.int16, device=dev)
+            for _ in range(2):
+                B.bitnet_linear(p, g, xi)
+                B.bitnet_linear_tl2(p, g, xi)
     elif case in ("batched8", "batched16"):
         M = int(case[len("batched"):])
         packs = build_decode_chain(B, inputs, torch, dev, n_layers=6)
@@ -671,7 +681,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--profile-case", choices=["prefill", "prefill_down", "ffn2048", "gemv_big", "batched8", "batched16",
-                             "chain2b"],
+                             "chain2b", "tl2"],
                     default=None,
                     help="run a few calls of one workload for an ncu capture, print nothing")
     args = ap.parse_args()

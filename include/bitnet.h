@@ -352,6 +352,51 @@ BITNET_API bitnet_status bitnet_linear_a48(const uint8_t* packed, const float* g
                                            size_t workspace_bytes, void* stream);
 
 /*
+ * The FFN block split over G devices (tensor parallel), for models too large
+ * for one GPU: [D] (100B-class models), [A] section
+ * "推論コストはどれだけ下がったのか" (70B-class serving).  Gate and up are split
+ * by rows (shard r holds intermediate features [I_r0, I_r1), Ir of them),
+ * down by columns (the same features), norm2_w likewise; every shard holds
+ * the whole token x and the whole-matrix gammas (pack the whole matrix, then
+ * slice the packed rows / byte columns).  Per block:
+ *   1. bitnet_ffn_tp_gate_up on every shard: h' [M,Ir] (fp32), the shard's
+ *      absmax of h' * n2 (amax2 [M]) and sum of h'^2 (sumsq_h [M], fp64),
+ *      and the token's sum of x^2 (sumsq_x [M], fp64; equal on every shard);
+ *   2. all-reduce amax2 with MAX and sumsq_h with SUM over the shards;
+ *   3. bitnet_ffn_tp_down on every shard: h' * n2 quantised with the
+ *      all-reduced absmax (the codes the whole-block quantiser gives these
+ *      features), times the shard's down columns: partial integer
+ *      accumulators acc [M,H] (int32);
+ *   4. all-reduce acc with SUM (exact integers: sharding changes no code or
+ *      accumulator);
+ *   5. bitnet_ffn_tp_finish: y = bf16((fp32(acc) * (gamma_d / s2)) *
+ *      fp32(r1^3 r2)) with r1, r2 from sumsq_x and the all-reduced sumsq_h,
+ *      I the whole intermediate width, as bitnet_ffn computes it.
+ * Codes and accumulators equal the single-device block's bit for bit; y32
+ * differs only through the rounding order of the all-reduced fp64 sum
+ * (within 1e-5 relative).  The collectives are the caller's (the Python
+ * module tensor_parallel runs them with torch.distributed).
+ * Shapes: H % 64 == 0, Ir % 64 == 0; workspace >=
+ * bitnet_ffn_tp_workspace_size(M, H, Ir) for steps 1 and 3.
+ */
+BITNET_API size_t bitnet_ffn_tp_workspace_size(int64_t M, int64_t H, int64_t Ir);
+BITNET_API bitnet_status bitnet_ffn_tp_gate_up(const uint16_t* x, int64_t M, int64_t H, int64_t Ir,
+                                               const float* norm1_w, const uint8_t* gate,
+                                               const float* gamma_gate, const uint8_t* up,
+                                               const float* gamma_up, const float* norm2_w,
+                                               float* h, float* amax2, double* sumsq_h,
+                                               double* sumsq_x, void* workspace,
+                                               size_t workspace_bytes, void* stream);
+BITNET_API bitnet_status bitnet_ffn_tp_down(const float* h, int64_t M, int64_t H, int64_t Ir,
+                                            const float* norm2_w, const uint8_t* down,
+                                            const float* amax2, int32_t* acc, void* workspace,
+                                            size_t workspace_bytes, void* stream);
+BITNET_API bitnet_status bitnet_ffn_tp_finish(const int32_t* acc, int64_t M, int64_t H, int64_t I,
+                                              const float* gamma_down, const float* amax2,
+                                              const double* sumsq_x, const double* sumsq_h,
+                                              float eps, uint16_t* y, float* y_f32, void* stream);
+
+/*
  * Synchronise `stream`, then return and clear the device status word of the
  * current device: BITNET_OK, BITNET_ERR_TIMEOUT (a bounded wait expired; the
  * affected outputs are unspecified) or BITNET_ERR_NONFINITE.  A failing

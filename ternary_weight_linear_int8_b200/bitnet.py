@@ -52,6 +52,12 @@ SIGNATURES = {
     "bitnet_linear_a48_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "bitnet_linear_a48": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I64, _I64, _P, _P, _P, _P, _P,
                                          _SZ, _P]),
+    "bitnet_ffn_tp_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "bitnet_ffn_tp_gate_up": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
+                                             _P, _P, _P, _SZ, _P]),
+    "bitnet_ffn_tp_down": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _SZ, _P]),
+    "bitnet_ffn_tp_finish": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _F, _P, _P,
+                                            _P]),
 }
 
 
@@ -444,6 +450,59 @@ def bitnet_linear_a48(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor
                                  _ptr(y32), _ptr(acc4), _ptr(acc8), _ptr(ws), nb, _stream())
     _check("bitnet_linear_a48", st)
     return y, y32, acc4, acc8
+
+
+def bitnet_ffn_tp_workspace_size(M: int, H: int, Ir: int) -> int:
+    return lib().bitnet_ffn_tp_workspace_size(M, H, Ir)
+
+
+def bitnet_ffn_tp_gate_up(x, gate, gamma_gate, up, gamma_up, norm1_w=None, norm2_w=None,
+                          workspace=None):
+    """Tensor-parallel FFN step 1 on this shard.  Returns (h [M,Ir] fp32,
+    amax2 [M] fp32, sumsq_h [M] fp64, sumsq_x [M] fp64)."""
+    _bits16(x, "x")
+    M, H = x.shape
+    Ir = gate.shape[0]
+    dev = x.device
+    h = torch.empty((M, Ir), dtype=torch.float32, device=dev)
+    amax2 = torch.empty(M, dtype=torch.float32, device=dev)
+    ssh = torch.empty(M, dtype=torch.float64, device=dev)
+    ssx = torch.empty(M, dtype=torch.float64, device=dev)
+    nb = lib().bitnet_ffn_tp_workspace_size(M, H, Ir)
+    ws = _workspace(nb, dev, workspace)
+    st = lib().bitnet_ffn_tp_gate_up(_ptr(x), M, H, Ir, _ptr(norm1_w), _ptr(gate), _ptr(gamma_gate),
+                                     _ptr(up), _ptr(gamma_up), _ptr(norm2_w), _ptr(h), _ptr(amax2),
+                                     _ptr(ssh), _ptr(ssx), _ptr(ws), nb, _stream())
+    _check("bitnet_ffn_tp_gate_up", st)
+    return h, amax2, ssh, ssx
+
+
+def bitnet_ffn_tp_down(h, down, amax2, norm2_w=None, workspace=None):
+    """Tensor-parallel FFN step 3 on this shard: partial int32 accumulators [M,H]."""
+    _dev(h, "h")
+    M, Ir = h.shape
+    H = down.shape[0]
+    acc = torch.empty((M, H), dtype=torch.int32, device=h.device)
+    nb = lib().bitnet_ffn_tp_workspace_size(M, H, Ir)
+    ws = _workspace(nb, h.device, workspace)
+    st = lib().bitnet_ffn_tp_down(_ptr(h), M, H, Ir, _ptr(norm2_w), _ptr(down), _ptr(amax2),
+                                  _ptr(acc), _ptr(ws), nb, _stream())
+    _check("bitnet_ffn_tp_down", st)
+    return acc
+
+
+def bitnet_ffn_tp_finish(acc, I, gamma_down, amax2, sumsq_x, sumsq_h, eps=1e-5, y=None,
+                         want_f32=False):
+    """Tensor-parallel FFN step 5: y bf16 [M,H] (and y_f32) from the all-reduced values."""
+    _dev(acc, "acc")
+    M, H = acc.shape
+    y = torch.empty((M, H), dtype=torch.bfloat16, device=acc.device) if y is None else y
+    y32 = torch.empty((M, H), dtype=torch.float32, device=acc.device) if want_f32 else None
+    st = lib().bitnet_ffn_tp_finish(_ptr(acc), M, H, int(I), _ptr(gamma_down), _ptr(amax2),
+                                    _ptr(sumsq_x), _ptr(sumsq_h), float(eps), _ptr(y), _ptr(y32),
+                                    _stream())
+    _check("bitnet_ffn_tp_finish", st)
+    return y, y32
 
 
 def bitnet_last_device_status() -> int:

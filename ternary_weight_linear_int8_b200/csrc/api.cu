@@ -14,7 +14,7 @@ bitnet_status bitnet_pack_launch(const float* W, int64_t N, int64_t K, uint8_t* 
 bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* gain, int64_t M,
                                   int64_t K, int8_t* xq, int64_t ld_q, bool perm, float* scale,
                                   int32_t* rowsum, double* sumsq, int8_t* xq_natural,
-                                  cudaStream_t stream);
+                                  cudaStream_t stream, const float* amax_in, float* amax_out);
 bitnet_status bitnet_decode_launch(const DecodeOp& op, int M, int num_sms, cudaStream_t stream);
 bool bitnet_resident_fits(int fmt, int64_t M, int64_t N, int64_t K, int num_sms);
 bitnet_status bitnet_resident_launch(int fmt, const uint8_t* w, const float* gamma, int N, int K,
@@ -63,6 +63,32 @@ __global__ void __launch_bounds__(256) generic_linear_kernel(const uint8_t* __re
     y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
     if (y_f32) y_f32[o] = y32;
     if (acc_out) acc_out[o] = acc;
+  }
+}
+
+// Last step of the tensor-parallel FFN: the all-reduced integer accumulators
+// of the down projection dequantised with the all-reduced statistics, in the
+// same steps as the single-GPU block: s2 = 127 / max(amax2, 1e-5),
+// r1 = 1/sqrt(sum x^2 / H + eps), r2 = 1/sqrt(r1^6 sum h'^2 / I + eps) (fp64),
+// y32 = (fp32(acc) * (gamma_d / s2)) * fp32(r1^3 r2).
+__global__ void __launch_bounds__(256) ffn_tp_finish_kernel(
+    const int32_t* __restrict__ acc, int M, int H, int I, const float* gamma_d,
+    const float* __restrict__ amax2, const double* __restrict__ ssx,
+    const double* __restrict__ ssh, float eps, uint16_t* y, float* y_f32) {
+  pdl_wait();
+  const int64_t total = (int64_t)M * H;
+  for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < total;
+       o += (int64_t)gridDim.x * blockDim.x) {
+    const int m = (int)(o / H);
+    const float d0 = __fdiv_rn(*gamma_d, qscale(amax2[m]));
+    const double e = (double)eps;
+    const double r1 = 1.0 / sqrt(ssx[m] / (double)H + e);
+    const double r1_3 = r1 * r1 * r1;
+    const double r2 = 1.0 / sqrt(r1_3 * r1_3 * (ssh[m] / (double)I) + e);
+    const float f = (float)(r1_3 * r2);
+    const float y32 = __fmul_rn(__fmul_rn(__int2float_rn(acc[o]), d0), f);
+    y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+    if (y_f32) y_f32[o] = y32;
   }
 }
 
@@ -192,6 +218,35 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 struct A48Ws {
   size_t rows, scale, rowsum, acc2, yscr, acc, total;
 };
+
+// Workspace of the tensor-parallel FFN steps on one shard of Ir intermediate
+// features: first-norm codes of x (gate/up step) or second-norm codes of h'
+// (down step), their scales and row sums, the statistics pass's codes, the
+// down step's unused bf16 rows, and the tensor-core kernel's split-K
+// accumulators (gate and up, or down).
+struct TpWs {
+  size_t xq, s, rs, xq2, s2, yscr, acc0, acc1, total;
+};
+
+TpWs tp_ws_layout(int64_t M, int64_t H, int64_t Ir) {
+  TpWs w{};
+  const int64_t HI = H > Ir ? H : Ir;
+  size_t off = 0;
+  w.xq = off; off += al256((size_t)M * HI);
+  w.s = off; off += al256((size_t)M * 4);
+  w.rs = off; off += al256((size_t)M * 4);
+  w.xq2 = off; off += al256((size_t)M * Ir);
+  w.s2 = off; off += al256((size_t)M * 4);
+  w.yscr = off; off += al256((size_t)M * H * 2);
+  w.acc0 = off;
+  if (M <= 256) {
+    off += splitk_acc_bytes(M, HI) + splitk_cnt_bytes(M, HI);
+    w.acc1 = off;
+    off += al256((size_t)M * Ir * 4);
+  }
+  w.total = off;
+  return w;
+}
 
 A48Ws a48_ws_layout(int64_t M, int64_t N, int64_t K) {
   A48Ws w{};
@@ -640,6 +695,127 @@ bitnet_status bitnet_linear_a48(const uint8_t* packed, const float* gamma, int64
   st = bitnet_gemm_launch(0 /*linear*/, rows, packed, nullptr, a, bn, d.num_sms, s);
   if (st != BITNET_OK) return st;
   return bitnet_a48_combine_launch(acc2, sc, gamma, M, N, y, y_f32, acc4, acc8, d.num_sms, s);
+}
+
+size_t bitnet_ffn_tp_workspace_size(int64_t M, int64_t H, int64_t Ir) {
+  if (M < 1 || H < 1 || Ir < 1) return 0;
+  return tp_ws_layout(M, H, Ir).total;
+}
+
+bitnet_status bitnet_ffn_tp_gate_up(const uint16_t* x, int64_t M, int64_t H, int64_t Ir,
+                                    const float* norm1_w, const uint8_t* gate,
+                                    const float* gamma_gate, const uint8_t* up,
+                                    const float* gamma_up, const float* norm2_w, float* h,
+                                    float* amax2, double* sumsq_h, double* sumsq_x,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !gate || !gamma_gate || !up || !gamma_up || !h || !amax2 || !sumsq_h || !sumsq_x)
+    return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || H < 64 || Ir < 64 || H % 64 != 0 || Ir % 64 != 0 || H > 524288 || Ir > 524288 ||
+      M > 0x7fffffff)
+    return BITNET_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(h) || !aligned16(gate) || !aligned16(up) ||
+      ((uintptr_t)amax2 & 3u) || ((uintptr_t)sumsq_h & 7u) || ((uintptr_t)sumsq_x & 7u))
+    return BITNET_ERR_ALIGN;
+  const TpWs L = tp_ws_layout(M, H, Ir);
+  if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* xq1 = reinterpret_cast<int8_t*>(ws + L.xq);
+  float* s1 = reinterpret_cast<float*>(ws + L.s);
+  int32_t* rs1 = reinterpret_cast<int32_t*>(ws + L.rs);
+  // every rank holds the whole token: the same codes on every shard
+  st = bitnet_quant_launch(x, false, norm1_w, M, H, xq1, H, true, s1, rs1, sumsq_x, nullptr, s,
+                           nullptr, nullptr);
+  if (st != BITNET_OK) return st;
+  const int bn = M > 128 ? 256 : bitnet_gemm_pick_bn((int)M, (int)Ir, d.num_sms);
+  GemmArgs g{};
+  g.M = (int)M; g.N = (int)Ir; g.K = (int)H;
+  g.ksplit = plan_ksplit(M, Ir, H, bn, d.num_sms);
+  g.scale = s1; g.rowsum = rs1; g.gamma0 = gamma_gate; g.gamma1 = gamma_up;
+  g.h = h;
+  if (g.ksplit > 1) {
+    g.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
+    g.acc_ws1 = reinterpret_cast<int32_t*>(ws + L.acc1);
+    g.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc0 + splitk_acc_bytes(M, Ir));
+    if (cudaMemsetAsync(g.acc_ws0, 0, splitk_acc_bytes(M, Ir) + splitk_cnt_bytes(M, Ir), s) !=
+            cudaSuccess ||
+        cudaMemsetAsync(g.acc_ws1, 0, (size_t)M * Ir * 4, s) != cudaSuccess)
+      return BITNET_ERR_CUDA;
+  }
+  st = bitnet_gemm_launch(1 /*glu*/, xq1, gate, up, g, bn, d.num_sms, s);
+  if (st != BITNET_OK) return st;
+  // this shard's statistics of h' * n2: absmax and sum of squares of h'
+  return bitnet_quant_launch(h, true, norm2_w, M, Ir, reinterpret_cast<int8_t*>(ws + L.xq2), Ir,
+                             false, reinterpret_cast<float*>(ws + L.s2), nullptr, sumsq_h,
+                             nullptr, s, nullptr, amax2);
+}
+
+bitnet_status bitnet_ffn_tp_down(const float* h, int64_t M, int64_t H, int64_t Ir,
+                                 const float* norm2_w, const uint8_t* down, const float* amax2,
+                                 int32_t* acc, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  if (!h || !down || !amax2 || !acc) return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || H < 64 || Ir < 64 || H % 64 != 0 || Ir % 64 != 0 || H > 524288 || Ir > 524288 ||
+      M > 0x7fffffff)
+    return BITNET_ERR_SHAPE;
+  if (!aligned16(h) || !aligned16(down) || ((uintptr_t)amax2 & 3u) || ((uintptr_t)acc & 3u))
+    return BITNET_ERR_ALIGN;
+  const TpWs L = tp_ws_layout(M, H, Ir);
+  if (!workspace || workspace_bytes < L.total) return BITNET_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* xq2 = reinterpret_cast<int8_t*>(ws + L.xq);
+  float* s2 = reinterpret_cast<float*>(ws + L.s);
+  int32_t* rs2 = reinterpret_cast<int32_t*>(ws + L.rs);
+  // the shard's h' * n2 quantised with the all-reduced absmax: the codes the
+  // whole-block quantiser gives these features
+  st = bitnet_quant_launch(h, true, norm2_w, M, Ir, xq2, Ir, true, s2, rs2, nullptr, nullptr, s,
+                           amax2, nullptr);
+  if (st != BITNET_OK) return st;
+  const int bn = bitnet_gemm_pick_bn((int)M, (int)H, d.num_sms);
+  GemmArgs a{};
+  a.M = (int)M; a.N = (int)H; a.K = (int)Ir;
+  a.ksplit = plan_ksplit(M, H, Ir, bn, d.num_sms);
+  a.scale = s2; a.rowsum = rs2; a.gamma0 = amax2;   // the bf16 rows are not used
+  a.y = reinterpret_cast<uint16_t*>(ws + L.yscr);
+  a.acc0 = acc;
+  if (a.ksplit > 1) {
+    a.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
+    a.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc0 + splitk_acc_bytes(M, H));
+    if (cudaMemsetAsync(a.acc_ws0, 0, splitk_acc_bytes(M, H) + splitk_cnt_bytes(M, H), s) !=
+        cudaSuccess)
+      return BITNET_ERR_CUDA;
+  }
+  return bitnet_gemm_launch(0 /*linear*/, xq2, down, nullptr, a, bn, d.num_sms, s);
+}
+
+bitnet_status bitnet_ffn_tp_finish(const int32_t* acc, int64_t M, int64_t H, int64_t I,
+                                   const float* gamma_down, const float* amax2,
+                                   const double* sumsq_x, const double* sumsq_h, float eps,
+                                   uint16_t* y, float* y_f32, void* stream) {
+  if (!acc || !gamma_down || !amax2 || !sumsq_x || !sumsq_h || !y) return BITNET_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !(eps < 3.0e38f)) return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || H < 1 || I < 1 || M > 0x7fffffff || H > 0x7fffffff || I > 0x7fffffff)
+    return BITNET_ERR_SHAPE;
+  if (((uintptr_t)acc & 3u) || ((uintptr_t)y & 1u) || ((uintptr_t)y_f32 & 3u) ||
+      ((uintptr_t)amax2 & 3u) || ((uintptr_t)sumsq_x & 7u) || ((uintptr_t)sumsq_h & 7u))
+    return BITNET_ERR_ALIGN;
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  int64_t blocks = (M * H + 255) / 256;
+  if (blocks > (int64_t)d.num_sms * 8) blocks = (int64_t)d.num_sms * 8;
+  ffn_tp_finish_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(
+      acc, (int)M, (int)H, (int)I, gamma_down, amax2, sumsq_x, sumsq_h, eps, y, y_f32);
+  return cudaGetLastError() == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
 
 bitnet_status bitnet_last_device_status(void* stream) {

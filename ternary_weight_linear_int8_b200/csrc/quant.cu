@@ -23,6 +23,9 @@ struct QuantArgs {
   int32_t* rowsum;        // [M] or null
   double* sumsq;          // [M] or null: sum over k of src^2 (not the gained value)
   int8_t* xq_natural;     // optional extra natural-layout copy (debug), [M,K]
+  const float* amax_in;   // [M] or null: the absmax to quantise with (a tensor-
+                          // parallel shard uses the all-reduced one)
+  float* amax_out;        // [M] or null: this row's absmax of src * gain
 };
 
 // 8 consecutive source values as floats (one 16-byte load of bf16, two of fp32).
@@ -102,7 +105,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
     }
     amax = warp_max(amax);
     if (a.sumsq) ss = warp_sum_d(ss);
-    const float s = qscale(amax);
+    if (a.amax_out && lane == 0) a.amax_out[m] = amax;
+    const float s = qscale(a.amax_in ? a.amax_in[m] : amax);
     // pass 2: quantise
     int rs = 0;
     if (kPerm) {
@@ -219,7 +223,8 @@ __global__ void __launch_bounds__(256) quant_token_kernel(QuantArgs a) {
   float am = s_max[0];
 #pragma unroll
   for (int w = 1; w < 8; ++w) am = fmaxf(am, s_max[w]);
-  const float s = qscale(am);
+  if (a.amax_out && threadIdx.x == 0) a.amax_out[m] = am;
+  const float s = qscale(a.amax_in ? a.amax_in[m] : am);
   // pass 2: quantise (groups of 16 for the permuted layout, else 4)
   int rs = 0;
   if (kPerm) {
@@ -286,8 +291,9 @@ using namespace bitnet;
 bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* gain, int64_t M,
                                   int64_t K, int8_t* xq, int64_t ld_q, bool perm, float* scale,
                                   int32_t* rowsum, double* sumsq, int8_t* xq_natural,
-                                  cudaStream_t stream) {
-  QuantArgs a{src, gain, M, K, xq, ld_q, scale, rowsum, sumsq, xq_natural};
+                                  cudaStream_t stream, const float* amax_in = nullptr,
+                                  float* amax_out = nullptr) {
+  QuantArgs a{src, gain, M, K, xq, ld_q, scale, rowsum, sumsq, xq_natural, amax_in, amax_out};
   cudaLaunchConfig_t cfg = {};
   // a CTA per token for up to 256 tokens or rows longer than 4096 values;
   // else a warp per token (measured faster for many short rows)
