@@ -206,6 +206,17 @@ def time_oracle_chain(layers, x_bits, repeats):
     return nbytes, dt
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline(target_s=10.0):
     from ternary_weight_linear_int8_b200 import inputs
     layers = oracle_decode_sample(2)
@@ -214,6 +225,7 @@ def cpu_baseline(target_s=10.0):
     reps = max(1, int(target_s / max(dt, 1e-3)))
     nbytes, dt = time_oracle_chain(layers, x, reps)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": blas_threads(),
+            "host_cores": os.cpu_count(), "cpu_model": cpu_model(),
             "kind": "oracle",
             "sample": f"{reps} passes over 2 of the 60 decode layers (up [6912,2560] then "
                       f"down [2560,6912]), M=1, oracle.linear from oracle-packed weights; "
@@ -245,7 +257,8 @@ def run_reference(args, world, rank):
                                "bounded sample: each step = 2 of the 60 layers "
                                "(up [6912,2560], down [2560,6912])",
                    "M": 1},
-        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": blas_threads(),
+                         "host_cores": os.cpu_count(), "cpu_model": cpu_model(), "kind": "oracle",
                          "sample": "each step: oracle.linear over 2 decode layers (one up, one "
                                    "down), M=1, oracle-packed weights"},
         "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -302,20 +315,22 @@ def time_graph(torch, graph, stream, steps, warmup, barrier=None):
     if barrier:
         barrier()
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    # an event between replays gives each step's time as well (median)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
     t0 = time.time()
     with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(steps):
+        ev[0].record(stream)
+        for i in range(steps):
             graph.replay()
-        e1.record(stream)
-    e1.synchronize()
+            ev[i + 1].record(stream)
+    ev[-1].synchronize()
     t1 = time.time()
     torch.cuda.synchronize()
     if barrier:
         barrier()
-    return e0.elapsed_time(e1), t0, t1
+    time_graph.last_median_ms = statistics.median(
+        ev[i].elapsed_time(ev[i + 1]) for i in range(steps))
+    return ev[0].elapsed_time(ev[-1]), t0, t1
 
 
 def secondary_measurements(B, inputs, torch, dev, stream, pk):
@@ -575,6 +590,7 @@ def run_ours(args, world, rank, local):
     sampler = ClockSampler(local)
     sampler.start()
     ms, t0, t1 = time_graph(torch, graph, stream, args.steps, args.warmup, barrier)
+    median_ms = time_graph.last_median_ms
     clocks = sampler.stop(t0, t1)
     ms = max_over_ranks(ms, dev)
     # the graph's output equals 60 eager bitnet_linear calls, bit for bit
@@ -639,6 +655,7 @@ def run_ours(args, world, rank, local):
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "ms_per_step_median": median_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
             "data": "synthetic",
             "config": {"workload": "2B-class decode GEMV chain, M=1: 30 layers x (up [6912,2560], "
