@@ -61,8 +61,8 @@ __device__ __forceinline__ void load4(const void* src, int64_t idx, float (&v)[4
 }
 
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-  return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
-         ((uint32_t)(d & 0xff) << 24);
+  return __byte_perm(__byte_perm((uint32_t)a, (uint32_t)b, 0x0040),
+                     __byte_perm((uint32_t)c, (uint32_t)d, 0x0040), 0x5410);
 }
 
 // One warp per token: two passes over the row (the second mostly from L1),
@@ -72,6 +72,9 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t m = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   pdl_wait();
+  // the kernel that consumes the codes may start its own set-up (and its
+  // weight loads) now; it reads the codes only after its dependency wait
+  pdl_launch_dependents();
   if (m < a.M) {
     const int64_t K = a.K;
     const int64_t base = m * K;
@@ -103,7 +106,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
         amax = fmaxf(amax, fabsf(g));
       }
     }
-    amax = warp_max(amax);
+    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
     if (a.sumsq) ss = warp_sum_d(ss);
     if (a.amax_out && lane == 0) a.amax_out[m] = amax;
     const float s = qscale(a.amax_in ? a.amax_in[m] : amax);
@@ -119,8 +122,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
         for (int c = 0; c < 8; ++c) {
           const float g0 = a.gain ? __fmul_rn(v0[c], a.gain[k + c]) : v0[c];
           const float g1 = a.gain ? __fmul_rn(v1[c], a.gain[k + 8 + c]) : v1[c];
-          q[c] = quant_code(g0, s);
-          q[8 + c] = quant_code(g1, s);
+          q[c] = quant_code_sat(g0, s);
+          q[8 + c] = quant_code_sat(g1, s);
         }
 #pragma unroll
         for (int c = 0; c < 16; ++c) rs += q[c];
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const float g = a.gain ? __fmul_rn(v[c], a.gain[k + c]) : v[c];
-          q[c] = quant_code(g, s);
+          q[c] = quant_code_sat(g, s);
           rs += q[c];
         }
         *reinterpret_cast<uint2*>(a.xq + m * a.ld_q + k) =
@@ -155,20 +158,19 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const float g = a.gain ? __fmul_rn(v[c], a.gain[k + c]) : v[c];
-          q[c] = quant_code(g, s);
+          q[c] = quant_code_sat(g, s);
           rs += q[c];
         }
         *reinterpret_cast<uint32_t*>(a.xq + m * a.ld_q + k) = pack4(q[0], q[1], q[2], q[3]);
       }
     }
-    rs = warp_sum_i(rs);
+    rs = __reduce_add_sync(0xffffffffu, rs);
     if (lane == 0) {
       a.scale[m] = s;
       if (a.rowsum) a.rowsum[m] = rs;
       if (a.sumsq) a.sumsq[m] = ss;
     }
   }
-  pdl_launch_dependents();
 }
 
 // One 256-thread CTA per token, block reductions through shared memory: for
@@ -187,6 +189,7 @@ __global__ void __launch_bounds__(256) quant_token_kernel(QuantArgs a) {
   const int64_t K = a.K;
   const int64_t base = m * K;
   pdl_wait();
+  pdl_launch_dependents();
   // pass 1: absmax of src * gain, sum of squares of src; groups of 8
   // (16-byte bf16 loads) when rows start 16-byte aligned, else of 4
   float amax = 0.f;
@@ -213,7 +216,7 @@ __global__ void __launch_bounds__(256) quant_token_kernel(QuantArgs a) {
       amax = fmaxf(amax, fabsf(g));
     }
   }
-  amax = warp_max(amax);
+  amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
   if (a.sumsq) ss = warp_sum_d(ss);
   if (lane == 0) {
     s_max[warp] = amax;
@@ -237,8 +240,8 @@ __global__ void __launch_bounds__(256) quant_token_kernel(QuantArgs a) {
       for (int c = 0; c < 8; ++c) {
         const float g0 = a.gain ? __fmul_rn(v0[c], a.gain[k + c]) : v0[c];
         const float g1 = a.gain ? __fmul_rn(v1[c], a.gain[k + 8 + c]) : v1[c];
-        q[c] = quant_code(g0, s);
-        q[8 + c] = quant_code(g1, s);
+        q[c] = quant_code_sat(g0, s);
+        q[8 + c] = quant_code_sat(g1, s);
       }
 #pragma unroll
       for (int c = 0; c < 16; ++c) rs += q[c];
@@ -259,13 +262,13 @@ __global__ void __launch_bounds__(256) quant_token_kernel(QuantArgs a) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const float g = a.gain ? __fmul_rn(v[c], a.gain[k + c]) : v[c];
-        q[c] = quant_code(g, s);
+        q[c] = quant_code_sat(g, s);
         rs += q[c];
       }
       *reinterpret_cast<uint32_t*>(a.xq + m * a.ld_q + k) = pack4(q[0], q[1], q[2], q[3]);
     }
   }
-  rs = warp_sum_i(rs);
+  rs = __reduce_add_sync(0xffffffffu, rs);
   if (lane == 0) s_rs[warp] = rs;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -280,7 +283,6 @@ __global__ void __launch_bounds__(256) quant_token_kernel(QuantArgs a) {
     if (a.rowsum) a.rowsum[m] = t;
     if (a.sumsq) a.sumsq[m] = d;
   }
-  pdl_launch_dependents();
 }
 
 }  // namespace bitnet
