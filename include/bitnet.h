@@ -127,9 +127,14 @@ BITNET_API bitnet_status bitnet_quant_act(const uint16_t* x, int64_t M, int64_t 
  * acc     [M,N] int32, written with the exact accumulators when non-NULL.
  * workspace  >= bitnet_linear_workspace_size(M, N, K) bytes (0 bytes, and a
  *         NULL workspace, are accepted when that size is 0).
- * Requires M >= 1, N >= 1, K >= 4, K % 4 == 0, K <= 524288.  M <= 8 with
- * K % 64 == 0 runs the fused decode kernel (activation quantisation in its
- * prologue, no workspace); larger M runs the tensor-core kernel.
+ * Requires M >= 1, N >= 1, K >= 4, K % 4 == 0, K <= 524288.  With
+ * K % 64 == 0: M <= 8 runs a fused decode kernel (activation quantisation in
+ * its prologue, no workspace); 9 <= M <= 32, on layers whose packed weights
+ * spread over the SMs fit in shared memory (K <= 65536), runs an absmax pass
+ * over x and the batched decode kernel (int8 mma.sync on weights held in
+ * shared memory, split K through an int32 scratch in the workspace that the
+ * kernel leaves zero); other M run the activation quantiser and the
+ * tensor-core kernel.
  */
 BITNET_API size_t bitnet_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 BITNET_API bitnet_status bitnet_linear(const uint8_t* packed, const float* gamma, int64_t N, int64_t K,
@@ -201,7 +206,10 @@ BITNET_API bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int
  *
  * The layers are launched one after the other on `stream`, each with the
  * kernel bitnet_linear would use (decode kernels start loading their weights
- * while the layer before them finishes).
+ * while the layer before them finishes).  When every layer runs the batched
+ * decode kernel (9..32 tokens), x gets one absmax pass and each layer then
+ * hands the per-token absmax of its bf16 outputs to the next through the
+ * workspace, so the chain is one launch per layer plus one.
  *
  * L        number of layers, >= 1.
  * packed, gamma, N, K, y   HOST arrays of L entries; packed[l], gamma[l] and

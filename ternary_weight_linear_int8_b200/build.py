@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libbitnet_b200.so")
-SOURCES = ["bitnet_all.cu", "common.cuh", "pack.cu", "quant.cu", "gemv.cu", "resident.cu", "gemm.cu", "a48.cu", "api.cu",
+SOURCES = ["bitnet_all.cu", "common.cuh", "pack.cu", "quant.cu", "gemv.cu", "resident.cu", "batched.cu", "gemm.cu", "a48.cu", "api.cu",
            "noalloc.cu"]
 
 NVCC_FLAGS = [

@@ -36,6 +36,15 @@ bitnet_status bitnet_gemm_launch(int mode, const int8_t* xq, const uint8_t* w0,
                                  const uint8_t* w1, GemmArgs a, int bn, int num_sms,
                                  cudaStream_t stream);
 int bitnet_gemm_pick_bn(int M, int N, int num_sms);
+int bitnet_batched_splits(int64_t M, int64_t N, int64_t K, int num_sms);
+bitnet_status bitnet_batched_launch(const uint8_t* w, const float* gamma, int N, int K,
+                                    const uint16_t* x, int M, uint16_t* y, float* y_f32,
+                                    int32_t* acc, const float* amax_in, unsigned* amax_out,
+                                    float* amax_clear, int32_t* ws_acc, int ldw,
+                                    unsigned* ws_cnt, int num_sms, cudaStream_t stream);
+bitnet_status bitnet_batched_prep_launch(const uint16_t* x, int M, int K, float* amax,
+                                         void* zero, size_t zero_bytes, int num_sms,
+                                         cudaStream_t stream);
 
 namespace {
 
@@ -161,6 +170,35 @@ size_t splitk_cnt_bytes(int64_t M, int64_t N) {
   return al256((size_t)((N + 127) / 128) * (size_t)((M + 31) / 32) * 4);
 }
 
+// Scratch of the batched decode kernel (4..64 tokens): per-token absmax
+// slots -- slot 2 is filled from x by the prep kernel, slots 0 and 1 with slot
+// 2 form the hand-over ring of a chain -- then one arrival counter per row
+// group (at most 256 groups) and the split-K sums [M, ldw].  Everything after slot 2 is zeroed by
+// the prep kernel and left zero by the layers.
+struct BatchedWs {
+  size_t slot[3], cnt, acc, total;
+  int64_t ldw;
+};
+
+// Token counts the batched decode kernel serves.  Measured on the 2B decode
+// chain it beats the streaming decode kernel's matrix-multiply items from 9
+// tokens on and the tensor-core GEMM path up to 32 tokens; outside that range
+// those paths stay.
+bool batched_shape(int64_t M, int64_t K) { return M >= 9 && M <= 32 && K % 64 == 0; }
+
+BatchedWs batched_ws_layout(int64_t M, int64_t N) {
+  BatchedWs w{};
+  const size_t a = al256((size_t)M * 4);
+  w.slot[2] = 0;
+  w.slot[0] = a;
+  w.slot[1] = 2 * a;
+  w.cnt = 3 * a;
+  w.ldw = ((N + 16 * 256 + 3) / 4) * 4;     // at most 256 row groups, each padded to 16
+  w.acc = w.cnt + al256(256 * 4);
+  w.total = w.acc + al256((size_t)M * (size_t)w.ldw * 4);
+  return w;
+}
+
 struct LinearWs {
   size_t xq, scale, rowsum, acc, total;
 };
@@ -168,7 +206,11 @@ struct LinearWs {
 LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
   LinearWs w{};
   const LinearPath p = linear_path(M, K);
-  if (p == kPathGemv) return w;
+  const size_t bt = batched_shape(M, K) ? batched_ws_layout(M, N).total : 0;
+  if (p == kPathGemv) {
+    w.total = bt;
+    return w;
+  }
   w.xq = 0;
   w.scale = al256((size_t)M * K);
   w.rowsum = w.scale + al256((size_t)M * 4);
@@ -176,6 +218,7 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
   w.total = w.acc;
   // split-K accumulators are reserved for every small-M tensor-core shape
   if (p == kPathGemm && M <= 256) w.total = w.acc + splitk_acc_bytes(M, N) + splitk_cnt_bytes(M, N);
+  if (bt > w.total) w.total = bt;
   return w;
 }
 
@@ -335,6 +378,20 @@ bitnet_status linear_enqueue(const uint8_t* packed, const float* gamma, int64_t 
                              cudaStream_t s) {
   bitnet_status st = BITNET_OK;
   const LinearPath p = linear_path(M, K);
+  const int bsplit = batched_shape(M, K) ? bitnet_batched_splits(M, N, K, d.num_sms) : 0;
+  if (bsplit > 0) {
+    // absmax of x (and a cleared split-K scratch), then the batched kernel
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const BatchedWs b = batched_ws_layout(M, N);
+    float* amax = reinterpret_cast<float*>(ws + b.slot[2]);
+    st = bitnet_batched_prep_launch(x, (int)M, (int)K, amax, ws + b.cnt,
+                                    bsplit > 1 ? b.total - b.cnt : 0, d.num_sms, s);
+    if (st != BITNET_OK) return st;
+    return bitnet_batched_launch(packed, gamma, (int)N, (int)K, x, (int)M, y, y_f32, acc, amax,
+                                 nullptr, nullptr, reinterpret_cast<int32_t*>(ws + b.acc),
+                                 (int)b.ldw, reinterpret_cast<unsigned*>(ws + b.cnt), d.num_sms,
+                                 s);
+  }
   if (p == kPathGemv) {
     if (bitnet_resident_fits(0, M, N, K, d.num_sms))
       return bitnet_resident_launch(0, packed, gamma, (int)N, (int)K, x, (int)M, y, y_f32, acc,
@@ -544,10 +601,44 @@ bitnet_status bitnet_linear_chain(int64_t L, const uint8_t* const* packed,
   DevInfo d;
   bitnet_status st = device_info(&d);
   if (st != BITNET_OK) return st;
-  // one launch per layer, in order on the stream (validated above, planned
-  // here); each decode kernel starts loading its weights while the layer
-  // before it finishes
   const cudaStream_t s = as_stream(stream);
+  // 4..64 tokens on layers that all fit the batched decode kernel: one absmax
+  // pass over x, then one launch per layer, each handing its outputs' per-token
+  // absmax to the next through a ring of three slots (layer l reads slot
+  // (l + 2) % 3, folds its own into slot l % 3 and clears slot (l + 1) % 3,
+  // which the layer before it has finished reading)
+  bool batched = batched_shape(M, K[0]);
+  bool any_split = false;
+  int64_t n_max = 0;
+  for (int64_t l = 0; batched && l < L; ++l) {
+    const int sp = bitnet_batched_splits(M, N[l], K[l], d.num_sms);
+    batched = sp > 0;
+    any_split = any_split || sp > 1;
+    if (N[l] > n_max) n_max = N[l];
+  }
+  if (batched) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const BatchedWs b = batched_ws_layout(M, n_max);
+    float* slot[3];
+    for (int i = 0; i < 3; ++i) slot[i] = reinterpret_cast<float*>(ws + b.slot[i]);
+    st = bitnet_batched_prep_launch(x, (int)M, (int)K[0], slot[2], ws + b.slot[0],
+                                    (any_split ? b.total : b.acc) - b.slot[0], d.num_sms, s);
+    if (st != BITNET_OK) return st;
+    for (int64_t l = 0; l < L; ++l) {
+      const bool last = l + 1 == L;
+      st = bitnet_batched_launch(
+          packed[l], gamma[l], (int)N[l], (int)K[l], l == 0 ? x : y[l - 1], (int)M, y[l],
+          nullptr, nullptr, slot[(l + 2) % 3],
+          last ? nullptr : reinterpret_cast<unsigned*>(slot[l % 3]),
+          last ? nullptr : slot[(l + 1) % 3], reinterpret_cast<int32_t*>(ws + b.acc),
+          (int)b.ldw, reinterpret_cast<unsigned*>(ws + b.cnt), d.num_sms, s);
+      if (st != BITNET_OK) return st;
+    }
+    return BITNET_OK;
+  }
+  // otherwise one launch per layer, in order on the stream (validated above,
+  // planned here); each decode kernel starts loading its weights while the
+  // layer before it finishes
   for (int64_t l = 0; l < L; ++l) {
     const LinearWs lw = linear_ws_layout(M, N[l], K[l]);
     st = linear_enqueue(packed[l], gamma[l], N[l], K[l], l == 0 ? x : y[l - 1], M, y[l], nullptr,

@@ -5,6 +5,7 @@
 #include "quant.cu"
 #include "gemv.cu"
 #include "resident.cu"
+#include "batched.cu"
 #include "gemm.cu"
 #include "a48.cu"
 #include "api.cu"
