@@ -141,9 +141,10 @@ def test_quant_act_matches_oracle(M, K, outl):
 # ------------------------------------------------------------- BitLinear
 # (M, N, K): resident decode kernel (M <= 3), streaming decode kernel (M <= 8),
 # batched decode kernel (9 <= M <= 32, with and without split K, ragged row
-# groups), tensor-core kernel (with and without split-K), and the ragged-K
-# kernel.
+# groups), tensor-core kernel (with and without split-K, ragged last token
+# tiles), and the ragged-K kernel.
 LINEAR_SHAPES = [
+    (512, 1000, 1024), (777, 400, 2560), (1000, 2560, 6912), (600, 257, 640),
     (24, 300, 2560), (32, 1000, 2560), (9, 6912, 64), (31, 5, 6912), (12, 4096, 4096),
     (20, 257, 640), (13, 2560, 2560), (7, 129, 192), (33, 1000, 2560), (48, 6912, 64),
     (1, 6912, 2560), (1, 2560, 6912), (8, 400, 512), (2, 7, 64), (3, 1, 128), (5, 33, 1024),
