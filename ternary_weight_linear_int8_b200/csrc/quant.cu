@@ -285,6 +285,107 @@ __global__ void __launch_bounds__(256) quant_token_kernel(QuantArgs a) {
   }
 }
 
+// quant_token_kernel for bf16 rows of at most 8192 values with K % 16 == 0:
+// each thread loads its (at most two) 16-value groups once and keeps them in
+// registers for the second pass, so a token costs one round of loads instead
+// of two.  Same arithmetic and outputs as quant_token_kernel.
+template <bool kPerm>
+__global__ void __launch_bounds__(256) quant_token_cached_kernel(QuantArgs a) {
+  constexpr int kGroups = 2;
+  __shared__ float s_max[8];
+  __shared__ double s_ss[8];
+  __shared__ int s_rs[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t m = blockIdx.x;
+  const int64_t K = a.K;
+  const uint16_t* row = static_cast<const uint16_t*>(a.src) + m * K;
+  pdl_wait();
+  pdl_launch_dependents();
+  uint4 v[kGroups][2];
+#pragma unroll
+  for (int i = 0; i < kGroups; ++i) {
+    const int64_t k = ((int64_t)threadIdx.x + 256 * i) * 16;
+    v[i][0] = v[i][1] = make_uint4(0, 0, 0, 0);
+    if (k < K) {
+      v[i][0] = *reinterpret_cast<const uint4*>(row + k);
+      v[i][1] = *reinterpret_cast<const uint4*>(row + k + 8);
+    }
+  }
+  auto value = [&](int i, int c) {             // value c of group i, as fp32
+    const uint4& h = v[i][c >> 3];
+    const int j = (c & 7) >> 1;
+    const uint32_t w = j == 0 ? h.x : j == 1 ? h.y : j == 2 ? h.z : h.w;
+    return __uint_as_float((c & 1) ? (w & 0xffff0000u) : (w << 16));
+  };
+  float amax = 0.f;
+  double ss = 0.0;
+#pragma unroll
+  for (int i = 0; i < kGroups; ++i) {
+    const int64_t k = ((int64_t)threadIdx.x + 256 * i) * 16;
+    if (k < K) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float x = value(i, c);
+        if (a.sumsq) ss += (double)x * (double)x;
+        const float g = a.gain ? __fmul_rn(x, a.gain[k + c]) : x;
+        amax = fmaxf(amax, fabsf(g));
+      }
+    }
+  }
+  amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+  if (a.sumsq) ss = warp_sum_d(ss);
+  if (lane == 0) {
+    s_max[warp] = amax;
+    s_ss[warp] = ss;
+  }
+  __syncthreads();
+  float am = s_max[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) am = fmaxf(am, s_max[w]);
+  if (a.amax_out && threadIdx.x == 0) a.amax_out[m] = am;
+  const float s = qscale(a.amax_in ? a.amax_in[m] : am);
+  int rs = 0;
+#pragma unroll
+  for (int i = 0; i < kGroups; ++i) {
+    const int64_t k = ((int64_t)threadIdx.x + 256 * i) * 16;
+    if (k < K) {
+      int q[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float x = value(i, c);
+        q[c] = quant_code_sat(a.gain ? __fmul_rn(x, a.gain[k + c]) : x, s);
+        rs += q[c];
+      }
+      const uint4 nat = make_uint4(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]),
+                                   pack4(q[8], q[9], q[10], q[11]), pack4(q[12], q[13], q[14], q[15]));
+      if (kPerm) {
+        // slot 4*t + b holds natural index 4*b + t
+        *reinterpret_cast<uint4*>(a.xq + m * a.ld_q + k) =
+            make_uint4(pack4(q[0], q[4], q[8], q[12]), pack4(q[1], q[5], q[9], q[13]),
+                       pack4(q[2], q[6], q[10], q[14]), pack4(q[3], q[7], q[11], q[15]));
+        if (a.xq_natural) *reinterpret_cast<uint4*>(a.xq_natural + m * K + k) = nat;
+      } else {
+        *reinterpret_cast<uint4*>(a.xq + m * a.ld_q + k) = nat;
+      }
+    }
+  }
+  rs = __reduce_add_sync(0xffffffffu, rs);
+  if (lane == 0) s_rs[warp] = rs;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    double d = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      t += s_rs[w];
+      d += s_ss[w];
+    }
+    a.scale[m] = s;
+    if (a.rowsum) a.rowsum[m] = t;
+    if (a.sumsq) a.sumsq[m] = d;
+  }
+}
+
 }  // namespace bitnet
 
 using namespace bitnet;
@@ -310,7 +411,13 @@ bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* ga
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (per_token) {
+  // bf16 rows of at most 8192 values in 16-byte-aligned groups of 16: the
+  // register-cached CTA-per-token kernel
+  const bool cached = per_token && !src_f32 && K % 16 == 0 && K <= 8192 && ld_q % 16 == 0;
+  if (cached) {
+    e = perm ? cudaLaunchKernelEx(&cfg, quant_token_cached_kernel<true>, a)
+             : cudaLaunchKernelEx(&cfg, quant_token_cached_kernel<false>, a);
+  } else if (per_token) {
     if (src_f32) {
       e = perm ? cudaLaunchKernelEx(&cfg, quant_token_kernel<true, true>, a)
                : cudaLaunchKernelEx(&cfg, quant_token_kernel<true, false>, a);
