@@ -43,6 +43,8 @@ __global__ void __launch_bounds__(kA48Threads) a48_quant_kernel(
   __shared__ int wrs4[kA48Threads / 32], wrs8[kA48Threads / 32];
   __shared__ int sel[4];        // B, J (threshold key), r (ties taken), flag
   pdl_wait();
+  // the consumer of the code rows reads them only after its dependency wait
+  pdl_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int m = blockIdx.x;
   const uint16_t* xr = x + (int64_t)m * K;
@@ -253,9 +255,18 @@ using namespace bitnet;
 bitnet_status bitnet_a48_quant_launch(const uint16_t* x, int64_t M, int64_t K, int64_t n_out,
                                       int8_t* rows, float* scale, int32_t* rowsum, int8_t* q4n,
                                       int8_t* q8n, float* s4, float* s8, cudaStream_t stream) {
-  a48_quant_kernel<<<(unsigned)M, kA48Threads, 0, stream>>>(x, (int)K, (int)n_out, rows, scale,
-                                                            rowsum, q4n, q8n, s4, s8);
-  return cudaGetLastError() == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)M);
+  cfg.blockDim = dim3(kA48Threads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, a48_quant_kernel, x, (int)K, (int)n_out, rows,
+                                           scale, rowsum, q4n, q8n, s4, s8);
+  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
 
 bitnet_status bitnet_a48_combine_launch(const int32_t* acc2, const float* scale,

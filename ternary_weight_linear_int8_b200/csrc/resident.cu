@@ -34,11 +34,18 @@
 //    holds x0 (c0 - 1) + x1 (c1 - 1) at c0 + 4 c1; a packed nibble is exactly
 //    that index, so a byte costs two lookups.  One token; one CTA per SM (the
 //    tables take 16 K bytes).
+//  * kResA48 -- the ternary I2_S weights on one token in BitNet a4.8 form
+//    (youngju.dev page, section "BitNet a4.8：ハイブリッド量子化戦略"): the
+//    token arrives already quantised as two code rows in the kernel order,
+//    the 4-bit codes of the ordinary values and the 8-bit codes of the
+//    largest ones, with their scales and row sums (bitnet_quant_act_a48's
+//    rows); the dp4a items run on both rows and the epilogue forms
+//    fp32(acc4) (gamma / s4) + fp32(acc8) (gamma / s8).
 #include "common.cuh"
 
 namespace bitnet {
 
-enum ResFmt : int { kResI2S = 0, kResW1 = 1, kResTL2 = 2 };
+enum ResFmt : int { kResI2S = 0, kResW1 = 1, kResTL2 = 2, kResA48 = 3 };
 
 struct ResidentParams {
   const uint8_t* w;        // packed [N, K/4] (I2_S) or [N, K/8] (sign bits)
@@ -54,6 +61,10 @@ struct ResidentParams {
   uint32_t lut_off;        // pair tables (kResTL2)
   uint32_t acc_off;
   uint32_t w_off;
+  const int8_t* xq_in;     // kResA48: code rows [2][K] (kernel order)
+  const float* s_in;       // kResA48: their scales [2]
+  const int32_t* rs_in;    // kResA48: their row sums [2]
+  int32_t* acc8;           // kResA48: optional [N] (acc holds acc4)
 };
 
 constexpr int kResWarps = 16;
@@ -124,6 +135,16 @@ __global__ void __launch_bounds__(kResThreads, FMT == kResTL2 ? 1 : 2)
 
   pdl_wait();
 
+  int rtot[MM];
+  if constexpr (FMT == kResA48) {
+    // the two code rows as they are, their dequant factors and row sums
+    for (int i = tid * 16; i < M * K; i += kResThreads * 16)
+      sts_v4(smem_u32(xq + i), *reinterpret_cast<const uint4*>(p.xq_in + i));
+    if (tid < M) tok_d[tid] = __fdiv_rn(*p.gamma, p.s_in[tid]);
+#pragma unroll
+    for (int m = 0; m < MM; ++m) rtot[m] = m < M ? p.rs_in[m] : 0;
+    __syncthreads();
+  } else {
   // ---- per-token absmax (pass 1) and quantisation (pass 2).  A thread owns
   // (token, 8 consecutive values) pairs; up to two pairs per thread stay in
   // registers between the passes, otherwise pass 2 loads them again.
@@ -277,11 +298,11 @@ __global__ void __launch_bounds__(kResThreads, FMT == kResTL2 ? 1 : 2)
     __syncthreads();
   }
   // each token's row sum (identical in every thread)
-  int rtot[MM];
 #pragma unroll
   for (int m = 0; m < MM; ++m) {
     const int v = (m < M && lane < kResWarps) ? red_i[lane * kResMaxTok + m] : 0;
     rtot[m] = __reduce_add_sync(0xffffffffu, v);
+  }
   }
 
   // ---- products: items (4-row block b, K-slice q), dealt round robin to the
@@ -298,11 +319,24 @@ __global__ void __launch_bounds__(kResThreads, FMT == kResTL2 ? 1 : 2)
     if (p.y_f32) p.y_f32[o] = y32;
     if (p.acc) p.acc[o] = ac;
   };
+  // kResA48: one token from its two code rows (4-bit, then 8-bit), the two
+  // fp32 products added in that order
+  auto finish_a48 = [&](int r, int v4, int v8) {
+    const int a4 = v4 - rtot[0], a8 = v8 - rtot[MM > 1 ? 1 : 0];
+    const float y32 = __fadd_rn(__fmul_rn(__int2float_rn(a4), tok_d[0]),
+                                __fmul_rn(__int2float_rn(a8), tok_d[1]));
+    const int64_t o = n0 + r;
+    p.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y32));
+    if (p.y_f32) p.y_f32[o] = y32;
+    if (p.acc) p.acc[o] = a4;
+    if (p.acc8) p.acc8[o] = a8;
+  };
   const uint32_t x_addr = smem_u32(xq), w_addr = smem_u32(wsm);
   const uint32_t lut_addr = smem_u32(g_res_smem + p.lut_off);
   bool ok = true;
   int pc = 0;            // weight piece of the current block (blocks only grow)
-  constexpr int kUnroll = (MT == 1 && FMT == kResI2S) ? 4 : 2;
+  constexpr bool kTern = FMT == kResI2S || FMT == kResA48;   // I2_S codes, dp4a
+  constexpr int kUnroll = (MT == 1 && kTern) ? 4 : 2;
   const int wkl = __ffs(WK) - 1;
   const int nitems = nblk * WK;
   for (int it = warp; it < nitems; it += kResWarps) {
@@ -329,7 +363,7 @@ __global__ void __launch_bounds__(kResThreads, FMT == kResTL2 ? 1 : 2)
         uint32_t w[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) w[r] = lds_u32(rowa[r] + 4u * j);
-        if constexpr (FMT == kResI2S) {
+        if constexpr (kTern) {
           uint4 xv[MT];
 #pragma unroll
           for (int t = 0; t < MT; ++t) xv[t] = lds_v4(xt + (uint32_t)(t * K) + 16u * j);
@@ -388,11 +422,12 @@ __global__ void __launch_bounds__(kResThreads, FMT == kResTL2 ? 1 : 2)
           }
         }
       }
-      if constexpr (MT == 1 && FMT == kResI2S) {
+      if constexpr (MT == 1 && kTern) {
 #pragma unroll
         for (int r = 0; r < 4; ++r)
           acc_r[r][0] = acc4[r][0] + (acc4[r][1] >> 2) + (acc4[r][2] >> 4) + (acc4[r][3] >> 6);
       }
+      int tots[MT];
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
         const int v[4] = {acc_r[0][t], acc_r[1][t], acc_r[2][t], acc_r[3][t]};
@@ -404,19 +439,29 @@ __global__ void __launch_bounds__(kResThreads, FMT == kResTL2 ? 1 : 2)
         tot += __shfl_xor_sync(0xffffffffu, tot, 4);
         tot += __shfl_xor_sync(0xffffffffu, tot, 2);
         tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+        tots[t] = tot;
         const int r = 4 * b + (lane >> 3), m = tg + t;
         if ((lane & 7) == 0 && m < M && r < R) {
-          if (WK == 1) finish(r, m, tot);
-          else atomicAdd(&accs[r * kResMaxTok + m], tot);
+          if (WK > 1) atomicAdd(&accs[r * kResMaxTok + m], tot);
+          else if constexpr (FMT != kResA48) finish(r, m, tot);
         }
+      }
+      if constexpr (FMT == kResA48) {
+        const int r = 4 * b + (lane >> 3);
+        if (WK == 1 && (lane & 7) == 0 && r < R) finish_a48(r, tots[0], tots[MT - 1]);
       }
     }
   }
   if (WK > 1) {
     __syncthreads();
-    for (int o = tid; o < R * M; o += kResThreads) {
-      const int r = MM == 1 ? o : o / M, m = o - r * M;
-      finish(r, m, accs[r * kResMaxTok + m]);
+    if constexpr (FMT == kResA48) {
+      for (int r = tid; r < R; r += kResThreads)
+        finish_a48(r, accs[r * kResMaxTok], accs[r * kResMaxTok + 1]);
+    } else {
+      for (int o = tid; o < R * M; o += kResThreads) {
+        const int r = MM == 1 ? o : o / M, m = o - r * M;
+        finish(r, m, accs[r * kResMaxTok + m]);
+      }
     }
   }
   if (!ok) {
@@ -514,7 +559,9 @@ bitnet_status bitnet_resident_launch(int fmt, const uint8_t* w, const float* gam
   if (!plan_resident(fmt, M, N, K, num_sms, &pl)) return BITNET_ERR_UNSUPPORTED;
   pl.p.w = w; pl.p.gamma = gamma; pl.p.x = x; pl.p.y = y; pl.p.y_f32 = y_f32; pl.p.acc = acc;
   cudaError_t e;
-  if (fmt == kResTL2) {
+  if (fmt == kResA48) {
+    return BITNET_ERR_UNSUPPORTED;             // bitnet_resident_a48_launch
+  } else if (fmt == kResTL2) {
     e = launch_resident_t<kResTL2, 1, 1>(pl, stream);
   } else if (fmt == kResW1) {
     if (M == 1) e = launch_resident_t<kResW1, 1, 1>(pl, stream);
@@ -525,5 +572,25 @@ bitnet_status bitnet_resident_launch(int fmt, const uint8_t* w, const float* gam
     else if (M == 2) e = launch_resident_t<kResI2S, 2, 2>(pl, stream);
     else e = launch_resident_t<kResI2S, 2, 4>(pl, stream);
   }
+  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
+
+// One token of BitNet a4.8 on the resident kernel: rows = the token's two
+// code rows [2][K] in the kernel order (q4 then q8), scale/rowsum their [2]
+// scales and row sums (bitnet_quant_act_a48's layout); acc4/acc8 optional.
+bool bitnet_resident_a48_fits(int64_t N, int64_t K, int num_sms) {
+  return bitnet_resident_fits(kResA48, 2, N, K, num_sms);
+}
+
+bitnet_status bitnet_resident_a48_launch(const uint8_t* w, const float* gamma, int N, int K,
+                                         const int8_t* rows, const float* scale,
+                                         const int32_t* rowsum, uint16_t* y, float* y_f32,
+                                         int32_t* acc4, int32_t* acc8, int num_sms,
+                                         cudaStream_t stream) {
+  ResidentPlan pl;
+  if (!plan_resident(kResA48, 2, N, K, num_sms, &pl)) return BITNET_ERR_UNSUPPORTED;
+  pl.p.w = w; pl.p.gamma = gamma; pl.p.y = y; pl.p.y_f32 = y_f32; pl.p.acc = acc4;
+  pl.p.xq_in = rows; pl.p.s_in = scale; pl.p.rs_in = rowsum; pl.p.acc8 = acc8;
+  const cudaError_t e = launch_resident_t<kResA48, 2, 2>(pl, stream);
   return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
