@@ -29,6 +29,40 @@ constexpr int kA48Threads = 512;
 // the sign cleared.
 __device__ __forceinline__ uint32_t mag_key(uint32_t bits16) { return bits16 & 0x7fffu; }
 
+// One warp over a histogram of 32 * PER bins (bin b counts keys whose digit
+// is b): the highest bin B whose suffix count (keys with digit >= B, plus
+// `above_in` keys above all of them) reaches `need`, and the count above B.
+// Lane l holds bins [PER l, PER l + PER); a suffix scan over the lanes and
+// one ballot find the lane that holds B, which then walks its own bins.
+template <int PER>
+__device__ __forceinline__ void warp_select_bin(const unsigned* hist, int need, int above_in,
+                                                int lane, int& B, int& above) {
+  int loc = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) loc += (int)hist[PER * lane + i];
+  int suf = loc;                       // sum over lanes >= lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += v;
+  }
+  const unsigned ok = __ballot_sync(0xffffffffu, above_in + suf >= need);
+  // lanes 0..L satisfy it (suffix counts do not increase with the lane)
+  const int L = ok ? 31 - __clz(ok) : 0;
+  const int suf_above = __shfl_sync(0xffffffffu, suf - loc, L);   // lanes > L
+  if (lane == L) {
+    int acc = above_in + suf_above, b = PER * L;
+    for (int i = PER - 1; i >= 0; --i) {
+      if (acc + (int)hist[PER * L + i] >= need) { b = PER * L + i; break; }
+      acc += (int)hist[PER * L + i];
+    }
+    B = b;
+    above = acc;
+  }
+  B = __shfl_sync(0xffffffffu, B, L);
+  above = __shfl_sync(0xffffffffu, above, L);
+}
+
 // Quantise one token per CTA.  Outputs (any may be null except the scales):
 //   rows   [2M, K] int8 in the kernels' K order (row 2m: q4, row 2m+1: q8)
 //   scale  [2M] fp32 (s4, s8), rowsum [2M] int32
@@ -76,14 +110,13 @@ __global__ void __launch_bounds__(kA48Threads) a48_quant_kernel(
       for (int i = 0; i < 8; ++i) atomicAdd(&hist[k[i] >> 7], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      int above = 0, B = 0;
-      for (int bb = 255; bb >= 0; --bb) {
-        if (above + (int)hist[bb] >= n_out) { B = bb; break; }
-        above += (int)hist[bb];
+    if (warp == 0) {
+      int B = 0, above = 0;
+      warp_select_bin<8>(hist, n_out, 0, lane, B, above);
+      if (lane == 0) {
+        sel[0] = B;
+        sel[1] = above;
       }
-      sel[0] = B;
-      sel[1] = above;
     }
     __syncthreads();
     const int B = sel[0];
@@ -99,14 +132,13 @@ __global__ void __launch_bounds__(kA48Threads) a48_quant_kernel(
         if ((int)(k[i] >> 7) == B) atomicAdd(&hist[k[i] & 127u], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      int J = 0;
-      for (int j = 127; j >= 0; --j) {
-        if (above + (int)hist[j] >= n_out) { J = j; break; }
-        above += (int)hist[j];
+    if (warp == 0) {
+      int J = 0, ab = 0;
+      warp_select_bin<4>(hist, n_out, above, lane, J, ab);
+      if (lane == 0) {
+        sel[2] = (B << 7) | J;
+        sel[3] = n_out - ab;    // values equal to T taken, in channel order
       }
-      sel[2] = (B << 7) | J;
-      sel[3] = n_out - above;   // values equal to T taken, in channel order
     }
     __syncthreads();
     T = sel[2];
