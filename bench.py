@@ -462,8 +462,8 @@ def secondary_measurements(B, inputs, torch, dev, stream, pk):
     out["decode_chain_a48_M1"] = {"GB/s": round(nbytes / t / 1e9, 1),
                                   "us_per_layer": round(t / 60 * 1e6, 3),
                                   "frac_hbm": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4),
-                                  "launches_per_layer": "a4.8 quantiser, resident kernel on "
-                                                        "the two code rows"}
+                                  "launches_per_layer": "one: the resident kernel quantises the "
+                                                        "token into its two code rows"}
     del g, wsa
     # FFN 100B-class: two distinct blocks rotated
     H, I = 8192, 28672

@@ -346,10 +346,11 @@ BITNET_API bitnet_status bitnet_linear_tl2(const uint8_t* packed, const float* g
  * bitnet_linear_a48: packed [N,K/4], gamma as bitnet_linear; y [M,N] bf16
  * bits; y_f32, acc4, acc8 optional [M,N]; workspace >=
  * bitnet_linear_a48_workspace_size(M, N, K) bytes.  Requires K % 64 == 0,
- * 0 <= n_out <= K.  Runs the a4.8 quantiser (one CTA per token), then for
- * one token whose weight slices fit shared memory the resident decode kernel
- * on its two code rows (combined in its epilogue), otherwise the tensor-core
- * kernel on the 2M code rows and a combine kernel.
+ * 0 <= n_out <= K.  One token whose weight slices fit shared memory: the
+ * resident decode kernel alone, quantising the token into its two code rows
+ * in every CTA and combining them in its epilogue; otherwise the a4.8
+ * quantiser (one CTA per token), the tensor-core kernel on the 2M code rows
+ * and a combine kernel.
  */
 BITNET_API bitnet_status bitnet_quant_act_a48(const uint16_t* x, int64_t M, int64_t K,
                                               int64_t n_out, int8_t* q4, float* s4, int8_t* q8,

@@ -18,7 +18,9 @@
 // values equal to it by channel, block maxima of the two parts, then the
 // two code rows); the tensor-core kernel on the 2M rows (q4 of token m at
 // row 2m, q8 at row 2m + 1), which writes the exact accumulators; and a
-// combine kernel for y.
+// combine kernel for y.  For one token the resident decode kernel runs the
+// same per-token quantisation (a48_quant_token) in every CTA's prologue and
+// combines the two rows in its epilogue.
 #include "common.cuh"
 
 namespace bitnet {
@@ -63,25 +65,23 @@ __device__ __forceinline__ void warp_select_bin(const unsigned* hist, int need, 
   above = __shfl_sync(0xffffffffu, above, L);
 }
 
-// Quantise one token per CTA.  Outputs (any may be null except the scales):
-//   rows   [2M, K] int8 in the kernels' K order (row 2m: q4, row 2m+1: q8)
-//   scale  [2M] fp32 (s4, s8), rowsum [2M] int32
-//   q4n, q8n [M, K] int8 natural order (for the standalone quantiser)
-//   s4, s8 [M] fp32
-__global__ void __launch_bounds__(kA48Threads) a48_quant_kernel(
-    const uint16_t* __restrict__ x, int K, int n_out, int8_t* rows, float* scale, int32_t* rowsum,
-    int8_t* q4n, int8_t* q8n, float* s4o, float* s8o) {
+// One token's a4.8 codes, computed by a block of kA48Threads threads (every
+// thread of the block calls it).  Writes, where given (global or shared
+// memory): row4 / row8 [K] in the kernels' K order, q4n / q8n [K] in natural
+// order; returns the scales and row sums to every thread.
+struct A48Token {
+  float s4, s8;
+  int rs4, rs8;
+};
+
+__device__ A48Token a48_quant_token(const uint16_t* __restrict__ xr, int K, int n_out,
+                                    int8_t* row4, int8_t* row8, int8_t* q4n, int8_t* q8n) {
   __shared__ unsigned hist[256];
   __shared__ unsigned wsum[kA48Threads / 32];
   __shared__ float wmax4[kA48Threads / 32], wmax8[kA48Threads / 32];
   __shared__ int wrs4[kA48Threads / 32], wrs8[kA48Threads / 32];
   __shared__ int sel[4];        // B, J (threshold key), r (ties taken), flag
-  pdl_wait();
-  // the consumer of the code rows reads them only after its dependency wait
-  pdl_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int m = blockIdx.x;
-  const uint16_t* xr = x + (int64_t)m * K;
   const int npiece = K >> 3;                               // 8-value pieces
   const int cp = (npiece + kA48Threads - 1) / kA48Threads;  // pieces per thread
   const int p0 = min(npiece, tid * cp), p1 = min(npiece, p0 + cp);
@@ -198,8 +198,6 @@ __global__ void __launch_bounds__(kA48Threads) a48_quant_kernel(
   // ---- quantise both parts (the tie ranks are recomputed in the same order)
   rank = wbase + incl - ties;
   int rs4 = 0, rs8 = 0;
-  int8_t* row4 = rows ? rows + (int64_t)(2 * m) * K : nullptr;
-  int8_t* row8 = rows ? rows + (int64_t)(2 * m + 1) * K : nullptr;
   for (int pc = p0; pc < p1; ++pc) {
     uint32_t k[8], b[8];
     load8(pc, k, b);
@@ -220,11 +218,11 @@ __global__ void __launch_bounds__(kA48Threads) a48_quant_kernel(
     if (q4n) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        q4n[(int64_t)m * K + k0 + i] = (int8_t)q4[i];
-        q8n[(int64_t)m * K + k0 + i] = (int8_t)q8[i];
+        q4n[k0 + i] = (int8_t)q4[i];
+        q8n[k0 + i] = (int8_t)q8[i];
       }
     }
-    if (rows) {
+    if (row4) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int64_t kk = perm_k(k0 + i);
@@ -240,22 +238,42 @@ __global__ void __launch_bounds__(kA48Threads) a48_quant_kernel(
     wrs8[warp] = rs8;
   }
   __syncthreads();
-  if (tid == 0) {
-    int t4 = 0, t8 = 0;
-    for (int w = 0; w < kA48Threads / 32; ++w) {
-      t4 += wrs4[w];
-      t8 += wrs8[w];
-    }
+  A48Token t{s4, s8, 0, 0};
+  for (int w = 0; w < kA48Threads / 32; ++w) {
+    t.rs4 += wrs4[w];
+    t.rs8 += wrs8[w];
+  }
+  __syncthreads();                     // the block's shared scratch is free again
+  return t;
+}
+
+// Quantise one token per CTA.  Outputs (any may be null except the scales):
+//   rows   [2M, K] int8 in the kernels' K order (row 2m: q4, row 2m+1: q8)
+//   scale  [2M] fp32 (s4, s8), rowsum [2M] int32
+//   q4n, q8n [M, K] int8 natural order (for the standalone quantiser)
+//   s4, s8 [M] fp32
+__global__ void __launch_bounds__(kA48Threads) a48_quant_kernel(
+    const uint16_t* __restrict__ x, int K, int n_out, int8_t* rows, float* scale, int32_t* rowsum,
+    int8_t* q4n, int8_t* q8n, float* s4o, float* s8o) {
+  pdl_wait();
+  // the consumer of the code rows reads them only after its dependency wait
+  pdl_launch_dependents();
+  const int m = blockIdx.x;
+  const A48Token t = a48_quant_token(
+      x + (int64_t)m * K, K, n_out, rows ? rows + (int64_t)(2 * m) * K : nullptr,
+      rows ? rows + (int64_t)(2 * m + 1) * K : nullptr, q4n ? q4n + (int64_t)m * K : nullptr,
+      q8n ? q8n + (int64_t)m * K : nullptr);
+  if (threadIdx.x == 0) {
     if (scale) {
-      scale[2 * m] = s4;
-      scale[2 * m + 1] = s8;
+      scale[2 * m] = t.s4;
+      scale[2 * m + 1] = t.s8;
     }
     if (rowsum) {
-      rowsum[2 * m] = t4;
-      rowsum[2 * m + 1] = t8;
+      rowsum[2 * m] = t.rs4;
+      rowsum[2 * m + 1] = t.rs8;
     }
-    if (s4o) s4o[m] = s4;
-    if (s8o) s8o[m] = s8;
+    if (s4o) s4o[m] = t.s4;
+    if (s8o) s8o[m] = t.s8;
   }
 }
 

@@ -19,10 +19,10 @@ bitnet_status bitnet_decode_launch(const DecodeOp& op, int M, int num_sms, cudaS
 bool bitnet_resident_fits(int fmt, int64_t M, int64_t N, int64_t K, int num_sms);
 bool bitnet_resident_a48_fits(int64_t N, int64_t K, int num_sms);
 bitnet_status bitnet_resident_a48_launch(const uint8_t* w, const float* gamma, int N, int K,
-                                         const int8_t* rows, const float* scale,
-                                         const int32_t* rowsum, uint16_t* y, float* y_f32,
-                                         int32_t* acc4, int32_t* acc8, int num_sms,
-                                         cudaStream_t stream);
+                                         const uint16_t* x, int n_out, const int8_t* rows,
+                                         const float* scale, const int32_t* rowsum, uint16_t* y,
+                                         float* y_f32, int32_t* acc4, int32_t* acc8,
+                                         int num_sms, cudaStream_t stream);
 bitnet_status bitnet_resident_launch(int fmt, const uint8_t* w, const float* gamma, int N, int K,
                                      const uint16_t* x, int M, uint16_t* y, float* y_f32,
                                      int32_t* acc, int num_sms, cudaStream_t stream);
@@ -770,14 +770,15 @@ bitnet_status bitnet_linear_a48(const uint8_t* packed, const float* gamma, int64
   float* sc = reinterpret_cast<float*>(ws + L.scale);
   int32_t* rs = reinterpret_cast<int32_t*>(ws + L.rowsum);
   int32_t* acc2 = reinterpret_cast<int32_t*>(ws + L.acc2);
+  // one token whose weight slices fit shared memory: the resident kernel
+  // quantises the token itself (every CTA) and combines the two code rows in
+  // its epilogue; one launch
+  if (M == 1 && bitnet_resident_a48_fits(N, K, d.num_sms))
+    return bitnet_resident_a48_launch(packed, gamma, (int)N, (int)K, x, (int)n_out, nullptr,
+                                      nullptr, nullptr, y, y_f32, acc4, acc8, d.num_sms, s);
   st = bitnet_a48_quant_launch(x, M, K, n_out, rows, sc, rs, nullptr, nullptr, nullptr, nullptr,
                                s);
   if (st != BITNET_OK) return st;
-  // one token whose weight slices fit shared memory: the resident kernel on
-  // the two code rows, combined in its epilogue
-  if (M == 1 && bitnet_resident_a48_fits(N, K, d.num_sms))
-    return bitnet_resident_a48_launch(packed, gamma, (int)N, (int)K, rows, sc, rs, y, y_f32, acc4,
-                                      acc8, d.num_sms, s);
   // the integer products of all 2M code rows on the tensor-core kernel
   const int64_t M2 = 2 * M;
   const int bn = bitnet_gemm_pick_bn((int)M2, (int)N, d.num_sms);

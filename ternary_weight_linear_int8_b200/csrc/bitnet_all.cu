@@ -4,9 +4,9 @@
 #include "pack.cu"
 #include "quant.cu"
 #include "gemv.cu"
+#include "a48.cu"
 #include "resident.cu"
 #include "batched.cu"
 #include "gemm.cu"
-#include "a48.cu"
 #include "api.cu"
 #include "noalloc.cu"

@@ -36,10 +36,11 @@
 //    tables take 16 K bytes).
 //  * kResA48 -- the ternary I2_S weights on one token in BitNet a4.8 form
 //    (youngju.dev page, section "BitNet a4.8：ハイブリッド量子化戦略"): the
-//    token arrives already quantised as two code rows in the kernel order,
-//    the 4-bit codes of the ordinary values and the 8-bit codes of the
-//    largest ones, with their scales and row sums (bitnet_quant_act_a48's
-//    rows); the dp4a items run on both rows and the epilogue forms
+//    token becomes two code rows in the kernel order, the 4-bit codes of the
+//    ordinary values and the 8-bit codes of the largest ones, with their
+//    scales and row sums -- computed by every CTA from the bf16 token in its
+//    prologue (the a4.8 selection, the same in every CTA), or given already
+//    quantised; the dp4a items run on both rows and the epilogue forms
 //    fp32(acc4) (gamma / s4) + fp32(acc8) (gamma / s8).
 #include "common.cuh"
 
@@ -61,7 +62,9 @@ struct ResidentParams {
   uint32_t lut_off;        // pair tables (kResTL2)
   uint32_t acc_off;
   uint32_t w_off;
-  const int8_t* xq_in;     // kResA48: code rows [2][K] (kernel order)
+  const int8_t* xq_in;     // kResA48: code rows [2][K] (kernel order), or null:
+                           // quantise x with n_out 8-bit values in the prologue
+  int n_out;
   const float* s_in;       // kResA48: their scales [2]
   const int32_t* rs_in;    // kResA48: their row sums [2]
   int32_t* acc8;           // kResA48: optional [N] (acc holds acc4)
@@ -137,12 +140,26 @@ __global__ void __launch_bounds__(kResThreads, FMT == kResTL2 ? 1 : 2)
 
   int rtot[MM];
   if constexpr (FMT == kResA48) {
-    // the two code rows as they are, their dequant factors and row sums
-    for (int i = tid * 16; i < M * K; i += kResThreads * 16)
-      sts_v4(smem_u32(xq + i), *reinterpret_cast<const uint4*>(p.xq_in + i));
-    if (tid < M) tok_d[tid] = __fdiv_rn(*p.gamma, p.s_in[tid]);
+    static_assert(kResThreads == kA48Threads, "the a4.8 selection runs on the whole block");
+    if (p.xq_in) {
+      // the two code rows as they are, their dequant factors and row sums
+      for (int i = tid * 16; i < M * K; i += kResThreads * 16)
+        sts_v4(smem_u32(xq + i), *reinterpret_cast<const uint4*>(p.xq_in + i));
+      if (tid < M) tok_d[tid] = __fdiv_rn(*p.gamma, p.s_in[tid]);
 #pragma unroll
-    for (int m = 0; m < MM; ++m) rtot[m] = m < M ? p.rs_in[m] : 0;
+      for (int m = 0; m < MM; ++m) rtot[m] = m < M ? p.rs_in[m] : 0;
+    } else {
+      // the token's a4.8 selection and codes (identical in every CTA),
+      // straight into the shared code rows
+      const A48Token t = a48_quant_token(p.x, K, p.n_out, reinterpret_cast<int8_t*>(xq),
+                                         reinterpret_cast<int8_t*>(xq + K), nullptr, nullptr);
+      if (tid == 0) {
+        tok_d[0] = __fdiv_rn(*p.gamma, t.s4);
+        tok_d[1] = __fdiv_rn(*p.gamma, t.s8);
+      }
+      rtot[0] = t.rs4;
+      rtot[MM - 1] = t.rs8;
+    }
     __syncthreads();
   } else {
   // ---- per-token absmax (pass 1) and quantisation (pass 2).  A thread owns
@@ -575,21 +592,24 @@ bitnet_status bitnet_resident_launch(int fmt, const uint8_t* w, const float* gam
   return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
 
-// One token of BitNet a4.8 on the resident kernel: rows = the token's two
-// code rows [2][K] in the kernel order (q4 then q8), scale/rowsum their [2]
-// scales and row sums (bitnet_quant_act_a48's layout); acc4/acc8 optional.
+// One token of BitNet a4.8 on the resident kernel: either rows = the token's
+// two code rows [2][K] in the kernel order (q4 then q8) with scale/rowsum
+// their [2] scales and row sums (bitnet_quant_act_a48's layout), or rows =
+// null and the kernel quantises the bf16 token x [K] itself with n_out 8-bit
+// values; acc4/acc8 optional.
 bool bitnet_resident_a48_fits(int64_t N, int64_t K, int num_sms) {
   return bitnet_resident_fits(kResA48, 2, N, K, num_sms);
 }
 
 bitnet_status bitnet_resident_a48_launch(const uint8_t* w, const float* gamma, int N, int K,
-                                         const int8_t* rows, const float* scale,
-                                         const int32_t* rowsum, uint16_t* y, float* y_f32,
-                                         int32_t* acc4, int32_t* acc8, int num_sms,
-                                         cudaStream_t stream) {
+                                         const uint16_t* x, int n_out, const int8_t* rows,
+                                         const float* scale, const int32_t* rowsum, uint16_t* y,
+                                         float* y_f32, int32_t* acc4, int32_t* acc8,
+                                         int num_sms, cudaStream_t stream) {
   ResidentPlan pl;
   if (!plan_resident(kResA48, 2, N, K, num_sms, &pl)) return BITNET_ERR_UNSUPPORTED;
   pl.p.w = w; pl.p.gamma = gamma; pl.p.y = y; pl.p.y_f32 = y_f32; pl.p.acc = acc4;
+  pl.p.x = x; pl.p.n_out = n_out;
   pl.p.xq_in = rows; pl.p.s_in = scale; pl.p.rs_in = rowsum; pl.p.acc8 = acc8;
   const cudaError_t e = launch_resident_t<kResA48, 2, 2>(pl, stream);
   return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
