@@ -252,12 +252,19 @@ __device__ A48Token a48_quant_token(const uint16_t* __restrict__ xr, int K, int 
 //   scale  [2M] fp32 (s4, s8), rowsum [2M] int32
 //   q4n, q8n [M, K] int8 natural order (for the standalone quantiser)
 //   s4, s8 [M] fp32
+//   zero   [zero16] 16-byte words cleared after the dependency wait (the
+//          split-K scratch of the GEMM that follows), or null
 __global__ void __launch_bounds__(kA48Threads) a48_quant_kernel(
     const uint16_t* __restrict__ x, int K, int n_out, int8_t* rows, float* scale, int32_t* rowsum,
-    int8_t* q4n, int8_t* q8n, float* s4o, float* s8o) {
+    int8_t* q4n, int8_t* q8n, float* s4o, float* s8o, uint4* zero, int64_t zero16) {
   pdl_wait();
   // the consumer of the code rows reads them only after its dependency wait
   pdl_launch_dependents();
+  if (zero) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < zero16; i += stride)
+      zero[i] = make_uint4(0, 0, 0, 0);
+  }
   const int m = blockIdx.x;
   const A48Token t = a48_quant_token(
       x + (int64_t)m * K, K, n_out, rows ? rows + (int64_t)(2 * m) * K : nullptr,
@@ -304,7 +311,8 @@ using namespace bitnet;
 
 bitnet_status bitnet_a48_quant_launch(const uint16_t* x, int64_t M, int64_t K, int64_t n_out,
                                       int8_t* rows, float* scale, int32_t* rowsum, int8_t* q4n,
-                                      int8_t* q8n, float* s4, float* s8, cudaStream_t stream) {
+                                      int8_t* q8n, float* s4, float* s8, cudaStream_t stream,
+                                      void* zero = nullptr, size_t zero_bytes = 0) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)M);
   cfg.blockDim = dim3(kA48Threads);
@@ -314,8 +322,9 @@ bitnet_status bitnet_a48_quant_launch(const uint16_t* x, int64_t M, int64_t K, i
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, a48_quant_kernel, x, (int)K, (int)n_out, rows,
-                                           scale, rowsum, q4n, q8n, s4, s8);
+  const cudaError_t e =
+      cudaLaunchKernelEx(&cfg, a48_quant_kernel, x, (int)K, (int)n_out, rows, scale, rowsum, q4n,
+                         q8n, s4, s8, static_cast<uint4*>(zero), (int64_t)(zero_bytes / 16));
   return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
 

@@ -14,7 +14,8 @@ bitnet_status bitnet_pack_launch(const float* W, int64_t N, int64_t K, uint8_t* 
 bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* gain, int64_t M,
                                   int64_t K, int8_t* xq, int64_t ld_q, bool perm, float* scale,
                                   int32_t* rowsum, double* sumsq, int8_t* xq_natural,
-                                  cudaStream_t stream, const float* amax_in, float* amax_out);
+                                  cudaStream_t stream, const float* amax_in, float* amax_out,
+                                  void* zero, size_t zero_bytes);
 bitnet_status bitnet_decode_launch(const DecodeOp& op, int M, int num_sms, cudaStream_t stream);
 bool bitnet_resident_fits(int fmt, int64_t M, int64_t N, int64_t K, int num_sms);
 bool bitnet_resident_a48_fits(int64_t N, int64_t K, int num_sms);
@@ -33,7 +34,8 @@ bitnet_status bitnet_sign_to_i2s_launch(const uint8_t* sign, int64_t nbytes, uin
                                         int num_sms, cudaStream_t stream);
 bitnet_status bitnet_a48_quant_launch(const uint16_t* x, int64_t M, int64_t K, int64_t n_out,
                                       int8_t* rows, float* scale, int32_t* rowsum, int8_t* q4n,
-                                      int8_t* q8n, float* s4, float* s8, cudaStream_t stream);
+                                      int8_t* q8n, float* s4, float* s8, cudaStream_t stream,
+                                      void* zero, size_t zero_bytes);
 bitnet_status bitnet_a48_combine_launch(const int32_t* acc2, const float* scale,
                                         const float* gamma, int64_t M, int64_t N, uint16_t* y,
                                         float* y_f32, int32_t* acc4, int32_t* acc8, int num_sms,
@@ -423,8 +425,6 @@ bitnet_status linear_enqueue(const uint8_t* packed, const float* gamma, int64_t 
                                                           xq, sc, y, y_f32, acc);
     return cudaGetLastError() == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
   }
-  st = bitnet_quant_launch(x, false, nullptr, M, K, xq, K, true, sc, rs, nullptr, nullptr, s);
-  if (st != BITNET_OK) return st;
   const int bn = bitnet_gemm_pick_bn((int)M, (int)N, d.num_sms);
   GemmArgs a{};
   a.M = (int)M; a.N = (int)N; a.K = (int)K;
@@ -434,10 +434,13 @@ bitnet_status linear_enqueue(const uint8_t* packed, const float* gamma, int64_t 
   if (a.ksplit > 1) {
     a.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc);
     a.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc + splitk_acc_bytes(M, N));
-    if (cudaMemsetAsync(a.acc_ws0, 0, splitk_acc_bytes(M, N) + splitk_cnt_bytes(M, N), s) !=
-        cudaSuccess)
-      return BITNET_ERR_CUDA;
   }
+  // the quantiser also clears the split-K accumulators and tile counters
+  // (after its dependency wait; the GEMM adds into them only after its own)
+  st = bitnet_quant_launch(x, false, nullptr, M, K, xq, K, true, sc, rs, nullptr, nullptr, s,
+                           nullptr, nullptr, a.ksplit > 1 ? a.acc_ws0 : nullptr,
+                           a.ksplit > 1 ? splitk_acc_bytes(M, N) + splitk_cnt_bytes(M, N) : 0);
+  if (st != BITNET_OK) return st;
   return bitnet_gemm_launch(0 /*linear*/, xq, packed, nullptr, a, bn, d.num_sms, s);
 }
 
@@ -526,8 +529,6 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
   int32_t* rs2 = reinterpret_cast<int32_t*>(ws + L.rs2);
   double* ss2 = reinterpret_cast<double*>(ws + L.ss2);
   float* hbuf = dbg.h ? dbg.h : h;
-  st = bitnet_quant_launch(x, false, norm1_w, M, H, xq1, H, true, s1, rs1, ss1, dbg.xq1, s);
-  if (st != BITNET_OK) return st;
   // gate and up share the activation tile: keep it at the full 256 tokens
   const int bn = M > 128 ? 256 : bitnet_gemm_pick_bn((int)M, (int)I, d.num_sms);
   GemmArgs g{};
@@ -539,14 +540,13 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
     g.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
     g.acc_ws1 = reinterpret_cast<int32_t*>(ws + L.acc1);
     g.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc0 + splitk_acc_bytes(M, I));
-    if (cudaMemsetAsync(g.acc_ws0, 0, splitk_acc_bytes(M, I) + splitk_cnt_bytes(M, I), s) !=
-            cudaSuccess ||
-        cudaMemsetAsync(g.acc_ws1, 0, (size_t)M * I * 4, s) != cudaSuccess)
-      return BITNET_ERR_CUDA;
   }
-  st = bitnet_gemm_launch(1 /*glu*/, xq1, gate, up, g, bn, d.num_sms, s);
+  // each quantiser also clears the split-K scratch of the GEMM after it
+  st = bitnet_quant_launch(x, false, norm1_w, M, H, xq1, H, true, s1, rs1, ss1, dbg.xq1, s,
+                           nullptr, nullptr, g.ksplit > 1 ? ws + L.acc0 : nullptr,
+                           g.ksplit > 1 ? (L.acc1 - L.acc0) + al256((size_t)M * I * 4) : 0);
   if (st != BITNET_OK) return st;
-  st = bitnet_quant_launch(hbuf, true, norm2_w, M, I, xq2, I, true, s2, rs2, ss2, dbg.xq2, s);
+  st = bitnet_gemm_launch(1 /*glu*/, xq1, gate, up, g, bn, d.num_sms, s);
   if (st != BITNET_OK) return st;
   GemmArgs dn{};
   const int bn_d = bitnet_gemm_pick_bn((int)M, (int)H, d.num_sms);
@@ -558,10 +558,11 @@ bitnet_status bitnet_ffn(const uint16_t* x, int64_t M, int64_t H, int64_t I,
   if (dn.ksplit > 1) {
     dn.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
     dn.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc0 + splitk_acc_bytes(M, H));
-    if (cudaMemsetAsync(dn.acc_ws0, 0, splitk_acc_bytes(M, H) + splitk_cnt_bytes(M, H), s) !=
-        cudaSuccess)
-      return BITNET_ERR_CUDA;
   }
+  st = bitnet_quant_launch(hbuf, true, norm2_w, M, I, xq2, I, true, s2, rs2, ss2, dbg.xq2, s,
+                           nullptr, nullptr, dn.ksplit > 1 ? ws + L.acc0 : nullptr,
+                           dn.ksplit > 1 ? splitk_acc_bytes(M, H) + splitk_cnt_bytes(M, H) : 0);
+  if (st != BITNET_OK) return st;
   return bitnet_gemm_launch(2 /*down*/, xq2, down, nullptr, dn, bn_d, d.num_sms, s);
 }
 
@@ -738,7 +739,7 @@ bitnet_status bitnet_quant_act_a48(const uint16_t* x, int64_t M, int64_t K, int6
   bitnet_status st = device_info(&d);
   if (st != BITNET_OK) return st;
   return bitnet_a48_quant_launch(x, M, K, n_out, nullptr, nullptr, nullptr, q4, q8, s4, s8,
-                                 as_stream(stream));
+                                 as_stream(stream), nullptr, 0);
 }
 
 size_t bitnet_linear_a48_workspace_size(int64_t M, int64_t N, int64_t K) {
@@ -776,9 +777,6 @@ bitnet_status bitnet_linear_a48(const uint8_t* packed, const float* gamma, int64
   if (M == 1 && bitnet_resident_a48_fits(N, K, d.num_sms))
     return bitnet_resident_a48_launch(packed, gamma, (int)N, (int)K, x, (int)n_out, nullptr,
                                       nullptr, nullptr, y, y_f32, acc4, acc8, d.num_sms, s);
-  st = bitnet_a48_quant_launch(x, M, K, n_out, rows, sc, rs, nullptr, nullptr, nullptr, nullptr,
-                               s);
-  if (st != BITNET_OK) return st;
   // the integer products of all 2M code rows on the tensor-core kernel
   const int64_t M2 = 2 * M;
   const int bn = bitnet_gemm_pick_bn((int)M2, (int)N, d.num_sms);
@@ -791,10 +789,13 @@ bitnet_status bitnet_linear_a48(const uint8_t* packed, const float* gamma, int64
   if (a.ksplit > 1) {
     a.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc);
     a.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc + splitk_acc_bytes(M2, N));
-    if (cudaMemsetAsync(a.acc_ws0, 0, splitk_acc_bytes(M2, N) + splitk_cnt_bytes(M2, N), s) !=
-        cudaSuccess)
-      return BITNET_ERR_CUDA;
   }
+  // the quantiser also clears the GEMM's split-K scratch
+  st = bitnet_a48_quant_launch(x, M, K, n_out, rows, sc, rs, nullptr, nullptr, nullptr, nullptr,
+                               s, a.ksplit > 1 ? a.acc_ws0 : nullptr,
+                               a.ksplit > 1 ? splitk_acc_bytes(M2, N) + splitk_cnt_bytes(M2, N)
+                                            : 0);
+  if (st != BITNET_OK) return st;
   st = bitnet_gemm_launch(0 /*linear*/, rows, packed, nullptr, a, bn, d.num_sms, s);
   if (st != BITNET_OK) return st;
   return bitnet_a48_combine_launch(acc2, sc, gamma, M, N, y, y_f32, acc4, acc8, d.num_sms, s);
@@ -830,10 +831,6 @@ bitnet_status bitnet_ffn_tp_gate_up(const uint16_t* x, int64_t M, int64_t H, int
   int8_t* xq1 = reinterpret_cast<int8_t*>(ws + L.xq);
   float* s1 = reinterpret_cast<float*>(ws + L.s);
   int32_t* rs1 = reinterpret_cast<int32_t*>(ws + L.rs);
-  // every rank holds the whole token: the same codes on every shard
-  st = bitnet_quant_launch(x, false, norm1_w, M, H, xq1, H, true, s1, rs1, sumsq_x, nullptr, s,
-                           nullptr, nullptr);
-  if (st != BITNET_OK) return st;
   const int bn = M > 128 ? 256 : bitnet_gemm_pick_bn((int)M, (int)Ir, d.num_sms);
   GemmArgs g{};
   g.M = (int)M; g.N = (int)Ir; g.K = (int)H;
@@ -844,17 +841,19 @@ bitnet_status bitnet_ffn_tp_gate_up(const uint16_t* x, int64_t M, int64_t H, int
     g.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
     g.acc_ws1 = reinterpret_cast<int32_t*>(ws + L.acc1);
     g.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc0 + splitk_acc_bytes(M, Ir));
-    if (cudaMemsetAsync(g.acc_ws0, 0, splitk_acc_bytes(M, Ir) + splitk_cnt_bytes(M, Ir), s) !=
-            cudaSuccess ||
-        cudaMemsetAsync(g.acc_ws1, 0, (size_t)M * Ir * 4, s) != cudaSuccess)
-      return BITNET_ERR_CUDA;
   }
+  // every rank holds the whole token: the same codes on every shard (the
+  // quantiser also clears the GEMM's split-K scratch)
+  st = bitnet_quant_launch(x, false, norm1_w, M, H, xq1, H, true, s1, rs1, sumsq_x, nullptr, s,
+                           nullptr, nullptr, g.ksplit > 1 ? ws + L.acc0 : nullptr,
+                           g.ksplit > 1 ? (L.acc1 - L.acc0) + al256((size_t)M * Ir * 4) : 0);
+  if (st != BITNET_OK) return st;
   st = bitnet_gemm_launch(1 /*glu*/, xq1, gate, up, g, bn, d.num_sms, s);
   if (st != BITNET_OK) return st;
   // this shard's statistics of h' * n2: absmax and sum of squares of h'
   return bitnet_quant_launch(h, true, norm2_w, M, Ir, reinterpret_cast<int8_t*>(ws + L.xq2), Ir,
                              false, reinterpret_cast<float*>(ws + L.s2), nullptr, sumsq_h,
-                             nullptr, s, nullptr, amax2);
+                             nullptr, s, nullptr, amax2, nullptr, 0);
 }
 
 bitnet_status bitnet_ffn_tp_down(const float* h, int64_t M, int64_t H, int64_t Ir,
@@ -880,9 +879,6 @@ bitnet_status bitnet_ffn_tp_down(const float* h, int64_t M, int64_t H, int64_t I
   int32_t* rs2 = reinterpret_cast<int32_t*>(ws + L.rs);
   // the shard's h' * n2 quantised with the all-reduced absmax: the codes the
   // whole-block quantiser gives these features
-  st = bitnet_quant_launch(h, true, norm2_w, M, Ir, xq2, Ir, true, s2, rs2, nullptr, nullptr, s,
-                           amax2, nullptr);
-  if (st != BITNET_OK) return st;
   const int bn = bitnet_gemm_pick_bn((int)M, (int)H, d.num_sms);
   GemmArgs a{};
   a.M = (int)M; a.N = (int)H; a.K = (int)Ir;
@@ -893,10 +889,11 @@ bitnet_status bitnet_ffn_tp_down(const float* h, int64_t M, int64_t H, int64_t I
   if (a.ksplit > 1) {
     a.acc_ws0 = reinterpret_cast<int32_t*>(ws + L.acc0);
     a.tile_cnt = reinterpret_cast<int32_t*>(ws + L.acc0 + splitk_acc_bytes(M, H));
-    if (cudaMemsetAsync(a.acc_ws0, 0, splitk_acc_bytes(M, H) + splitk_cnt_bytes(M, H), s) !=
-        cudaSuccess)
-      return BITNET_ERR_CUDA;
   }
+  st = bitnet_quant_launch(h, true, norm2_w, M, Ir, xq2, Ir, true, s2, rs2, nullptr, nullptr, s,
+                           amax2, nullptr, a.ksplit > 1 ? ws + L.acc0 : nullptr,
+                           a.ksplit > 1 ? splitk_acc_bytes(M, H) + splitk_cnt_bytes(M, H) : 0);
+  if (st != BITNET_OK) return st;
   return bitnet_gemm_launch(0 /*linear*/, xq2, down, nullptr, a, bn, d.num_sms, s);
 }
 

@@ -26,7 +26,18 @@ struct QuantArgs {
   const float* amax_in;   // [M] or null: the absmax to quantise with (a tensor-
                           // parallel shard uses the all-reduced one)
   float* amax_out;        // [M] or null: this row's absmax of src * gain
+  uint4* zero;            // or null: a scratch range the grid clears after its
+  int64_t zero16;         // dependency wait (16-byte words), e.g. the split-K
+                          // accumulators of the kernel that follows
 };
+
+// Clear the scratch range, grid-stride over the whole launch.
+__device__ __forceinline__ void clear_scratch(const QuantArgs& a) {
+  if (!a.zero) return;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < a.zero16; i += stride)
+    a.zero[i] = make_uint4(0, 0, 0, 0);
+}
 
 // 8 consecutive source values as floats (one 16-byte load of bf16, two of fp32).
 template <bool kF32>
@@ -75,6 +86,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
   // the kernel that consumes the codes may start its own set-up (and its
   // weight loads) now; it reads the codes only after its dependency wait
   pdl_launch_dependents();
+  clear_scratch(a);
   if (m < a.M) {
     const int64_t K = a.K;
     const int64_t base = m * K;
@@ -190,6 +202,7 @@ __global__ void __launch_bounds__(256) quant_token_kernel(QuantArgs a) {
   const int64_t base = m * K;
   pdl_wait();
   pdl_launch_dependents();
+  clear_scratch(a);
   // pass 1: absmax of src * gain, sum of squares of src; groups of 8
   // (16-byte bf16 loads) when rows start 16-byte aligned, else of 4
   float amax = 0.f;
@@ -301,6 +314,7 @@ __global__ void __launch_bounds__(256) quant_token_cached_kernel(QuantArgs a) {
   const uint16_t* row = static_cast<const uint16_t*>(a.src) + m * K;
   pdl_wait();
   pdl_launch_dependents();
+  clear_scratch(a);
   uint4 v[kGroups][2];
 #pragma unroll
   for (int i = 0; i < kGroups; ++i) {
@@ -395,8 +409,13 @@ bitnet_status bitnet_quant_launch(const void* src, bool src_f32, const float* ga
                                   int64_t K, int8_t* xq, int64_t ld_q, bool perm, float* scale,
                                   int32_t* rowsum, double* sumsq, int8_t* xq_natural,
                                   cudaStream_t stream, const float* amax_in = nullptr,
-                                  float* amax_out = nullptr) {
-  QuantArgs a{src, gain, M, K, xq, ld_q, scale, rowsum, sumsq, xq_natural, amax_in, amax_out};
+                                  float* amax_out = nullptr, void* zero = nullptr,
+                                  size_t zero_bytes = 0) {
+  QuantArgs a{src,      gain,     M,
+              K,        xq,       ld_q,
+              scale,    rowsum,   sumsq,
+              xq_natural, amax_in, amax_out,
+              static_cast<uint4*>(zero), (int64_t)(zero_bytes / 16)};
   cudaLaunchConfig_t cfg = {};
   // a CTA per token for up to 256 tokens or rows longer than 4096 values;
   // else a warp per token (measured faster for many short rows)
