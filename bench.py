@@ -612,16 +612,20 @@ def run_ours(args, world, rank, local):
     traffic = profile_traffic("decode_resident_2b_m1.md")
 
     # --------------------------------------------------- e2e through the API
-    # per step: pinned host x -> device, one bitnet_linear_chain call through
-    # the binding (eager, no graph), device -> pinned host y
+    # per step: pinned host x -> device, one replay of the binding's prepared
+    # chain recorded as a CUDA graph (PreparedChain.capture: one launch for the
+    # 60 layers), device -> pinned host y
     xh = torch.from_numpy(x_host.view(np.int16)).pin_memory()
     yh = torch.empty((1, HIDDEN), dtype=torch.int16).pin_memory()
     xd = torch.empty((1, HIDDEN), dtype=torch.int16, device=dev)
     e2e_steps = max(5, min(args.steps, 200))
+    xd.copy_(xh)
+    replay = program.prep.capture(xd)
+    out = program.prep.ys[-1]
     with torch.cuda.stream(stream):
         for _ in range(3):
             xd.copy_(xh, non_blocking=True)
-            out = program(xd)
+            replay()
             yh.copy_(out.view(torch.int16), non_blocking=True)
         torch.cuda.synchronize()
         if barrier:
@@ -631,7 +635,7 @@ def run_ours(args, world, rank, local):
         e0.record(stream)
         for _ in range(e2e_steps):
             xd.copy_(xh, non_blocking=True)
-            out = program(xd)
+            replay()
             yh.copy_(out.view(torch.int16), non_blocking=True)
         e1.record(stream)
         e1.synchronize()
@@ -639,9 +643,9 @@ def run_ours(args, world, rank, local):
     e2e = {"value": weak_scaling_value(world, packed_bytes, e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
            "ms_per_step": e2e_ms,
-           "how": "pinned host x -> device, one eager bitnet_linear_chain call (60 layers) "
-                  "through the Python binding's prepared chain, device -> pinned host y; "
-                  "CUDA events"}
+           "how": "pinned host x -> device, one replay of the binding's prepared chain "
+                  "(60 layers) recorded as a CUDA graph by PreparedChain.capture, device -> "
+                  "pinned host y; CUDA events"}
 
     secondary = None
     if not args.no_secondary and rank == 0:

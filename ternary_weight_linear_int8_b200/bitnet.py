@@ -325,6 +325,27 @@ class PreparedChain:
         _check("bitnet_linear_chain", st)
         return self.ys[-1]
 
+    def capture(self, x: torch.Tensor):
+        """Record the chain on the input buffer x into a CUDA graph (one
+        eager call first, so that every kernel is loaded) and return a
+        function that replays it on the current stream: one launch for the
+        whole chain.  New inputs are written into x between replays; the
+        result is self.ys[-1].  The graph holds the buffers it was recorded
+        on (x, the outputs, the workspace)."""
+        if x.shape[0] != self.M or x.shape[1] != self.K0:
+            raise ValueError("x does not match the prepared chain")
+        side = torch.cuda.Stream(device=x.device)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self(x)
+        side.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            self(x)
+        self._graph = graph
+        self._graph_x = x
+        return graph.replay
+
 
 def bitnet_linear_noalloc(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, y=None):
     """BitLinear using the library's fixed device scratch array instead of a

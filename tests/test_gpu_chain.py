@@ -144,3 +144,24 @@ def test_chain_fullsize_2b_ping_pong_and_graph():
     torch.cuda.synchronize()
     assert np.array_equal(host_bits(bufs[1]), want[-1])
     assert np.array_equal(host_bits(bufs[0]), want[-2])
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_prepared_chain_graph_replay(M):
+    """PreparedChain.capture: the chain recorded once as a CUDA graph on a
+    fixed input buffer, replayed for two different inputs written into that
+    buffer; every replay's output equals the oracle's."""
+    dims = [512, 1024, 256, 768, 512]
+    rng = np.random.default_rng(70 + M)
+    Ws = [inputs.weights(dims[l + 1], dims[l], rng=rng) for l in range(len(dims) - 1)]
+    xs = [inputs.activations((M, dims[0]), rng=rng, outliers=True) for _ in range(2)]
+    packs = [B.bitnet_pack_weights(dev_f32(W)) for W in Ws]
+    ys = [torch.empty((M, W.shape[0]), dtype=torch.bfloat16, device="cuda") for W in Ws]
+    prog = B.PreparedChain([p for p, _ in packs], [g for _, g in packs], ys)
+    xd = dev_bits(xs[0]).clone()
+    replay = prog.capture(xd)
+    for x in xs * 2:
+        xd.copy_(dev_bits(x))
+        replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(host_bits(ys[-1]), _oracle_chain(Ws, x)[-1])
