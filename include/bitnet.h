@@ -254,7 +254,11 @@ BITNET_API bitnet_status bitnet_linear_chain(int64_t L, const uint8_t* const* pa
  *     nothing.
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress (once per device, with that device current); make
- *     that first call before capturing any stream.
+ *     that first call before capturing any stream.  With lazy module loading
+ *     (the CUDA default) the first launch of each kernel can load its code
+ *     as well, so before capturing make one call for every kind of shape
+ *     the capture will use (1-3 tokens, 4-8, 9-32, more tokens, K % 64 != 0:
+ *     they run different kernels).
  *   - All calls share the one array, which keeps the last call's contents;
  *     whatever must start at zero is cleared by the call itself.  Calls that
  *     may overlap on the GPU (other streams, other host threads) race on the
