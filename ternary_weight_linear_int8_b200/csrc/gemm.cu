@@ -59,15 +59,27 @@ constexpr int kGemmThreads = 448;        // 14 warps: TMA, MMA, 4 unpack, 8 epil
 
 template <int BN, int NMAT>
 struct GemmCfg {
+  // The unpacked weights are the MMA's A operand.  With one matrix and tiles
+  // of at most 192 tokens they live in tensor memory (the unpack warps write
+  // them with tcgen05.st, the MMA reads them from there), beside two
+  // accumulator sets: each stage then moves only the token tile and the
+  // packed weights through shared memory.  Otherwise they are staged in
+  // shared memory in the 128-byte-swizzled layout.
+  static constexpr bool kTS = NMAT == 1 && BN <= 192;
   static constexpr int kB = BN * kBK;                 // x_q tile bytes
-  static constexpr int kA = kBM * kBK;                // one unpacked weight tile
+  static constexpr int kA = kTS ? 0 : kBM * kBK;      // one unpacked weight tile (shared)
   static constexpr int kP = kBM * (kBK / 4);          // one packed weight tile
   static constexpr int kStage = kB + NMAT * (kA + kP);
-  static constexpr int kStages0 = (218 * 1024 - ((NMAT == 1) ? 32 * 128 * 2 : 0)) / kStage;
-  static constexpr int kStages = kStages0 > 6 ? 6 : (kStages0 < 2 ? 2 : kStages0);
   // accumulator sets in TMEM (512 columns): two when they fit
   static constexpr int kAcc = (2 * NMAT * BN <= 512) ? 2 : 1;
-  static constexpr int kCols0 = kAcc * NMAT * BN;
+  static constexpr int kStages0 = (218 * 1024 - ((NMAT == 1) ? 32 * 128 * 2 : 0)) / kStage;
+  static constexpr int kStagesSm = kStages0 > 6 ? 6 : (kStages0 < 2 ? 2 : kStages0);
+  // weight stages in TMEM: 32 columns each (128 int8 of K per lane)
+  static constexpr int kStagesTm = kTS ? (512 - kAcc * NMAT * BN) / 32 : kStagesSm;
+  static constexpr int kStages = kStagesSm < kStagesTm ? kStagesSm : kStagesTm;
+  static constexpr int kACol = kAcc * NMAT * BN;      // first weight-stage column (kTS)
+  static_assert(!kTS || (kStages >= 2 && kACol + 32 * kStages <= 512), "TMEM columns");
+  static constexpr int kCols0 = kTS ? 512 : kAcc * NMAT * BN;
   static constexpr int kTmemCols = kCols0 <= 32 ? 32 : kCols0 <= 64 ? 64 : kCols0 <= 128 ? 128
                                  : kCols0 <= 256 ? 256 : 512;
   static constexpr int kAux = 512;                    // barriers + tmem slot
@@ -107,6 +119,30 @@ __device__ __forceinline__ void tc_mma_i8(uint32_t dtmem, uint64_t adesc, uint64
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+// A (weights) from tensor memory at column a_tmem, B from shared memory.
+__device__ __forceinline__ void tc_mma_i8_ts(uint32_t dtmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(dtmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 consecutive columns of this warp's 32 TMEM lanes, one register each.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile(
@@ -312,14 +348,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           uint8_t* st = smem + (size_t)s * C::kStage;
           const uint64_t bdesc = sw128_desc(smem_u32(st));
+          if constexpr (C::kTS) {
+            // the stage's weights: 32 TMEM columns from kACol + 32 s, 8 per MMA
 #pragma unroll
-          for (int mat = 0; mat < NMAT; ++mat) {
-            const uint64_t adesc = sw128_desc(smem_u32(st + C::kB + mat * C::kA));
+            for (int q = 0; q < kBK / 32; ++q)
+              tc_mma_i8_ts(dt, tmem + (uint32_t)(C::kACol + 32 * s + 8 * q), bdesc + 2 * q,
+                           C::kIdesc, (kk > 0 || q > 0) ? 1u : 0u);
+          } else {
 #pragma unroll
-            for (int q = 0; q < kBK / 32; ++q) {
-              // advance 32 bytes of K inside the swizzle atom: +2 in 16-byte units
-              tc_mma_i8(dt + mat * BN, adesc + 2 * q, bdesc + 2 * q, C::kIdesc,
-                        (kk > 0 || q > 0) ? 1u : 0u);
+            for (int mat = 0; mat < NMAT; ++mat) {
+              const uint64_t adesc = sw128_desc(smem_u32(st + C::kB + mat * C::kA));
+#pragma unroll
+              for (int q = 0; q < kBK / 32; ++q) {
+                // advance 32 bytes of K inside the swizzle atom: +2 in 16-byte units
+                tc_mma_i8(dt + mat * BN, adesc + 2 * q, bdesc + 2 * q, C::kIdesc,
+                          (kk > 0 || q > 0) ? 1u : 0u);
+              }
             }
           }
           tc_commit(&mma_done[s]);
@@ -329,7 +373,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp < 6) {
     // ---------------------------------------------------- unpack warps
-    const int ut = tid - 64;                 // 0..127: one weight row each
+    // one weight row each; with the weights in TMEM, warp w writes lanes
+    // 32 (w % 4) .. + 31 (the lanes a warp may access), its rows
+    const int ut = C::kTS ? 32 * (warp & 3) + lane : tid - 64;
     int u = 0;
     bool ok = true;
     for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
@@ -339,24 +385,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int s = u % S;
         if (!mbar_wait(&tma_full[s], (u / S) & 1)) { ok = false; break; }
         uint8_t* st = smem + (size_t)s * C::kStage;
-#pragma unroll
-        for (int mat = 0; mat < NMAT; ++mat) {
-          const uint4* pk = reinterpret_cast<const uint4*>(st + C::kB + NMAT * C::kA +
-                                                           mat * C::kP + ut * (kBK / 4));
+        if constexpr (C::kTS) {
+          // the stage's previous MMA (which read these columns) has completed:
+          // its commit came before the producer refilled this stage
+          tc_fence_after();
+          const uint4* pk = reinterpret_cast<const uint4*>(st + C::kB + ut * (kBK / 4));
           const uint4 p0 = pk[0], p1 = pk[1];
           const uint32_t wv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-          uint8_t* arow = st + C::kB + mat * C::kA + ut * kBK;
+          uint32_t o[32];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const uint32_t w = wv[j];
-            const uint4 o = make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u,
-                                       (w >> 4) & 0x03030303u, (w >> 6) & 0x03030303u);
-            *reinterpret_cast<uint4*>(arow + ((j ^ (ut & 7)) << 4)) = o;
+            o[4 * j] = wv[j] & 0x03030303u;
+            o[4 * j + 1] = (wv[j] >> 2) & 0x03030303u;
+            o[4 * j + 2] = (wv[j] >> 4) & 0x03030303u;
+            o[4 * j + 3] = (wv[j] >> 6) & 0x03030303u;
           }
+          tmem_st32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(C::kACol + 32 * s),
+                    o);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[s]);
+        } else {
+#pragma unroll
+          for (int mat = 0; mat < NMAT; ++mat) {
+            const uint4* pk = reinterpret_cast<const uint4*>(st + C::kB + NMAT * C::kA +
+                                                             mat * C::kP + ut * (kBK / 4));
+            const uint4 p0 = pk[0], p1 = pk[1];
+            const uint32_t wv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            uint8_t* arow = st + C::kB + mat * C::kA + ut * kBK;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint32_t w = wv[j];
+              const uint4 o = make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u,
+                                         (w >> 4) & 0x03030303u, (w >> 6) & 0x03030303u);
+              *reinterpret_cast<uint4*>(arow + ((j ^ (ut & 7)) << 4)) = o;
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[s]);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[s]);
       }
     }
   } else {
