@@ -234,6 +234,42 @@ BITNET_API bitnet_status bitnet_linear_chain(int64_t L, const uint8_t* const* pa
                                              size_t workspace_bytes, void* stream);
 
 /*
+ * Several BitLinear layers applied to ONE input:
+ *   y[l] = BitLinear(packed[l], gamma[l])(x)   for l = 0 .. L-1,
+ * each identical, bit for bit, to what bitnet_linear computes for that
+ * matrix and x.  [A] section "モデル構造": the model keeps the LLaMA-style
+ * block (RMSNorm, SwiGLU, RoPE) with every nn.Linear a BitLinear, so the
+ * gate and up projections of the SwiGLU read the same input, and so do the
+ * query, key and value projections of the attention ([Y] section
+ * "BitAttentionとMGQA" passes one x as query, key and value).  The
+ * activation quantisation (per-token absmax, [Y] "Absmean量子化関数") does
+ * not depend on the matrix, so it is done once where bitnet_linear runs the
+ * tensor-core GEMM (K % 64 == 0 and more than 32 tokens, or fewer tokens on
+ * rows too long for the decode kernels): one quantiser launch writes the
+ * codes, then one GEMM per matrix reads them.  On the decode paths and for
+ * K % 64 != 0 the kernels quantise in their own prologues and the call is
+ * one bitnet_linear per matrix, in order.
+ *
+ * L        number of matrices, >= 1.
+ * packed, gamma, N, y   HOST arrays of L entries; packed[l], gamma[l] and
+ *          y[l] are device pointers.  Matrix l is [N[l], K] (all share K).
+ *          The arrays are read during the call only.
+ * x        [M, K] bf16 bits, device.   y[l]  [M, N[l]] bf16 bits, written.
+ * No output may overlap x or another output: BITNET_ERR_INVALID_ARG.
+ * workspace  >= bitnet_linear_multi_workspace_size(L, N, K, M) bytes,
+ *          device (0, and NULL allowed, when nothing is needed).
+ * Other requirements and errors as bitnet_linear, per matrix; everything is
+ * validated before anything is enqueued.
+ */
+BITNET_API size_t bitnet_linear_multi_workspace_size(int64_t L, const int64_t* N, int64_t K,
+                                                     int64_t M);
+BITNET_API bitnet_status bitnet_linear_multi(int64_t L, const uint8_t* const* packed,
+                                             const float* const* gamma, const int64_t* N,
+                                             int64_t K, const uint16_t* x, int64_t M,
+                                             uint16_t* const* y, void* workspace,
+                                             size_t workspace_bytes, void* stream);
+
+/*
  * BitLinear without a caller workspace, for callers that cannot allocate
  * device memory: code that issues work while a CUDA stream is being
  * captured into a graph (a cudaMalloc there is not part of the capture),

@@ -43,6 +43,8 @@ SIGNATURES = {
     "bitnet_linear_noalloc": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I64, _P, _P]),
     "bitnet_linear_chain_workspace_size": (_SZ, [_I64, _P, _P, _I64]),
     "bitnet_linear_chain": (ctypes.c_int, [_I64, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
+    "bitnet_linear_multi_workspace_size": (_SZ, [_I64, _P, _I64, _I64]),
+    "bitnet_linear_multi": (ctypes.c_int, [_I64, _P, _P, _P, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "bitnet_pack_w1_workspace_size": (_SZ, [_I64, _I64]),
     "bitnet_pack_weights_w1": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "bitnet_linear_w1_workspace_size": (_SZ, [_I64, _I64, _I64]),
@@ -290,6 +292,38 @@ def bitnet_linear_chain(packs, gammas, x: torch.Tensor, ys=None, workspace=None)
     ws = _workspace(nb, x.device, workspace)
     st = lib().bitnet_linear_chain(L, P, G, Ns, Ks, _ptr(x), M, Y, _ptr(ws), nb, _stream())
     _check("bitnet_linear_chain", st)
+    return ys
+
+
+def bitnet_linear_multi_workspace_size(Ns, K: int, M: int) -> int:
+    L = len(Ns)
+    n = (ctypes.c_int64 * L)(*Ns)
+    return lib().bitnet_linear_multi_workspace_size(L, n, K, M)
+
+
+def bitnet_linear_multi(packs, gammas, x: torch.Tensor, ys=None, workspace=None):
+    """Matrices l = 0..L-1 on one input: y[l] = BitLinear(packs[l], gammas[l])(x)
+    (e.g. query/key/value or gate/up projections).  All matrices share K;
+    `ys` (optional) are the output tensors, one per matrix, none overlapping
+    x or each other.  Returns ys."""
+    _bits16(x, "x")
+    if len(packs) != len(gammas) or not packs:
+        raise ValueError("packs and gammas must be non-empty lists of equal length")
+    M, K = x.shape
+    for p, g in zip(packs, gammas):
+        _dev(p, "packed")
+        _dev(g, "gamma")
+        if int(p.shape[1]) * 4 != K:
+            raise ValueError("every packed matrix must have K/4 columns")
+    if ys is None:
+        ys = [torch.empty((M, p.shape[0]), dtype=torch.bfloat16, device=x.device) for p in packs]
+    for y in ys:
+        _bits16(y, "y")
+    L, Ns, _, P, G, Y = _host_arrays(packs, gammas, ys, x)
+    nb = lib().bitnet_linear_multi_workspace_size(L, Ns, K, M)
+    ws = _workspace(nb, x.device, workspace)
+    st = lib().bitnet_linear_multi(L, P, G, Ns, K, _ptr(x), M, Y, _ptr(ws), nb, _stream())
+    _check("bitnet_linear_multi", st)
     return ys
 
 

@@ -655,6 +655,123 @@ bitnet_status bitnet_linear_chain(int64_t L, const uint8_t* const* packed,
   return BITNET_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Scratch of bitnet_linear_multi.  On the tensor-core path (shared codes):
+// the codes, scales and row sums of x once, then for tokens <= 256 one
+// split-K region (accumulators + tile counters) per matrix, all cleared by
+// the one quantiser launch.  Otherwise the largest matrix's bitnet_linear
+// scratch, reused by each call in turn.
+struct MultiWs {
+  bool shared;
+  size_t xq, scale, rowsum, acc, total;
+};
+
+MultiWs multi_ws_layout(int64_t L, const int64_t* N, int64_t K, int64_t M) {
+  MultiWs w{};
+  w.shared = linear_path(M, K) == kPathGemm && !batched_shape(M, K);
+  if (!w.shared) {
+    for (int64_t l = 0; l < L; ++l) {
+      const size_t b = linear_ws_layout(M, N[l], K).total;
+      if (b > w.total) w.total = b;
+    }
+    return w;
+  }
+  w.xq = 0;
+  w.scale = al256((size_t)M * K);
+  w.rowsum = w.scale + al256((size_t)M * 4);
+  w.acc = w.rowsum + al256((size_t)M * 4);
+  w.total = w.acc;
+  if (M <= 256)
+    for (int64_t l = 0; l < L; ++l) w.total += splitk_acc_bytes(M, N[l]) + splitk_cnt_bytes(M, N[l]);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bitnet_linear_multi_workspace_size(int64_t L, const int64_t* N, int64_t K, int64_t M) {
+  if (L < 1 || !N || M < 1 || K < 4) return 0;
+  for (int64_t l = 0; l < L; ++l)
+    if (N[l] < 1) return 0;
+  return multi_ws_layout(L, N, K, M).total;
+}
+
+bitnet_status bitnet_linear_multi(int64_t L, const uint8_t* const* packed,
+                                  const float* const* gamma, const int64_t* N, int64_t K,
+                                  const uint16_t* x, int64_t M, uint16_t* const* y,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (L < 1 || !packed || !gamma || !N || !x || !y) return BITNET_ERR_INVALID_ARG;
+  if (M < 1 || M > 0x7fffffff || K < 4 || K % 4 != 0 || K > 524288) return BITNET_ERR_SHAPE;
+  if (!aligned16(x)) return BITNET_ERR_ALIGN;
+  const uintptr_t in = reinterpret_cast<uintptr_t>(x);
+  const uintptr_t in_end = in + (uintptr_t)(M * K * 2);
+  for (int64_t l = 0; l < L; ++l) {
+    if (!packed[l] || !gamma[l] || !y[l]) return BITNET_ERR_INVALID_ARG;
+    if (N[l] < 1 || N[l] > 0x7fffffff) return BITNET_ERR_SHAPE;
+    if (!aligned16(packed[l]) || !aligned16(y[l]) || ((uintptr_t)gamma[l] & 3u))
+      return BITNET_ERR_ALIGN;
+    // no output may overlap the input (read by every matrix) or another output
+    const uintptr_t out = reinterpret_cast<uintptr_t>(y[l]);
+    const uintptr_t out_end = out + (uintptr_t)(M * N[l] * 2);
+    if (in < out_end && out < in_end) return BITNET_ERR_INVALID_ARG;
+    for (int64_t j = 0; j < l; ++j) {
+      const uintptr_t o2 = reinterpret_cast<uintptr_t>(y[j]);
+      const uintptr_t o2_end = o2 + (uintptr_t)(M * N[j] * 2);
+      if (o2 < out_end && out < o2_end) return BITNET_ERR_INVALID_ARG;
+    }
+  }
+  const MultiWs W = multi_ws_layout(L, N, K, M);
+  if (W.total > 0) {
+    if (!workspace || workspace_bytes < W.total) return BITNET_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BITNET_ERR_ALIGN;
+  }
+  DevInfo d;
+  bitnet_status st = device_info(&d);
+  if (st != BITNET_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  if (!W.shared) {
+    // decode and generic paths quantise inside their own kernels: one
+    // bitnet_linear per matrix, in order on the stream
+    for (int64_t l = 0; l < L; ++l) {
+      st = linear_enqueue(packed[l], gamma[l], N[l], K, x, M, y[l], nullptr, nullptr, workspace,
+                          linear_ws_layout(M, N[l], K), d, s);
+      if (st != BITNET_OK) return st;
+    }
+    return BITNET_OK;
+  }
+  // tensor-core path: one quantiser launch (which also clears every matrix's
+  // split-K region), then one GEMM per matrix on the shared codes
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + W.xq);
+  float* sc = reinterpret_cast<float*>(ws + W.scale);
+  int32_t* rs = reinterpret_cast<int32_t*>(ws + W.rowsum);
+  st = bitnet_quant_launch(x, false, nullptr, M, K, xq, K, true, sc, rs, nullptr, nullptr, s,
+                           nullptr, nullptr, W.total > W.acc ? ws + W.acc : nullptr,
+                           W.total - W.acc);
+  if (st != BITNET_OK) return st;
+  size_t acc_off = W.acc;
+  for (int64_t l = 0; l < L; ++l) {
+    const int bn = bitnet_gemm_pick_bn((int)M, (int)N[l], d.num_sms);
+    GemmArgs a{};
+    a.M = (int)M; a.N = (int)N[l]; a.K = (int)K;
+    a.ksplit = plan_ksplit(M, N[l], K, bn, d.num_sms);
+    a.scale = sc; a.rowsum = rs; a.gamma0 = gamma[l];
+    a.y = y[l];
+    if (a.ksplit > 1) {
+      a.acc_ws0 = reinterpret_cast<int32_t*>(ws + acc_off);
+      a.tile_cnt = reinterpret_cast<int32_t*>(ws + acc_off + splitk_acc_bytes(M, N[l]));
+    }
+    if (M <= 256) acc_off += splitk_acc_bytes(M, N[l]) + splitk_cnt_bytes(M, N[l]);
+    st = bitnet_gemm_launch(0 /*linear*/, xq, packed[l], nullptr, a, bn, d.num_sms, s);
+    if (st != BITNET_OK) return st;
+  }
+  return BITNET_OK;
+}
+
 size_t bitnet_pack_w1_workspace_size(int64_t N, int64_t K) {
   (void)N;
   (void)K;

@@ -153,3 +153,45 @@ def test_chain_workspace_and_validation(L):
     need = L.bitnet_linear_chain_workspace_size(2, I64(6912, 2560), I64(2560, 6912), 64)
     assert call(M=64, ws=FAKE, nb=need - 1) == 4
     assert call(M=64, ws=MIS, nb=need) == 3
+
+
+def test_multi_workspace_and_validation(L):
+    I64 = ctypes.c_int64 * 3
+    Ns = I64(2560, 512, 512)          # e.g. query, key and value projections
+    # decode-range token counts quantise inside their kernels: no scratch
+    assert L.bitnet_linear_multi_workspace_size(3, Ns, 2560, 1) == 0
+    # tensor-core path: the codes, scales and row sums once (plus split-K
+    # regions per matrix for <= 256 tokens), less than one scratch per matrix
+    big = L.bitnet_linear_multi_workspace_size(3, Ns, 2560, 4096)
+    assert 4096 * 2560 + 2 * 4096 * 4 <= big < 3 * L.bitnet_linear_workspace_size(4096, 2560, 2560)
+    mid = L.bitnet_linear_multi_workspace_size(3, Ns, 2560, 64)
+    assert mid >= 64 * 2560 + sum(64 * n * 4 for n in (2560, 512, 512))
+    # 9..32 tokens may run the batched decode kernel: the largest single scratch
+    assert L.bitnet_linear_multi_workspace_size(3, Ns, 2560, 16) == max(
+        L.bitnet_linear_workspace_size(16, n, 2560) for n in (2560, 512, 512))
+    assert L.bitnet_linear_multi_workspace_size(0, Ns, 2560, 1) == 0
+    y = [0x100000, 0x200000, 0x300000]
+    VP = ctypes.c_void_p * 3
+    P, G, Y = VP(FAKE, FAKE, FAKE), VP(FAKE, FAKE, FAKE), VP(*y)
+
+    def call(**kw):
+        a = dict(n=3, P=P, G=G, N=Ns, K=2560, x=FAKE, M=1, Y=Y, ws=None, nb=0)
+        a.update(kw)
+        return L.bitnet_linear_multi(a["n"], a["P"], a["G"], a["N"], a["K"], a["x"], a["M"],
+                                     a["Y"], a["ws"], a["nb"], None)
+
+    assert call(n=0) == 1
+    assert call(G=None) == 1
+    assert call(Y=VP(y[0], None, y[2])) == 1
+    assert call(M=0) == 2
+    assert call(K=2562) == 2
+    assert call(N=I64(2560, 0, 512)) == 2
+    assert call(x=MIS) == 3
+    assert call(Y=VP(y[0], MIS, y[2])) == 3
+    # an output overlapping the input, or another output
+    assert call(Y=VP(y[0], FAKE + 64, y[2])) == 1
+    assert call(Y=VP(y[0], y[0] + 16, y[2])) == 1
+    need = L.bitnet_linear_multi_workspace_size(3, Ns, 2560, 64)
+    assert call(M=64) == 4
+    assert call(M=64, ws=FAKE, nb=need - 1) == 4
+    assert call(M=64, ws=MIS, nb=need) == 3
