@@ -83,6 +83,7 @@ struct GemmCfg {
   static constexpr int kTmemCols = kCols0 <= 32 ? 32 : kCols0 <= 64 ? 64 : kCols0 <= 128 ? 128
                                  : kCols0 <= 256 ? 256 : 512;
   static constexpr int kAux = 512;                    // barriers + tmem slot
+  static_assert(8 * (4 * kStages + 2 * kAcc) + 4 <= kAux - 16, "barrier area");
   static constexpr int kTok = BN * 12;                // per-token scalars: d0, rowsum, d1-or-f
   // bf16 output staging for the TMA stores: 8 warps x 2 buffers x (8 tokens x 32 features)
   static constexpr int kStaging = (NMAT == 1) ? 32 * kBM * 2 : 0;
@@ -241,8 +242,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
   uint8_t* aux = smem + (size_t)S * C::kStage;
-  uint64_t* tma_full = reinterpret_cast<uint64_t*>(aux);
-  uint64_t* a_full = tma_full + S;
+  uint64_t* tma_full = reinterpret_cast<uint64_t*>(aux);   // the stage's token tile
+  uint64_t* w_full = tma_full + S;                         // the stage's packed weights
+  uint64_t* a_full = w_full + S;
   uint64_t* mma_done = a_full + S;
   uint64_t* acc_full = mma_done + S;         // [NACC]
   uint64_t* acc_empty = acc_full + NACC;     // [NACC]
@@ -275,6 +277,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&tma_full[s], 1);
+      mbar_init(&w_full[s], 1);
       mbar_init(&a_full[s], 4);
       mbar_init(&mma_done[s], 1);
     }
@@ -305,7 +308,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_normal();
       const uint64_t pol_x = policy_evict_last();
-      const uint32_t bytes = (uint32_t)(C::kB + NMAT * C::kP);
       bool waited = false;
       int u = 0;                               // running stage counter
       for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
@@ -316,13 +318,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (u >= S && !mbar_wait(&mma_done[s], ((u / S) - 1) & 1)) { u = -1; break; }
           uint8_t* st = smem + (size_t)s * C::kStage;
           const int kx = (k0 + kk) * kBK;
-          mbar_arrive_expect_tx(&tma_full[s], bytes);
-          // weights never depend on the previous kernel: load them first
-          tma_load_2d(st + C::kB + NMAT * C::kA, &tw0, &tma_full[s], kx / 4, nt * kBM, pol_w);
+          // weights never depend on the previous kernel: load them first, on
+          // their own barrier, so the unpack warps start while the token
+          // tile is still arriving
+          mbar_arrive_expect_tx(&w_full[s], (uint32_t)(NMAT * C::kP));
+          tma_load_2d(st + C::kB + NMAT * C::kA, &tw0, &w_full[s], kx / 4, nt * kBM, pol_w);
           if (NMAT == 2)
-            tma_load_2d(st + C::kB + NMAT * C::kA + C::kP, &tw1, &tma_full[s], kx / 4, nt * kBM,
+            tma_load_2d(st + C::kB + NMAT * C::kA + C::kP, &tw1, &w_full[s], kx / 4, nt * kBM,
                         pol_w);
           if (!waited) { pdl_wait(); waited = true; }
+          mbar_arrive_expect_tx(&tma_full[s], (uint32_t)C::kB);
           tma_load_2d(st, &tx, &tma_full[s], kx, mt * BN, pol_x);
         }
         if (u < 0) break;
@@ -383,7 +388,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       decode_unit(unit, nt, mt, k0, nk);
       for (int kk = 0; kk < nk; ++kk, ++u) {
         const int s = u % S;
-        if (!mbar_wait(&tma_full[s], (u / S) & 1)) { ok = false; break; }
+        if (!mbar_wait(&w_full[s], (u / S) & 1)) { ok = false; break; }
         uint8_t* st = smem + (size_t)s * C::kStage;
         if constexpr (C::kTS) {
           // the stage's previous MMA (which read these columns) has completed:

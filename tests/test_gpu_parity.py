@@ -119,7 +119,11 @@ def test_pack_nonfinite_is_reported():
 # few tokens or long rows: a CTA per token; many short rows: a warp per token
 QUANT_SHAPES = [(1, 2560, False), (8, 512, False), (3, 68, False), (17, 4, False),
                 (64, 6912, True), (5, 28672, True), (300, 1024, True), (600, 6912, True),
-                (297, 2560, False), (1000, 400, True), (260, 68, False)]
+                (297, 2560, False), (1000, 400, True), (260, 68, False),
+                # the persistent quantiser's edges: longest row it takes, one
+                # group of 16, a row one group past a whole warp, and many
+                # short rows per CTA
+                (2000, 8192, True), (40, 16, False), (33, 1040, True), (6000, 400, False)]
 
 
 @pytest.mark.parametrize("M,K,outl", QUANT_SHAPES)
