@@ -171,15 +171,23 @@ __global__ void __launch_bounds__(kBThreads, 2)
   // handed over) are in flight together
   const uint32_t x_addr = smem_u32(xq);
   const int npk = ks >> 3, nit = M * npk;
+  // (token, pack) of item i: one division per thread up front, then each
+  // step of kBThreads items is an addition with a carry
+  const int dm = kBThreads / npk, dpi = kBThreads - dm * npk;
+  auto advance = [&](int& m, int& pi) {
+    pi += dpi;
+    m += dm;
+    if (pi >= npk) { pi -= npk; ++m; }
+  };
+  int bm = tid / npk, bpi = tid - bm * npk;    // item of the batch's first step
   uint4 v[XB];
   auto load_batch = [&](int i0) {
+    int m = bm, pi = bpi;
 #pragma unroll
     for (int b = 0; b < XB; ++b) {
-      const int i = i0 + b * kBThreads;
-      if (i < nit) {
-        const int m = i / npk, pi = i - m * npk;
+      if (i0 + b * kBThreads < nit)
         v[b] = *reinterpret_cast<const uint4*>(p.x + (int64_t)m * K + k0 + 8 * pi);
-      }
+      advance(m, pi);
     }
   };
   load_batch(tid);
@@ -192,11 +200,11 @@ __global__ void __launch_bounds__(kBThreads, 2)
   __syncthreads();
   for (int i0 = tid; i0 < nit; i0 += XB * kBThreads) {
     if (i0 != tid) load_batch(i0);
+    int m = bm, pi = bpi;
 #pragma unroll
-    for (int b = 0; b < XB; ++b) {
+    for (int b = 0; b < XB; ++b, advance(m, pi)) {
       const int i = i0 + b * kBThreads;
       if (i < nit) {
-        const int m = i / npk, pi = i - m * npk;
         const float sc = s_sc[m];
         const uint32_t w[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
         int q[8];
@@ -214,6 +222,8 @@ __global__ void __launch_bounds__(kBThreads, 2)
           sts_u16(base + 4 * c, (uint16_t)__byte_perm((uint32_t)q[c], (uint32_t)q[4 + c], 0x0040));
       }
     }
+    bm = m;      // XB steps on: the next batch's first item
+    bpi = pi;
   }
   __syncthreads();
 
