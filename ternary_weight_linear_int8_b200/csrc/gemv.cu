@@ -245,7 +245,8 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
   int n0, n1;
   op_rows(a, n0, n1);
   const int nchunks = (n1 - n0 + RS - 1) / RS;
-  int gc = 0;   // stages consumed
+  int gs = 0;            // ring stage of the current chunk
+  uint32_t gph = 0;      // its phase parity
 
   // -------------------------------------------------------------- prologue
   // gamma loads go out with the activation loads (their latencies overlap)
@@ -470,8 +471,10 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
     }
   };
   int base = 0;   // the warp that takes item 0 of the current stage
-  for (int c = 0; c < nchunks; ++c, ++gc) {
-    const int s = gc % S;
+  for (int c = 0; c < nchunks; ++c) {
+    const int s = gs;
+    const uint32_t ph = gph;
+    if (++gs == S) { gs = 0; gph ^= 1u; }
     const int r0 = n0 + c * RS;
     const int nr = min(RS, n1 - r0);
     const int nitems = ((nr + RB - 1) / RB) * WK;
@@ -481,7 +484,7 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
     // every warp waits for the stage's data before it releases the stage,
     // also with no item in it: an early release could count towards the
     // previous use of the stage, which slower warps may still be reading
-    if (ring_ok && !mbar_wait(&sm.full()[s], (gc / S) & 1)) ring_ok = false;
+    if (ring_ok && !mbar_wait(&sm.full()[s], ph)) ring_ok = false;
     if (first < nitems && ring_ok) {
       const uint32_t st_addr = smem_u32(sm.ring() + (size_t)s * sm.stage_bytes);
       int* acc = sm.acc_s() + s * acc_words;
@@ -502,7 +505,7 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
       const bool tok_ok = g < M;
       for (int it = first; it < nitems; it += kConsumerWarps) {
         const int b = it >> wk_log2, q = it & (WK - 1);
-        const int w0 = (q * nwin) / WK, w1 = ((q + 1) * nwin) / WK;
+        const int w0 = (q * nwin) >> wk_log2, w1 = ((q + 1) * nwin) >> wk_log2;
         uint32_t rowa[NMAT][2];
 #pragma unroll
         for (int mat = 0; mat < NMAT; ++mat)
@@ -593,7 +596,7 @@ __device__ __forceinline__ void run_op(const DecodeOp& a, const int M, const Dec
       } else {
       for (int it = first; it < nitems; it += kConsumerWarps) {
         const int b = it >> wk_log2, q = it & (WK - 1);
-        const int j0 = (q * Kw) / WK, j1 = ((q + 1) * Kw) / WK;
+        const int j0 = (q * Kw) >> wk_log2, j1 = ((q + 1) * Kw) >> wk_log2;
         uint32_t rowa[NR];             // shared-window byte address of each row
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
