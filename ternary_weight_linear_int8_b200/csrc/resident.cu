@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(kResThreads, FMT == kResTL2 ? 1 : 2)
   bool ok = true;
   int pc = 0;            // weight piece of the current block (blocks only grow)
   constexpr bool kTern = FMT == kResI2S || FMT == kResA48;   // I2_S codes, dp4a
-  constexpr int kUnroll = (MT == 1 && kTern) ? 4 : 2;
+  constexpr int kUnroll = (MT == 1 && kTern) ? 1 : 2;
   const int wkl = __ffs(WK) - 1;
   const int nitems = nblk * WK;
   for (int it = warp; it < nitems; it += kResWarps) {
