@@ -37,3 +37,15 @@ def test_traffic_only_for_the_current_kernel_sources(tmp_path, monkeypatch):
     assert bench.profile_traffic("q.md") is None
     assert bench.profile_traffic("missing.md") is None
 
+
+
+def test_committed_decode_profile_is_for_the_current_sources():
+    """The committed summary of the headline kernel was captured on the
+    sources in the tree, so the benchmark line carries its traffic figure
+    (an edit of the kernel without a new capture fails here)."""
+    bench = _bench()
+    t = bench.profile_traffic("decode_resident_2b_m1.md")
+    assert t is not None
+    # the capture read the packed weights about once: algorithmic bytes of a
+    # 2B layer (4,423,680 packed + 2 K + 2 N + 4) within 2 %
+    assert abs(t / 4442628.0 - 1.0) < 0.02
