@@ -31,6 +31,11 @@
  *     a non-finite weight) are recorded in a per-device status word that
  *     bitnet_last_device_status() reports.
  *   - Pointers to x, y, packed and the workspace must be 16-byte aligned.
+ *   - The library keeps small per-device host caches (SM count, kernel
+ *     shared-memory settings, occupancy, the no-alloc scratch address),
+ *     filled on first use and safe across host threads.  They belong to the
+ *     device's primary context: after cudaDeviceReset() (which destroys it)
+ *     reload the library before calling it again on that device.
  */
 #ifndef BITNET_B200_H_
 #define BITNET_B200_H_
