@@ -195,3 +195,22 @@ def test_multi_workspace_and_validation(L):
     assert call(M=64) == 4
     assert call(M=64, ws=FAKE, nb=need - 1) == 4
     assert call(M=64, ws=MIS, nb=need) == 3
+
+
+def test_binding_rejects_host_tensors_before_any_call():
+    """The Python binding only marshals: tensors that are not on a GPU are
+    refused before anything reaches the library."""
+    import torch
+    x = torch.zeros((4, 64), dtype=torch.bfloat16)
+    p = torch.zeros((8, 16), dtype=torch.uint8)
+    g = torch.ones((1,), dtype=torch.float32)
+    for fn, args in ((B.bitnet_linear, (p, g, x)),
+                     (B.bitnet_linear_multi, ([p], [g], x)),
+                     (B.bitnet_linear_chain, ([p], [g], x)),
+                     (B.bitnet_quant_act, (x,))):
+        with pytest.raises(ValueError):
+            fn(*args)
+    with pytest.raises(ValueError):
+        B.bitnet_linear_multi([], [], x)
+    with pytest.raises(ValueError):
+        B.bitnet_linear_multi([p, p], [g], x)
